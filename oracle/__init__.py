@@ -1,0 +1,251 @@
+"""CPU oracle of the quantized recurrent-state decode step.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline / reference leg of ``bench.py`` may import this package.  The
+product path (``bit_recurrent_state_decode_b200``) never imports it and shares
+no code with it.
+
+The arithmetic lives in ``qstate_oracle.c`` (plain scalar C, fp32 with an
+explicit operation order, fp64 only for exact products); this module only
+builds it and marshals numpy arrays.  It follows "Preserving Updates in
+Low-Bit Recurrent State Quantization" (Table 1, Abstract, Figure 4, Table 6)
+and "When Dynamic Scaling Fails" (Abstract); the readings of the points those
+pages leave open are written next to the C code that implements them.
+
+Every oracle function is pinned in ``tests/test_oracle_*.py`` against closed
+forms, invariants, exhaustive enumeration or independent library routines.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import sys
+
+import numpy as np
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+SRC = os.path.join(HERE, "qstate_oracle.c")
+LIB = os.path.join(HERE, "liboracle.so")
+
+RETNET, MAMBA2, GLA, GDN = 0, 1, 2, 3
+DYNAMIC, PERSISTENT, YOKED = 0, 1, 2
+RTN, BDR = 0, 1
+NONE, LOST, MOVED, REVERSED = 0, 1, 2, 3
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (no fast-math, no FMA contraction)."""
+    if (not force and os.path.exists(LIB)
+            and os.path.getmtime(LIB) >= max(os.path.getmtime(SRC),
+                                             os.path.getmtime(SRC[:-2] + ".h"))):
+        return LIB
+    cmd = ["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math",
+           "-Wall", "-shared", "-fPIC", "-o", LIB + ".tmp", SRC, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(LIB + ".tmp", LIB)
+    return LIB
+
+
+class _Cfg(ctypes.Structure):
+    _fields_ = [("d_k", ctypes.c_int), ("d_v", ctypes.c_int), ("kind", ctypes.c_int),
+                ("group", ctypes.c_int), ("scale_mode", ctypes.c_int),
+                ("round_mode", ctypes.c_int), ("scale_f32", ctypes.c_int),
+                ("gamma", ctypes.c_float), ("eps_b", ctypes.c_float),
+                ("taxonomy", ctypes.c_int)]
+
+
+class Counts(ctypes.Structure):
+    _fields_ = [("nonfinite", ctypes.c_int64), ("saturated", ctypes.c_int64),
+                ("lost", ctypes.c_int64), ("moved", ctypes.c_int64),
+                ("reversed", ctypes.c_int64), ("bdr_applied", ctypes.c_int64)]
+
+    def as_dict(self):
+        return {n: int(getattr(self, n)) for n, _ in self._fields_}
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        _lib = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        _lib.or_f32_to_f16.restype = ctypes.c_uint16
+        _lib.or_f32_to_f16.argtypes = [ctypes.c_float]
+        _lib.or_f16_to_f32.restype = ctypes.c_float
+        _lib.or_f16_to_f32.argtypes = [ctypes.c_uint16]
+        _lib.or_bf16_to_f32.restype = ctypes.c_float
+        _lib.or_bf16_to_f32.argtypes = [ctypes.c_uint16]
+        _lib.or_f32_to_bf16.restype = ctypes.c_uint16
+        _lib.or_f32_to_bf16.argtypes = [ctypes.c_float]
+        _lib.or_tile_bytes.restype = ctypes.c_int64
+        _lib.or_tile_bytes.argtypes = [ctypes.c_int] * 3
+        _lib.or_pack.argtypes = [ctypes.c_int] * 3 + [P, P]
+        _lib.or_unpack.argtypes = [ctypes.c_int] * 3 + [P, P]
+        _lib.or_canon_dot.restype = ctypes.c_float
+        _lib.or_canon_dot.argtypes = [ctypes.c_int, P, ctypes.c_int, P]
+        _lib.or_round_rtn.restype = ctypes.c_int
+        _lib.or_round_rtn.argtypes = [ctypes.c_float, ctypes.c_float, ctypes.c_int]
+        _lib.or_round.restype = ctypes.c_int
+        _lib.or_round.argtypes = [ctypes.POINTER(_Cfg), ctypes.c_float, ctypes.c_float,
+                                  ctypes.c_float, ctypes.c_int, ctypes.POINTER(Counts)]
+        _lib.or_classify.restype = ctypes.c_int
+        _lib.or_classify.argtypes = [ctypes.c_float] * 3 + [ctypes.c_int]
+        _lib.or_step.restype = ctypes.c_int
+        _lib.or_step.argtypes = [ctypes.POINTER(_Cfg), ctypes.c_int64, P, P, P, P, P,
+                                 P, P, P, P, P, P, ctypes.POINTER(Counts)]
+        _lib.or_n_scales.restype = ctypes.c_int
+        _lib.or_n_scales.argtypes = [ctypes.POINTER(_Cfg)]
+        _lib.or_dequant.argtypes = [ctypes.POINTER(_Cfg), ctypes.c_int, P, P, P]
+    return _lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _f32(a):
+    return np.ascontiguousarray(a, dtype=np.float32)
+
+
+# ---------------------------------------------------------------- formats
+def f32_to_f16_bits(x: float) -> int:
+    return int(lib().or_f32_to_f16(float(x)))
+
+
+def f16_bits_to_f32(h: int) -> float:
+    return float(lib().or_f16_to_f32(int(h)))
+
+
+def bf16_bits_to_f32(h: int) -> float:
+    return float(lib().or_bf16_to_f32(int(h)))
+
+
+def f32_to_bf16_bits(x: float) -> int:
+    return int(lib().or_f32_to_bf16(float(x)))
+
+
+# ---------------------------------------------------------------- layout
+def tile_bytes(bits: int, d_k: int, d_v: int) -> int:
+    return int(lib().or_tile_bytes(bits, d_k, d_v))
+
+
+def pack(bits: int, codes: np.ndarray) -> np.ndarray:
+    """codes [..., d_k, d_v] int8 -> packed bytes [..., tile_bytes] uint8."""
+    codes = np.ascontiguousarray(codes, dtype=np.int8)
+    d_k, d_v = codes.shape[-2:]
+    lead = codes.shape[:-2]
+    flat = codes.reshape(-1, d_k, d_v)
+    nb = tile_bytes(bits, d_k, d_v)
+    out = np.zeros((flat.shape[0], nb), dtype=np.uint8)
+    for t in range(flat.shape[0]):
+        lib().or_pack(bits, d_k, d_v, _ptr(flat[t]), _ptr(out[t]))
+    return out.reshape(*lead, nb)
+
+
+def unpack(bits: int, d_k: int, d_v: int, data: np.ndarray) -> np.ndarray:
+    data = np.ascontiguousarray(data, dtype=np.uint8)
+    nb = tile_bytes(bits, d_k, d_v)
+    lead = data.shape[:-1]
+    flat = data.reshape(-1, nb)
+    out = np.zeros((flat.shape[0], d_k, d_v), dtype=np.int8)
+    for t in range(flat.shape[0]):
+        lib().or_unpack(bits, d_k, d_v, _ptr(flat[t]), _ptr(out[t]))
+    return out.reshape(*lead, d_k, d_v)
+
+
+def canon_dot(a: np.ndarray, b: np.ndarray) -> float:
+    """Canonical-order sum_i a[i] b[i] (blocks of 8 rows, pairwise tree)."""
+    a = _f32(a)
+    b = _f32(b)
+    return float(lib().or_canon_dot(len(a), _ptr(a), 1, _ptr(b)))
+
+
+def round_rtn(x: float, inv: float, qmax: int) -> int:
+    return int(lib().or_round_rtn(float(x), float(inv), int(qmax)))
+
+
+def classify(a: float, x: float, inv: float, qmax: int) -> int:
+    return int(lib().or_classify(float(a), float(x), float(inv), int(qmax)))
+
+
+class Config:
+    """Per-tile configuration of the oracle (mirrors the step's parameters)."""
+
+    def __init__(self, d_k, d_v, kind, group, scale_mode=DYNAMIC, round_mode=RTN,
+                 scale_f32=False, gamma=1.0 - 2.0 ** -5, eps_b=0.0, taxonomy=False):
+        self.c = _Cfg(d_k, d_v, kind, group, scale_mode, round_mode, int(bool(scale_f32)),
+                      gamma, eps_b, int(bool(taxonomy)))
+
+    def __getattr__(self, name):
+        return getattr(self.__dict__["c"], name)
+
+    @property
+    def n_scales(self) -> int:
+        return int(lib().or_n_scales(ctypes.byref(self.c)))
+
+    def round(self, a, x, inv, qmax, counts=None) -> int:
+        return int(lib().or_round(ctypes.byref(self.c), float(a), float(x), float(inv),
+                                  int(qmax), ctypes.byref(counts) if counts else None))
+
+
+class State:
+    """Unpacked oracle state of ``ntiles`` independent tiles.
+
+    codes  [T, d_k, d_v] int8   (quantized tiles)
+    S      [T, d_k, d_v] f32    (32-bit tiles)
+    scales [T, n_scales] f32    (stored scale values, exactly)
+    ref    [T, d_k, d_v] f32    (yoked reference state)
+    """
+
+    def __init__(self, cfg: Config, tile_bits):
+        self.cfg = cfg
+        self.tile_bits = np.ascontiguousarray(tile_bits, dtype=np.int32)
+        T = len(self.tile_bits)
+        dk, dv = cfg.d_k, cfg.d_v
+        self.codes = np.zeros((T, dk, dv), np.int8)
+        self.S = np.zeros((T, dk, dv), np.float32)
+        self.scales = np.zeros((T, cfg.n_scales), np.float32)
+        self.ref = np.zeros((T, dk, dv), np.float32) if cfg.scale_mode == YOKED else None
+        self.counts = Counts()
+
+    @property
+    def ntiles(self):
+        return len(self.tile_bits)
+
+    def step(self, q, k, v, alpha=None, beta=None):
+        cfg = self.cfg
+        T = self.ntiles
+        q, k, v = _f32(q).reshape(T, -1), _f32(k).reshape(T, -1), _f32(v).reshape(T, -1)
+        if alpha is not None:
+            alpha = _f32(alpha).reshape(T, -1)
+        if beta is not None:
+            beta = _f32(beta).reshape(T)
+        out = np.zeros((T, cfg.d_v), np.float32)
+        rc = lib().or_step(ctypes.byref(cfg.c), T, _ptr(self.tile_bits), _ptr(self.codes),
+                           _ptr(self.S), _ptr(self.scales), _ptr(self.ref), _ptr(q), _ptr(k),
+                           _ptr(v), _ptr(alpha), _ptr(beta), _ptr(out),
+                           ctypes.byref(self.counts))
+        if rc != 0:
+            raise ValueError("oracle rejected the configuration")
+        return out
+
+    def dequant(self) -> np.ndarray:
+        T = self.ntiles
+        out = np.zeros((T, self.cfg.d_k, self.cfg.d_v), np.float32)
+        for t in range(T):
+            if self.tile_bits[t] == 32:
+                out[t] = self.S[t]
+            else:
+                lib().or_dequant(ctypes.byref(self.cfg.c), int(self.tile_bits[t]),
+                                 _ptr(self.codes[t]), _ptr(self.scales[t]), _ptr(out[t]))
+        return out
+
+    def packed(self, t: int) -> np.ndarray:
+        return pack(int(self.tile_bits[t]), self.codes[t])
+
+
+if __name__ == "__main__":  # pragma: no cover
+    print(build(force="--force" in sys.argv))

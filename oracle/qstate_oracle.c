@@ -1,0 +1,432 @@
+/*
+ * qstate_oracle.c -- plain, slow, scalar CPU oracle of the quantized
+ * recurrent-state decode step.  TEST INFRASTRUCTURE ONLY (see the header):
+ * the product path never includes, links or runs this file.
+ *
+ * Build: gcc -O2 -std=c11 -ffp-contract=off -fno-fast-math -shared -fPIC -lm
+ * (no contraction of a*b+c, so every float operation below is one IEEE
+ * binary32 operation with round-to-nearest-even, except where fmaf is
+ * written out; double is used only where the text says "exact").
+ *
+ * The recurrence is "Preserving Updates in Low-Bit Recurrent State
+ * Quantization", Table 1; the scale modes are "When Dynamic Scaling Fails",
+ * Abstract; BDR and the lost / moved / reversed taxonomy are the Abstract
+ * and the Figure 4 caption of the first of these pages.  Everything the pages
+ * do not fix is a reading, marked "Reading:" below.
+ */
+#include "qstate_oracle.h"
+
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ------------------------------------------------------------------------
+ * Number formats.  Written from the IEEE 754 definitions: binary16 has an
+ * 11-bit significand, exponent bias 15, smallest normal 2^-14 and smallest
+ * subnormal 2^-24; bfloat16 is the top 16 bits of binary32.
+ * ---------------------------------------------------------------------- */
+uint16_t or_f32_to_f16(float x)
+{
+    uint32_t u;
+    memcpy(&u, &x, 4);
+    uint16_t sign = (uint16_t)((u >> 16) & 0x8000u);
+    if (isnan(x)) return (uint16_t)(sign | 0x7E00u);
+    double ax = fabs((double)x);              /* exact widening */
+    /* 65520 is the midpoint between 65504 (odd significand) and 2^16, so
+     * round-to-nearest-even sends it and everything above to infinity. */
+    if (ax >= 65520.0) return (uint16_t)(sign | 0x7C00u);
+    if (ax < 0x1p-14) {
+        /* subnormal range: units of 2^-24; nearbyint rounds half to even */
+        double n = nearbyint(ax * 0x1p24);    /* scaling by 2^24 is exact */
+        return (uint16_t)(sign | (uint16_t)n);  /* n == 1024 is the smallest normal */
+    }
+    int e;
+    (void)frexp(ax, &e);                      /* ax = f * 2^e, f in [0.5, 1) */
+    int E = e - 1;                            /* ax in [2^E, 2^(E+1)) */
+    double n = nearbyint(ldexp(ax, 10 - E));  /* significand in units of 2^(E-10) */
+    if (n == 2048.0) { n = 1024.0; E += 1; }
+    if (E + 15 >= 31) return (uint16_t)(sign | 0x7C00u);
+    return (uint16_t)(sign | (uint16_t)((E + 15) << 10) | (uint16_t)(n - 1024.0));
+}
+
+float or_f16_to_f32(uint16_t h)
+{
+    int s = (h >> 15) & 1, e = (h >> 10) & 0x1F, m = h & 0x3FF;
+    double v;
+    if (e == 0) v = ldexp((double)m, -24);
+    else if (e == 31) v = m ? NAN : INFINITY;
+    else v = ldexp((double)(1024 + m), e - 25);
+    return (float)(s ? -v : v);
+}
+
+float or_bf16_to_f32(uint16_t h)
+{
+    uint32_t u = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return f;
+}
+
+uint16_t or_f32_to_bf16(float x)
+{
+    uint32_t u;
+    memcpy(&u, &x, 4);
+    if (isnan(x)) return (uint16_t)((u >> 16) | 0x40u);
+    /* keep the top 16 bits, rounding the dropped 16 to nearest, ties to even */
+    uint32_t low = u & 0xFFFFu, top = u >> 16;
+    if (low > 0x8000u || (low == 0x8000u && (top & 1u))) top += 1;
+    return (uint16_t)top;
+}
+
+/* ------------------------------------------------------------------------
+ * Packed code layout of one d_k x d_v tile, row-major, packed along d_v.
+ * Reading (the pages give no layout): two's-complement codes;
+ *   8 bits: one byte per code;
+ *   4 bits: code 2m in the low nibble of byte m, code 2m+1 in the high one;
+ *   2 bits: code 4m+s in bits 2s..2s+1 of byte m;
+ *   6 bits: two planes, first the low 4 bits of every code in the 4-bit
+ *           layout (d_k*d_v/2 bytes), then the high 2 bits in the 2-bit
+ *           layout (d_k*d_v/4 bytes).
+ * ---------------------------------------------------------------------- */
+int64_t or_tile_bytes(int bits, int d_k, int d_v)
+{
+    return (int64_t)d_k * d_v * bits / 8;
+}
+
+static void put_field(uint8_t* row, int j, int w, unsigned v)
+{
+    int per = 8 / w;
+    row[j / per] |= (uint8_t)((v & ((1u << w) - 1u)) << (w * (j % per)));
+}
+
+static int get_field(const uint8_t* row, int j, int w)
+{
+    int per = 8 / w;
+    return (row[j / per] >> (w * (j % per))) & ((1 << w) - 1);
+}
+
+void or_pack(int bits, int d_k, int d_v, const int8_t* codes, uint8_t* out)
+{
+    memset(out, 0, (size_t)or_tile_bytes(bits, d_k, d_v));
+    for (int i = 0; i < d_k; i++) {
+        for (int j = 0; j < d_v; j++) {
+            int c = codes[(size_t)i * d_v + j];
+            if (bits == 8) {
+                out[(size_t)i * d_v + j] = (uint8_t)c;
+            } else if (bits == 4 || bits == 2) {
+                put_field(out + (size_t)i * d_v * bits / 8, j, bits, (unsigned)c);
+            } else if (bits == 6) {
+                uint8_t* lo = out + (size_t)i * d_v / 2;
+                uint8_t* hi = out + (size_t)d_k * d_v / 2 + (size_t)i * d_v / 4;
+                put_field(lo, j, 4, (unsigned)c & 15u);
+                put_field(hi, j, 2, ((unsigned)c >> 4) & 3u);
+            }
+        }
+    }
+}
+
+void or_unpack(int bits, int d_k, int d_v, const uint8_t* in, int8_t* codes)
+{
+    for (int i = 0; i < d_k; i++) {
+        for (int j = 0; j < d_v; j++) {
+            int u;
+            if (bits == 8) {
+                u = in[(size_t)i * d_v + j];
+            } else if (bits == 4 || bits == 2) {
+                u = get_field(in + (size_t)i * d_v * bits / 8, j, bits);
+            } else {
+                int lo = get_field(in + (size_t)i * d_v / 2, j, 4);
+                int hi = get_field(in + (size_t)d_k * d_v / 2 + (size_t)i * d_v / 4, j, 2);
+                u = (hi << 4) | lo;
+            }
+            if (u >= (1 << (bits - 1))) u -= (1 << bits);   /* sign-extend */
+            codes[(size_t)i * d_v + j] = (int8_t)u;
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------
+ * Canonical reduction order of the two sums over the key index,
+ *   r_j = sum_i (A S)_ij k_i   (GDN, Table 1)   and   o_j = sum_i S_ij q_i.
+ * Reading (the pages fix no order): the rows are cut into blocks of 8
+ * consecutive rows; each block is summed in ascending row order with a fused
+ * multiply-add starting from +0; the block sums are then added pairwise,
+ * adjacent blocks first, as a balanced binary tree.  n must be 8 times a
+ * power of two.
+ * ---------------------------------------------------------------------- */
+float or_canon_dot(int n, const float* a, int stride, const float* b)
+{
+    float part[64];
+    int nb = n / 8;
+    for (int blk = 0; blk < nb; blk++) {
+        float p = 0.0f;
+        for (int r = 0; r < 8; r++) {
+            int i = 8 * blk + r;
+            p = fmaf(a[(size_t)i * stride], b[i], p);
+        }
+        part[blk] = p;
+    }
+    while (nb > 1) {
+        for (int t = 0; t < nb / 2; t++) part[t] = part[2 * t] + part[2 * t + 1];
+        nb /= 2;
+    }
+    return part[0];
+}
+
+/* ------------------------------------------------------------------------
+ * Rounding.
+ * Reading: symmetric codes in [-Qmax, Qmax], Qmax = 2^(b-1) - 1; the scaled
+ * value is the exact product x * inv (exact in double: two 24-bit
+ * significands), rounded half to even, then clamped.  A NaN product clamps
+ * to -Qmax (the maxNum rule of fmax).
+ * ---------------------------------------------------------------------- */
+int or_round_rtn(float x, float inv, int qmax)
+{
+    double w = (double)x * (double)inv;
+    double r = nearbyint(w);
+    if (!(r >= -(double)qmax)) r = -(double)qmax;
+    if (r > (double)qmax) r = (double)qmax;
+    return (int)r;
+}
+
+/* BDR.  Reading of "rounds reversed elements toward their updates" with the
+ * threshold eps_B of Table 6: the update of the element is d = x - a (a is
+ * the decayed state before the update), u = a * inv is where the element
+ * sits on the new grid without the update.  The element is reversed when its
+ * RTN code lies on the far side of u from the update by more than eps_B grid
+ * steps, measured as s = fma(a, inv, -c_rtn); it is then moved one grid
+ * step toward its update (which is the nearest grid point on the update's
+ * side of x), and clamped. */
+int or_round(const or_cfg* c, float a, float x, float inv, int qmax, or_counts* cnt)
+{
+    int code = or_round_rtn(x, inv, qmax);
+    if (c->round_mode == OR_BDR) {
+        float d = x - a;
+        if (d != 0.0f) {
+            float s = fmaf(a, inv, -(float)code);
+            if (d > 0.0f && s > c->eps_b) {
+                code = code + 1 > qmax ? qmax : code + 1;
+                if (cnt) cnt->bdr_applied++;
+            } else if (d < 0.0f && s < -c->eps_b) {
+                code = code - 1 < -qmax ? -qmax : code - 1;
+                if (cnt) cnt->bdr_applied++;
+            }
+        }
+    }
+    return code;
+}
+
+/* Taxonomy of Figure 4 (left) under RTN, in grid units of the new scale.
+ * Reading: an element with update d = x - a != 0 is "reversed" when its RTN
+ * code lies strictly on the other side of u = a*inv from the update, "lost"
+ * otherwise when the code equals the RTN code of u (the update left no
+ * trace), and "moved" otherwise.  All comparisons are exact. */
+int or_classify(float a, float x, float inv, int qmax)
+{
+    float d = x - a;
+    if (!(d != 0.0f)) return OR_NONE;
+    int c = or_round_rtn(x, inv, qmax);
+    double u = (double)a * (double)inv;         /* exact */
+    double diff = (double)c - u;                /* sign exact */
+    if ((diff < 0.0 && d > 0.0f) || (diff > 0.0 && d < 0.0f)) return OR_REVERSED;
+    return c == or_round_rtn(a, inv, qmax) ? OR_LOST : OR_MOVED;
+}
+
+/* ------------------------------------------------------------------------
+ * Scale conversion to the stored precision.
+ * Reading: binary16 scales (4.50 bits per INT4 element at group 32, Table 2
+ * of "Preserving Updates ...") are rounded to nearest even; an overflow
+ * saturates to 65504 and is counted.  binary32 scales are kept as is.
+ * ---------------------------------------------------------------------- */
+static float to_stored_scale(const or_cfg* c, float v, or_counts* cnt)
+{
+    if (c->scale_f32) return v;
+    uint16_t h = or_f32_to_f16(v);
+    if ((h & 0x7FFFu) == 0x7C00u) {
+        h = (uint16_t)((h & 0x8000u) | 0x7BFFu);
+        if (cnt) cnt->saturated++;
+    }
+    return or_f16_to_f32(h);
+}
+
+int or_n_scales(const or_cfg* c)
+{
+    return c->group ? c->d_k * (c->d_v / c->group) : 1;
+}
+
+static int valid_cfg(const or_cfg* c)
+{
+    if (c->d_k < 8 || c->d_k > 512 || c->d_k % 8) return 0;
+    int nb = c->d_k / 8;
+    if (nb & (nb - 1)) return 0;
+    if (c->d_v < 8 || c->d_v % 8) return 0;
+    if (c->group < 0 || (c->group && c->d_v % c->group)) return 0;
+    if (c->kind < OR_RETNET || c->kind > OR_GDN) return 0;
+    if (c->scale_mode < OR_DYNAMIC || c->scale_mode > OR_YOKED) return 0;
+    if (c->round_mode < OR_RTN || c->round_mode > OR_BDR) return 0;
+    return 1;
+}
+
+static int finite_all(const float* p, int n)
+{
+    for (int i = 0; i < n; i++)
+        if (!isfinite(p[i])) return 0;
+    return 1;
+}
+
+/* One step of one tile.  The order of operations is the specification the
+ * CUDA kernels implement; each line is one rounded binary32 operation. */
+static void tile_step(const or_cfg* c, int bits, int8_t* codes, float* S, float* scales,
+                      float* ref, const float* q, const float* k, const float* v,
+                      const float* alpha, float beta, float* out, or_counts* cnt,
+                      float* a, float* x, float* aref, float* xref)
+{
+    const int dk = c->d_k, dv = c->d_v;
+    const int yoked = (c->scale_mode == OR_YOKED) && bits != 32;
+    const int qmax = bits == 32 ? 0 : (1 << (bits - 1)) - 1;
+    const int gs = c->group ? c->group : dv;             /* group width in columns */
+    const int ng = dv / gs;                                /* groups per row */
+
+    /* 1. decay, A_t S_{t-1} (Table 1, decay column).
+     * Reading: the dequantized state S_hat = code * scale is decayed as
+     * code * (alpha_i * scale), i.e. one product alpha_i * scale per group,
+     * then one product per element. */
+    for (int i = 0; i < dk; i++) {
+        float al = c->kind == OR_RETNET ? c->gamma
+                 : c->kind == OR_GLA    ? alpha[i] : alpha[0];
+        for (int j = 0; j < dv; j++) {
+            size_t e = (size_t)i * dv + j;
+            if (bits == 32) {
+                a[e] = S[e] * al;
+            } else {
+                float delta = c->group ? scales[i * ng + j / gs] : scales[0];
+                float eta = al * delta;
+                a[e] = (float)codes[e] * eta;
+            }
+            if (yoked) aref[e] = ref[e] * al;
+        }
+    }
+
+    /* 2. update B_t (Table 1, update column). */
+    if (c->kind == OR_GDN) {
+        for (int j = 0; j < dv; j++) {
+            float r = or_canon_dot(dk, a + j, dv, k);       /* ((A S)^T k)_j */
+            float e = v[j] - r;
+            float rr = 0.0f, er = 0.0f;
+            if (yoked) { rr = or_canon_dot(dk, aref + j, dv, k); er = v[j] - rr; }
+            for (int i = 0; i < dk; i++) {
+                size_t idx = (size_t)i * dv + j;
+                float kap = beta * k[i];
+                x[idx] = fmaf(kap, e, a[idx]);
+                if (yoked) xref[idx] = fmaf(kap, er, aref[idx]);
+            }
+        }
+    } else {
+        for (int i = 0; i < dk; i++)
+            for (int j = 0; j < dv; j++) {
+                size_t idx = (size_t)i * dv + j;
+                x[idx] = fmaf(k[i], v[j], a[idx]);
+                if (yoked) xref[idx] = fmaf(k[i], v[j], aref[idx]);
+            }
+    }
+
+    /* 3. output o_t = S_t^T q_t from the updated, not yet rounded state.
+     * Reading: the output is taken before the scale and rounding steps. */
+    for (int j = 0; j < dv; j++) out[j] = or_canon_dot(dk, x + j, dv, q);
+
+    if (bits == 32) {                     /* quantization disabled */
+        memcpy(S, x, sizeof(float) * (size_t)dk * dv);
+        return;
+    }
+
+    int bad = !finite_all(q, dk) || !finite_all(k, dk) || !finite_all(v, dv);
+    if (c->kind == OR_GLA) bad |= !finite_all(alpha, dk);
+    else if (c->kind != OR_RETNET) bad |= !isfinite(alpha[0]);
+    if (c->kind == OR_GDN) bad |= !isfinite(beta);
+
+    /* 4-6. scale and rounding, group by group (a group is gs consecutive
+     * columns of one row, or the whole tile for a per-token scale). */
+    const int ngroups = or_n_scales(c);
+    const float fq = (float)qmax;
+    for (int g = 0; g < ngroups; g++) {
+        int i0 = c->group ? g / ng : 0, i1 = c->group ? i0 + 1 : dk;
+        int j0 = c->group ? (g % ng) * gs : 0, j1 = c->group ? j0 + gs : dv;
+        float m = 0.0f, mref = 0.0f;
+        for (int i = i0; i < i1; i++)
+            for (int j = j0; j < j1; j++) {
+                m = fmaxf(m, fabsf(x[(size_t)i * dv + j]));
+                if (yoked) mref = fmaxf(mref, fabsf(xref[(size_t)i * dv + j]));
+            }
+        if (!isfinite(m) || (yoked && !isfinite(mref))) bad = 1;
+        float delta;
+        if (c->scale_mode == OR_DYNAMIC) {
+            /* re-derived from this step's state */
+            delta = to_stored_scale(c, m / fq, cnt);
+        } else if (c->scale_mode == OR_PERSISTENT) {
+            /* Reading: carried across steps and regrown only when the group
+             * maximum overflows the code range of the carried scale. */
+            float dp = scales[g];
+            delta = (m > fq * dp) ? to_stored_scale(c, m / fq, cnt) : dp;
+        } else {
+            /* yoked to the full-precision reference state of this step */
+            delta = to_stored_scale(c, mref / fq, cnt);
+        }
+        scales[g] = delta;
+        float inv = delta == 0.0f ? 0.0f : 1.0f / delta;
+        for (int i = i0; i < i1; i++)
+            for (int j = j0; j < j1; j++) {
+                size_t e = (size_t)i * dv + j;
+                if (cnt && c->taxonomy) {
+                    int cls = or_classify(a[e], x[e], inv, qmax);
+                    if (cls == OR_LOST) cnt->lost++;
+                    else if (cls == OR_MOVED) cnt->moved++;
+                    else if (cls == OR_REVERSED) cnt->reversed++;
+                }
+                codes[e] = (int8_t)or_round(c, a[e], x[e], inv, qmax, cnt);
+            }
+    }
+    if (yoked) memcpy(ref, xref, sizeof(float) * (size_t)dk * dv);
+    if (bad && cnt) cnt->nonfinite++;
+}
+
+int or_step(const or_cfg* c, int64_t ntiles, const int* tile_bits,
+            int8_t* codes, float* S, float* scales, float* ref,
+            const float* q, const float* k, const float* v,
+            const float* alpha, const float* beta, float* out, or_counts* cnt)
+{
+    if (!valid_cfg(c)) return -1;
+    const int dk = c->d_k, dv = c->d_v;
+    const size_t n = (size_t)dk * dv;
+    const int nsc = or_n_scales(c);
+    const int na = c->kind == OR_GLA ? dk : 1;
+    for (int64_t t = 0; t < ntiles; t++) {
+        int b = tile_bits[t];
+        if (!(b == 2 || b == 4 || b == 6 || b == 8 || b == 32)) return -1;
+        if (c->scale_mode == OR_YOKED && b != 32 && !ref) return -1;
+    }
+    float* buf = (float*)malloc(sizeof(float) * n * 4);
+    if (!buf) return -1;
+    for (int64_t t = 0; t < ntiles; t++) {
+        tile_step(c, tile_bits[t],
+                  codes ? codes + t * n : NULL, S ? S + t * n : NULL,
+                  scales ? scales + t * nsc : NULL, ref ? ref + t * n : NULL,
+                  q + t * dk, k + t * dk, v + t * dv,
+                  alpha ? alpha + t * na : NULL, beta ? beta[t] : 0.0f,
+                  out + t * dv, cnt, buf, buf + n, buf + 2 * n, buf + 3 * n);
+    }
+    free(buf);
+    return 0;
+}
+
+void or_dequant(const or_cfg* c, int bits, const int8_t* codes, const float* scales,
+                float* S_out)
+{
+    (void)bits;
+    const int dk = c->d_k, dv = c->d_v;
+    const int gs = c->group ? c->group : dv, ng = dv / gs;
+    for (int i = 0; i < dk; i++)
+        for (int j = 0; j < dv; j++) {
+            float delta = c->group ? scales[i * ng + j / gs] : scales[0];
+            S_out[(size_t)i * dv + j] = (float)codes[(size_t)i * dv + j] * delta;
+        }
+}
