@@ -1,0 +1,388 @@
+// qstate_api.cu -- the C ABI declared in include/qstate.h: argument
+// validation, device memory of a state object, kernel dispatch and the
+// host-buffer step.  All compute runs in the kernels of qstate_kernel.cuh.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "../../include/qstate.h"
+#include "qstate_dispatch.h"
+
+namespace qs {
+void launch_dequant_64_64(const StepParams&, float*, cudaStream_t);
+void launch_dequant_64_128(const StepParams&, float*, cudaStream_t);
+void launch_dequant_128_64(const StepParams&, float*, cudaStream_t);
+void launch_dequant_128_128(const StepParams&, float*, cudaStream_t);
+
+void launch_dequant(int dk, int dv, const StepParams& p, float* S, cudaStream_t st) {
+    if (dk == 64 && dv == 64) launch_dequant_64_64(p, S, st);
+    else if (dk == 64) launch_dequant_64_128(p, S, st);
+    else if (dv == 64) launch_dequant_128_64(p, S, st);
+    else launch_dequant_128_128(p, S, st);
+}
+}  // namespace qs
+
+struct qstate {
+    qstate_layout L;
+    int bits, group, scale_mode, round_mode;
+    float eps_b;
+    int device;
+    int64_t tiles, code_bytes, scale_bytes, ref_bytes, n_scales, n_gate;
+    int64_t tile_bytes, row_bytes;   // uniform tile bytes; bytes of one (layer, batch) row
+    int64_t in_size, gate_size, scale_size;
+    std::vector<uint8_t> head_bits;  // empty when uniform
+    uint8_t* d_codes = nullptr;
+    void* d_scales = nullptr;
+    float* d_ref = nullptr;
+    unsigned long long* d_counters = nullptr;
+    long long* d_head_off = nullptr;
+    unsigned char* d_head_bits = nullptr;
+    const qs::StepEntry* entry = nullptr;
+    int grid = 1;
+    // staging buffers of qstate_step_host (allocated by its first call)
+    void* st_q = nullptr;
+    void* st_k = nullptr;
+    void* st_v = nullptr;
+    void* st_g = nullptr;
+    float* st_out = nullptr;
+};
+
+namespace {
+
+int64_t tile_bytes_of(int bits, int dk, int dv) { return (int64_t)dk * dv * bits / 8; }
+
+bool valid_bits(int b) { return b == 2 || b == 4 || b == 6 || b == 8 || b == 32; }
+
+qs::StepParams params_of(const qstate* s) {
+    qs::StepParams p{};
+    p.codes = s->d_codes;
+    p.scales = s->d_scales;
+    p.ref = s->d_ref;
+    p.counters = s->d_counters;
+    p.head_off = s->d_head_off;
+    p.head_bits = s->d_head_bits;
+    p.row_bytes = s->row_bytes;
+    p.tile_bytes = s->tile_bytes;
+    p.ntiles = s->tiles;
+    p.heads = s->L.heads;
+    p.bits = s->bits;
+    p.group = s->group;
+    p.n_scales = (int)s->n_scales;
+    p.kind = s->L.kind;
+    p.scale_mode = s->scale_mode;
+    p.n_gate = (int)s->n_gate;
+    p.qkv_bf16 = s->L.qkv_dtype == QSTATE_BF16;
+    p.gate_bf16 = s->L.gate_dtype == QSTATE_BF16;
+    p.scale_f32 = s->L.scale_dtype == QSTATE_F32;
+    p.gamma = s->L.gamma;
+    p.eps_b = s->eps_b;
+    return p;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+void free_all(qstate* s) {
+    if (!s) return;
+    cudaFree(s->d_codes);
+    cudaFree(s->d_scales);
+    cudaFree(s->d_ref);
+    cudaFree(s->d_counters);
+    cudaFree(s->d_head_off);
+    cudaFree(s->d_head_bits);
+    cudaFree(s->st_q);
+    cudaFree(s->st_k);
+    cudaFree(s->st_v);
+    cudaFree(s->st_g);
+    cudaFree(s->st_out);
+}
+
+int zero_state(qstate* s, cudaStream_t st) {
+    if (s->code_bytes && cudaMemsetAsync(s->d_codes, 0, s->code_bytes, st) != cudaSuccess)
+        return QSTATE_ECUDA;
+    if (s->scale_bytes && cudaMemsetAsync(s->d_scales, 0, s->scale_bytes, st) != cudaSuccess)
+        return QSTATE_ECUDA;
+    if (s->ref_bytes && cudaMemsetAsync(s->d_ref, 0, s->ref_bytes, st) != cudaSuccess)
+        return QSTATE_ECUDA;
+    if (cudaMemsetAsync(s->d_counters, 0, 2 * sizeof(unsigned long long), st) != cudaSuccess)
+        return QSTATE_ECUDA;
+    return QSTATE_OK;
+}
+
+int check_device(const qstate* s) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return QSTATE_ECUDA;
+    return dev == s->device ? QSTATE_OK : QSTATE_EINVAL;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* qstate_error_string(int code) {
+    switch (code) {
+        case QSTATE_OK: return "ok";
+        case QSTATE_EINVAL: return "invalid argument";
+        case QSTATE_ENOMEM: return "out of memory";
+        case QSTATE_ECUDA: return "CUDA runtime error";
+        case QSTATE_EUNSUPPORTED: return "unsupported configuration";
+        default: return "unknown error";
+    }
+}
+
+int qstate_create(const qstate_layout* L, int bits, int group, qstate_scale_mode sm,
+                  qstate_round_mode rm, float eps_b, qstate** out) {
+    if (!L || !out) return QSTATE_EINVAL;
+    *out = nullptr;
+    if (L->batch < 0 || L->heads < 1 || L->layers < 1) return QSTATE_EINVAL;
+    if (L->d_k < 8 || L->d_v < 8 || L->d_k % 8 || L->d_v % 8) return QSTATE_EINVAL;
+    if (L->kind < QSTATE_RETNET || L->kind > QSTATE_GDN) return QSTATE_EINVAL;
+    if (L->qkv_dtype != QSTATE_F32 && L->qkv_dtype != QSTATE_BF16) return QSTATE_EINVAL;
+    if (L->gate_dtype != QSTATE_F32 && L->gate_dtype != QSTATE_BF16) return QSTATE_EINVAL;
+    if (L->scale_dtype != QSTATE_F16 && L->scale_dtype != QSTATE_F32) return QSTATE_EINVAL;
+    if (L->kind == QSTATE_RETNET && !std::isfinite(L->gamma)) return QSTATE_EINVAL;
+    if (sm < QSTATE_DYNAMIC || sm > QSTATE_YOKED) return QSTATE_EINVAL;
+    if (rm < QSTATE_RTN || rm > QSTATE_BDR) return QSTATE_EINVAL;
+    if (!(eps_b >= 0.0f) || !std::isfinite(eps_b)) return QSTATE_EINVAL;
+    if (group < 0 || (group && (group % 8 || L->d_v % group))) return QSTATE_EINVAL;
+    std::vector<uint8_t> hb;
+    if (L->head_bits) {
+        hb.assign(L->head_bits, L->head_bits + L->heads);
+        for (uint8_t b : hb)
+            if (!(b == 2 || b == 4 || b == 6 || b == 8)) return QSTATE_EINVAL;
+    } else if (!valid_bits(bits)) {
+        return QSTATE_EINVAL;
+    }
+    if (sm == QSTATE_YOKED && hb.empty() && bits == 32) return QSTATE_EINVAL;
+    if (!((L->d_k == 64 || L->d_k == 128) && (L->d_v == 64 || L->d_v == 128)))
+        return QSTATE_EUNSUPPORTED;
+
+    qstate* s = new (std::nothrow) qstate();
+    if (!s) return QSTATE_ENOMEM;
+    s->L = *L;
+    s->L.head_bits = nullptr;
+    s->bits = hb.empty() ? bits : 0;
+    s->group = group;
+    s->scale_mode = sm;
+    s->round_mode = rm;
+    s->eps_b = eps_b;
+    s->head_bits = hb;
+    if (cudaGetDevice(&s->device) != cudaSuccess) { delete s; return QSTATE_ECUDA; }
+
+    const int dk = L->d_k, dv = L->d_v;
+    s->tiles = (int64_t)L->layers * L->batch * L->heads;
+    s->n_scales = group ? (int64_t)dk * (dv / group) : 1;
+    s->n_gate = L->kind == QSTATE_RETNET ? 0 : L->kind == QSTATE_MAMBA2 ? 1
+              : L->kind == QSTATE_GLA ? dk : 2;
+    s->in_size = L->qkv_dtype == QSTATE_BF16 ? 2 : 4;
+    s->gate_size = L->gate_dtype == QSTATE_BF16 ? 2 : 4;
+    s->scale_size = L->scale_dtype == QSTATE_F32 ? 4 : 2;
+    std::vector<long long> head_off;
+    if (hb.empty()) {
+        s->tile_bytes = tile_bytes_of(bits, dk, dv);
+        s->row_bytes = s->tile_bytes * L->heads;
+    } else {
+        s->tile_bytes = 0;
+        long long off = 0;
+        for (uint8_t b : hb) { head_off.push_back(off); off += tile_bytes_of(b, dk, dv); }
+        s->row_bytes = off;
+    }
+    s->code_bytes = s->row_bytes * (int64_t)L->layers * L->batch;
+    const bool quantized = !hb.empty() || bits != 32;
+    s->scale_bytes = quantized ? s->tiles * s->n_scales * s->scale_size : 0;
+    s->ref_bytes = sm == QSTATE_YOKED ? s->tiles * dk * dv * 4 : 0;
+
+    auto alloc = [&](void** p, size_t n) -> bool {
+        if (!n) return true;
+        return cudaMalloc(p, n) == cudaSuccess;
+    };
+    bool ok = alloc((void**)&s->d_codes, s->code_bytes) &&
+              alloc(&s->d_scales, s->scale_bytes) &&
+              alloc((void**)&s->d_ref, s->ref_bytes) &&
+              alloc((void**)&s->d_counters, 2 * sizeof(unsigned long long));
+    if (ok && !hb.empty()) {
+        ok = alloc((void**)&s->d_head_off, head_off.size() * sizeof(long long)) &&
+             alloc((void**)&s->d_head_bits, hb.size()) &&
+             cudaMemcpy(s->d_head_off, head_off.data(), head_off.size() * sizeof(long long),
+                        cudaMemcpyHostToDevice) == cudaSuccess &&
+             cudaMemcpy(s->d_head_bits, hb.data(), hb.size(), cudaMemcpyHostToDevice) == cudaSuccess;
+    }
+    if (!ok) {
+        cudaGetLastError();
+        free_all(s);
+        delete s;
+        return QSTATE_ENOMEM;
+    }
+
+    const qs::StepEntry* tab = dk == 64 ? (dv == 64 ? qs::step_table_64_64() : qs::step_table_64_128())
+                                        : (dv == 64 ? qs::step_table_128_64() : qs::step_table_128_128());
+    s->entry = &tab[(L->kind == QSTATE_GDN) * 4 + (sm == QSTATE_YOKED) * 2 + (rm == QSTATE_BDR)];
+    int sms = 0;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, s->device);
+    int per_sm = s->entry->blocks_per_sm();
+    if (per_sm < 1) per_sm = 1;
+    long long g = (long long)sms * per_sm;
+    if (g < 1) g = 1;
+    if (s->tiles < g) g = s->tiles > 0 ? s->tiles : 1;
+    s->grid = (int)g;
+
+    int rc = zero_state(s, nullptr);
+    if (rc == QSTATE_OK && cudaDeviceSynchronize() != cudaSuccess) rc = QSTATE_ECUDA;
+    if (rc != QSTATE_OK) {
+        free_all(s);
+        delete s;
+        return rc;
+    }
+    *out = s;
+    return QSTATE_OK;
+}
+
+int qstate_destroy(qstate* s) {
+    if (!s) return QSTATE_EINVAL;
+    free_all(s);
+    delete s;
+    return QSTATE_OK;
+}
+
+int qstate_reset(qstate* s, qstate_stream stream) {
+    if (!s) return QSTATE_EINVAL;
+    return zero_state(s, (cudaStream_t)stream);
+}
+
+int qstate_step(qstate* s, const void* q, const void* k, const void* v, const void* gates,
+                float* out, qstate_stream stream) {
+    if (!s || !q || !k || !v || !out) return QSTATE_EINVAL;
+    if (s->n_gate && !gates) return QSTATE_EINVAL;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+        (gates && !aligned16(gates)))
+        return QSTATE_EINVAL;
+    if (s->tiles == 0) return QSTATE_OK;
+    int rc = check_device(s);
+    if (rc != QSTATE_OK) return rc;
+    qs::StepParams p = params_of(s);
+    p.q = q;
+    p.k = k;
+    p.v = v;
+    p.gates = gates;
+    p.out = out;
+    s->entry->launch(p, s->grid, (cudaStream_t)stream);
+    return cudaGetLastError() == cudaSuccess ? QSTATE_OK : QSTATE_ECUDA;
+}
+
+int qstate_get_sizes(const qstate* s, qstate_sizes* o) {
+    if (!s || !o) return QSTATE_EINVAL;
+    o->tiles = s->tiles;
+    o->code_bytes = s->code_bytes;
+    o->scale_bytes = s->scale_bytes;
+    o->ref_bytes = s->ref_bytes;
+    o->n_scales = s->n_scales;
+    o->n_gate = s->n_gate;
+    o->q_bytes = s->tiles * s->L.d_k * s->in_size;
+    o->v_bytes = s->tiles * s->L.d_v * s->in_size;
+    o->gate_bytes = s->tiles * s->n_gate * s->gate_size;
+    o->out_bytes = s->tiles * s->L.d_v * 4;
+    return QSTATE_OK;
+}
+
+int qstate_step_host(qstate* s, const void* q, const void* k, const void* v, const void* gates,
+                     float* out, qstate_stream stream) {
+    if (!s || !q || !k || !v || !out) return QSTATE_EINVAL;
+    if (s->n_gate && !gates) return QSTATE_EINVAL;
+    if (s->tiles == 0) return QSTATE_OK;
+    int rc = check_device(s);
+    if (rc != QSTATE_OK) return rc;
+    qstate_sizes z;
+    qstate_get_sizes(s, &z);
+    if (!s->st_q) {
+        bool ok = cudaMalloc(&s->st_q, z.q_bytes) == cudaSuccess &&
+                  cudaMalloc(&s->st_k, z.q_bytes) == cudaSuccess &&
+                  cudaMalloc(&s->st_v, z.v_bytes) == cudaSuccess &&
+                  (!z.gate_bytes || cudaMalloc(&s->st_g, z.gate_bytes) == cudaSuccess) &&
+                  cudaMalloc((void**)&s->st_out, z.out_bytes) == cudaSuccess;
+        if (!ok) {
+            cudaGetLastError();
+            cudaFree(s->st_q); cudaFree(s->st_k); cudaFree(s->st_v);
+            cudaFree(s->st_g); cudaFree(s->st_out);
+            s->st_q = s->st_k = s->st_v = s->st_g = nullptr;
+            s->st_out = nullptr;
+            return QSTATE_ENOMEM;
+        }
+    }
+    cudaStream_t st = (cudaStream_t)stream;
+    if (cudaMemcpyAsync(s->st_q, q, z.q_bytes, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaMemcpyAsync(s->st_k, k, z.q_bytes, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaMemcpyAsync(s->st_v, v, z.v_bytes, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        (z.gate_bytes &&
+         cudaMemcpyAsync(s->st_g, gates, z.gate_bytes, cudaMemcpyHostToDevice, st) != cudaSuccess))
+        return QSTATE_ECUDA;
+    rc = qstate_step(s, s->st_q, s->st_k, s->st_v, s->st_g, s->st_out, stream);
+    if (rc != QSTATE_OK) return rc;
+    if (cudaMemcpyAsync(out, s->st_out, z.out_bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return QSTATE_ECUDA;
+    return QSTATE_OK;
+}
+
+int qstate_dequant(const qstate* s, float* S_out, qstate_stream stream) {
+    if (!s || !S_out) return QSTATE_EINVAL;
+    if (s->tiles == 0) return QSTATE_OK;
+    int rc = check_device(s);
+    if (rc != QSTATE_OK) return rc;
+    qs::launch_dequant(s->L.d_k, s->L.d_v, params_of(s), S_out, (cudaStream_t)stream);
+    return cudaGetLastError() == cudaSuccess ? QSTATE_OK : QSTATE_ECUDA;
+}
+
+int qstate_export(const qstate* s, void* codes, void* scales, float* ref, qstate_stream stream) {
+    if (!s || !codes || (s->scale_bytes && !scales) || (s->ref_bytes && !ref)) return QSTATE_EINVAL;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (s->code_bytes &&
+        cudaMemcpyAsync(codes, s->d_codes, s->code_bytes, cudaMemcpyDefault, st) != cudaSuccess)
+        return QSTATE_ECUDA;
+    if (s->scale_bytes &&
+        cudaMemcpyAsync(scales, s->d_scales, s->scale_bytes, cudaMemcpyDefault, st) != cudaSuccess)
+        return QSTATE_ECUDA;
+    if (s->ref_bytes &&
+        cudaMemcpyAsync(ref, s->d_ref, s->ref_bytes, cudaMemcpyDefault, st) != cudaSuccess)
+        return QSTATE_ECUDA;
+    return QSTATE_OK;
+}
+
+int qstate_import(qstate* s, const void* codes, const void* scales, const float* ref,
+                  qstate_stream stream) {
+    if (!s || !codes || (s->scale_bytes && !scales) || (s->ref_bytes && !ref)) return QSTATE_EINVAL;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (s->code_bytes &&
+        cudaMemcpyAsync(s->d_codes, codes, s->code_bytes, cudaMemcpyDefault, st) != cudaSuccess)
+        return QSTATE_ECUDA;
+    if (s->scale_bytes &&
+        cudaMemcpyAsync(s->d_scales, scales, s->scale_bytes, cudaMemcpyDefault, st) != cudaSuccess)
+        return QSTATE_ECUDA;
+    if (s->ref_bytes &&
+        cudaMemcpyAsync(s->d_ref, ref, s->ref_bytes, cudaMemcpyDefault, st) != cudaSuccess)
+        return QSTATE_ECUDA;
+    return QSTATE_OK;
+}
+
+int64_t qstate_bytes_per_step(const qstate* s) {
+    if (!s) return -1;
+    const int64_t dk = s->L.d_k, dv = s->L.d_v;
+    int64_t b = 2 * s->code_bytes + 2 * s->scale_bytes + 2 * s->ref_bytes;
+    b += s->tiles * ((2 * dk + dv) * s->in_size + s->n_gate * s->gate_size + dv * 4);
+    return b;
+}
+
+int qstate_status(qstate* s, qstate_counters* o, qstate_stream stream) {
+    if (!s || !o) return QSTATE_EINVAL;
+    unsigned long long h[2] = {0, 0};
+    cudaStream_t st = (cudaStream_t)stream;
+    if (cudaMemcpyAsync(h, s->d_counters, sizeof(h), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess)
+        return QSTATE_ECUDA;
+    o->nonfinite = h[0];
+    o->saturated = h[1];
+    return QSTATE_OK;
+}
+
+}  // extern "C"

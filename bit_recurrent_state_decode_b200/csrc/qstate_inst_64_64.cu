@@ -1,0 +1,45 @@
+// Step kernels for d_k = 64, d_v = 64: every (GDN?, yoked?, BDR?) variant.
+#include "qstate_dispatch.h"
+
+namespace qs {
+namespace {
+
+template <bool GDN, bool YOKED, bool BDR>
+void launch(const StepParams& p, int grid, cudaStream_t st) {
+    step_kernel<64, 64, GDN, YOKED, BDR><<<grid, Geo<64, 64>::NT, 0, st>>>(p);
+}
+
+template <bool GDN, bool YOKED, bool BDR>
+int blocks_per_sm() {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+            &n, step_kernel<64, 64, GDN, YOKED, BDR>, Geo<64, 64>::NT, 0) != cudaSuccess)
+        return 0;
+    return n;
+}
+
+template <bool GDN, bool YOKED, bool BDR>
+constexpr StepEntry entry() {
+    return StepEntry{&launch<GDN, YOKED, BDR>, &blocks_per_sm<GDN, YOKED, BDR>, Geo<64, 64>::NT};
+}
+
+const StepEntry kTable[8] = {
+    entry<false, false, false>(), entry<false, false, true>(),
+    entry<false, true, false>(),  entry<false, true, true>(),
+    entry<true, false, false>(),  entry<true, false, true>(),
+    entry<true, true, false>(),   entry<true, true, true>(),
+};
+
+}  // namespace
+
+const StepEntry* step_table_64_64() { return kTable; }
+
+void launch_dequant_64_64(const StepParams& p, float* S, cudaStream_t st) {
+    const long long n = p.ntiles * 64 * (64 / 8);
+    long long blocks = (n + 255) / 256;
+    if (blocks > 65535LL * 8) blocks = 65535LL * 8;
+    if (blocks < 1) blocks = 1;
+    dequant_kernel<64, 64><<<(unsigned)blocks, 256, 0, st>>>(p, S);
+}
+
+}  // namespace qs

@@ -1,0 +1,230 @@
+"""Thin ctypes binding of the C ABI in include/qstate.h (libqstate.so).
+
+Argument marshalling only: every step of the decode path runs in the CUDA
+kernels of the library.  PyTorch supplies device memory (tensors whose
+``data_ptr()`` is passed) and streams (``torch.cuda.current_stream()``).
+The library must have been built (``python -m bit_recurrent_state_decode_b200.build``);
+loading fails loudly otherwise -- there is no CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libqstate.so")
+
+OK, EINVAL, ENOMEM, ECUDA, EUNSUPPORTED = 0, -1, -2, -3, -4
+RETNET, MAMBA2, GLA, GDN = 0, 1, 2, 3
+DYNAMIC, PERSISTENT, YOKED = 0, 1, 2
+RTN, BDR = 0, 1
+F32, BF16, F16 = 0, 1, 2
+
+# every symbol include/qstate.h declares
+EXPORTS = ("qstate_create", "qstate_destroy", "qstate_reset", "qstate_step", "qstate_step_host",
+           "qstate_dequant", "qstate_export", "qstate_import", "qstate_get_sizes",
+           "qstate_bytes_per_step", "qstate_status", "qstate_error_string")
+
+
+class QStateError(RuntimeError):
+    def __init__(self, fn, code):
+        super().__init__(f"{fn} failed: {code} ({error_string(code)})")
+        self.code = code
+
+
+class Layout(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("heads", ctypes.c_int32), ("d_k", ctypes.c_int32),
+                ("d_v", ctypes.c_int32), ("layers", ctypes.c_int32), ("kind", ctypes.c_int32),
+                ("gamma", ctypes.c_float), ("qkv_dtype", ctypes.c_int32),
+                ("gate_dtype", ctypes.c_int32), ("scale_dtype", ctypes.c_int32),
+                ("head_bits", ctypes.POINTER(ctypes.c_uint8))]
+
+
+class Counters(ctypes.Structure):
+    _fields_ = [("nonfinite", ctypes.c_uint64), ("saturated", ctypes.c_uint64)]
+
+
+class Sizes(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int64) for n in ("tiles", "code_bytes", "scale_bytes", "ref_bytes",
+                                              "n_scales", "n_gate", "q_bytes", "v_bytes",
+                                              "gate_bytes", "out_bytes")]
+
+
+_lib = None
+
+
+def lib():
+    """Load libqstate.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m bit_recurrent_state_decode_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p
+        L.qstate_create.argtypes = [ctypes.POINTER(Layout), I, I, I, I, ctypes.c_float,
+                                    ctypes.POINTER(P)]
+        L.qstate_destroy.argtypes = [P]
+        L.qstate_reset.argtypes = [P, S]
+        L.qstate_step.argtypes = [P, P, P, P, P, P, S]
+        L.qstate_step_host.argtypes = [P, P, P, P, P, P, S]
+        L.qstate_dequant.argtypes = [P, P, S]
+        L.qstate_export.argtypes = [P, P, P, P, S]
+        L.qstate_import.argtypes = [P, P, P, P, S]
+        L.qstate_get_sizes.argtypes = [P, ctypes.POINTER(Sizes)]
+        L.qstate_bytes_per_step.argtypes = [P]
+        L.qstate_bytes_per_step.restype = ctypes.c_int64
+        L.qstate_status.argtypes = [P, ctypes.POINTER(Counters), S]
+        L.qstate_error_string.argtypes = [I]
+        L.qstate_error_string.restype = ctypes.c_char_p
+        for name in EXPORTS:
+            if name not in ("qstate_bytes_per_step", "qstate_error_string"):
+                getattr(L, name).restype = I
+        _lib = L
+    return _lib
+
+
+def error_string(code: int) -> str:
+    return lib().qstate_error_string(int(code)).decode()
+
+
+def _check(fn, rc):
+    if rc != OK:
+        raise QStateError(fn, rc)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, torch.Tensor):
+        return ctypes.c_void_p(t.data_ptr())
+    return ctypes.c_void_p(t.ctypes.data)   # numpy array (host buffers)
+
+
+def _stream(stream=None):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+_TORCH_OF = {F32: torch.float32, BF16: torch.bfloat16, F16: torch.float16}
+
+
+class QState:
+    """A quantized recurrent state of layers x batch x heads tiles of d_k x d_v.
+
+    Mirrors ``qstate_create``; the object owns its device memory until
+    ``close()`` (also called on garbage collection)."""
+
+    def __init__(self, batch, heads, d_k, d_v, kind, bits=4, group=64, scale_mode=DYNAMIC,
+                 round_mode=RTN, eps_b=0.0, layers=1, gamma=1.0 - 2.0 ** -5, qkv_dtype=F32,
+                 gate_dtype=F32, scale_dtype=F16, head_bits=None):
+        self._h = None
+        self._hb = None
+        L = Layout(batch, heads, d_k, d_v, layers, kind, gamma, qkv_dtype, gate_dtype,
+                   scale_dtype, None)
+        if head_bits is not None:
+            self._hb = (ctypes.c_uint8 * heads)(*[int(b) for b in head_bits])
+            L.head_bits = ctypes.cast(self._hb, ctypes.POINTER(ctypes.c_uint8))
+        h = ctypes.c_void_p()
+        _check("qstate_create", lib().qstate_create(ctypes.byref(L), int(bits), int(group),
+                                                    int(scale_mode), int(round_mode),
+                                                    float(eps_b), ctypes.byref(h)))
+        self._h = h
+        self.batch, self.heads, self.d_k, self.d_v, self.layers = batch, heads, d_k, d_v, layers
+        self.kind, self.bits, self.group = kind, bits, group
+        self.scale_mode, self.round_mode, self.eps_b = scale_mode, round_mode, eps_b
+        self.qkv_dtype, self.gate_dtype, self.scale_dtype = qkv_dtype, gate_dtype, scale_dtype
+        self.head_bits = None if head_bits is None else [int(b) for b in head_bits]
+        z = Sizes()
+        _check("qstate_get_sizes", lib().qstate_get_sizes(self._h, ctypes.byref(z)))
+        self.sizes = {n: int(getattr(z, n)) for n, _ in Sizes._fields_}
+
+    # ------------------------------------------------------------ lifetime
+    def close(self):
+        if self._h is not None and _lib is not None:
+            lib().qstate_destroy(self._h)
+        self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    # ------------------------------------------------------------ properties
+    @property
+    def tiles(self) -> int:
+        return self.sizes["tiles"]
+
+    @property
+    def n_gate(self) -> int:
+        return self.sizes["n_gate"]
+
+    @property
+    def qkv_torch_dtype(self):
+        return _TORCH_OF[self.qkv_dtype]
+
+    @property
+    def gate_torch_dtype(self):
+        return _TORCH_OF[self.gate_dtype]
+
+    def bytes_per_step(self) -> int:
+        return int(lib().qstate_bytes_per_step(self._h))
+
+    # ------------------------------------------------------------ calls
+    def reset(self, stream=None):
+        _check("qstate_reset", lib().qstate_reset(self._h, _stream(stream)))
+
+    def step(self, q, k, v, gates, out, stream=None):
+        """One decode step; q, k, v, gates, out are CUDA tensors in the
+        layouts of include/qstate.h (gates None for RetNet)."""
+        _check("qstate_step", lib().qstate_step(self._h, _ptr(q), _ptr(k), _ptr(v), _ptr(gates),
+                                                _ptr(out), _stream(stream)))
+
+    def step_host(self, q, k, v, gates, out, stream=None):
+        """The same step from host buffers (pinned CPU tensors or numpy arrays)."""
+        _check("qstate_step_host", lib().qstate_step_host(self._h, _ptr(q), _ptr(k), _ptr(v),
+                                                          _ptr(gates), _ptr(out), _stream(stream)))
+
+    def dequant(self, out=None, stream=None) -> torch.Tensor:
+        if out is None:
+            out = torch.empty((self.tiles, self.d_k, self.d_v), dtype=torch.float32, device="cuda")
+        _check("qstate_dequant", lib().qstate_dequant(self._h, _ptr(out), _stream(stream)))
+        return out
+
+    def export(self, stream=None):
+        """(codes uint8, scales, ref) as new CUDA tensors."""
+        z = self.sizes
+        codes = torch.empty(z["code_bytes"], dtype=torch.uint8, device="cuda")
+        sdt = torch.float32 if self.scale_dtype == F32 else torch.float16
+        scales = torch.empty(z["scale_bytes"] // (4 if self.scale_dtype == F32 else 2),
+                             dtype=sdt, device="cuda")
+        ref = (torch.empty(z["ref_bytes"] // 4, dtype=torch.float32, device="cuda")
+               if z["ref_bytes"] else None)
+        _check("qstate_export", lib().qstate_export(self._h, _ptr(codes), _ptr(scales), _ptr(ref),
+                                                    _stream(stream)))
+        return codes, scales, ref
+
+    def import_(self, codes, scales, ref=None, stream=None):
+        _check("qstate_import", lib().qstate_import(self._h, _ptr(codes), _ptr(scales), _ptr(ref),
+                                                    _stream(stream)))
+
+    def status(self, stream=None) -> dict:
+        c = Counters()
+        _check("qstate_status", lib().qstate_status(self._h, ctypes.byref(c), _stream(stream)))
+        return {"nonfinite": int(c.nonfinite), "saturated": int(c.saturated)}
+
+    # ------------------------------------------------------------ helpers
+    def alloc_inputs(self, device="cuda"):
+        """Empty q, k, v, gates, out buffers in the step layouts."""
+        T = self.tiles
+        q = torch.empty((T, self.d_k), dtype=self.qkv_torch_dtype, device=device)
+        k = torch.empty_like(q)
+        v = torch.empty((T, self.d_v), dtype=self.qkv_torch_dtype, device=device)
+        g = (torch.empty((T, self.n_gate), dtype=self.gate_torch_dtype, device=device)
+             if self.n_gate else None)
+        out = torch.empty((T, self.d_v), dtype=torch.float32, device=device)
+        return q, k, v, g, out

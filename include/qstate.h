@@ -1,0 +1,193 @@
+/*
+ * qstate.h -- C ABI of the fused quantized recurrent-state decode step
+ * (sm_100a).  Library: bit_recurrent_state_decode_b200/libqstate.so.
+ *
+ * WHAT ONE STEP COMPUTES
+ * The state of one (layer, batch, head) tile is a d_k x d_v matrix S stored in
+ * low-bit codes with per-group scales.  One step, per tile:
+ *   1. unpack the codes and decay the state: a = A_t S_hat_{t-1}
+ *   2. add the update:                       x = a + B_t
+ *   3. emit the output:                      o_t = x^T q_t
+ *   4. re-derive or carry the scale, 5. round, 6. repack.
+ * The recurrence (decay A_t, update B_t) is Table 1 of "Preserving Updates in
+ * Low-Bit Recurrent State Quantization":
+ *   RetNet  A = gamma I,        B = k v^T
+ *   Mamba2  A = alpha_t I,      B = k v^T
+ *   GLA     A = Diag(alpha_t),  B = k v^T          (alpha over the d_k rows)
+ *   GDN     A = alpha_t I,      B = beta_t k (v - (A S_{t-1})^T k)^T
+ * The scale modes (dynamic: re-derived from the state every step;
+ * persistent: carried and regrown only on overflow; yoked: derived from a
+ * full-precision reference state stepped in lockstep) are the Abstract of
+ * "When Dynamic Scaling Fails".  Round-to-nearest and Bounded Directional
+ * Rounding (a reversed element is rounded toward its update) are the Abstract
+ * and Figure 4 of the first page; eps_B is its Table 6.  Per-token scales and
+ * mixed per-head bit widths are the Abstract of "Low-Bit Recurrent States in
+ * Hybrid Language Models".
+ *
+ * EXACT ARITHMETIC (binary32, round-to-nearest-even, in this order)
+ *   eta_i   = alpha_i * scale_prev(i, g)            one per (row, group)
+ *   a_ij    = code_ij * eta_i                        (32-bit state: S_ij * alpha_i)
+ *   rank-1:  x_ij = fma(k_i, v_j, a_ij)
+ *   GDN:     r_j = csum_i(a_ij k_i);  e_j = v_j - r_j;  kap_i = beta * k_i;
+ *            x_ij = fma(kap_i, e_j, a_ij)
+ *   o_j     = csum_i(x_ij q_i)                       (before rounding)
+ *   m       = max |x| over the group (a group is `group` consecutive columns
+ *             of one row, or the whole tile when group == 0)
+ *   dynamic:    scale = cvt(m / Qmax)
+ *   persistent: scale = (m > Qmax * scale_prev) ? cvt(m / Qmax) : scale_prev
+ *   yoked:      scale = cvt(m_ref / Qmax), m_ref from the reference state
+ *               stepped with the same arithmetic on 32-bit values
+ *   inv     = scale == 0 ? 0 : 1 / scale
+ *   RTN:     code = clamp(round_half_even(x * inv exact), -Qmax, Qmax)
+ *   BDR:     d = x - a; s = fma(a, inv, -code);  if d > 0 and s > eps_B:
+ *            code = min(code + 1, Qmax); if d < 0 and s < -eps_B:
+ *            code = max(code - 1, -Qmax)
+ * csum is the canonical order: rows in blocks of 8 consecutive rows, each
+ * block an ascending fma chain from +0, block sums added as a balanced
+ * pairwise tree (adjacent blocks first).  cvt is binary16 round-to-nearest-
+ * even (overflow saturates to 65504 and is counted) or the identity for
+ * binary32 scales.  Qmax = 2^(bits-1) - 1 (codes are symmetric; the code
+ * -2^(bits-1) is accepted on input).
+ *
+ * MEMORY LAYOUT (all device memory, row-major, tile = (layer, b, h),
+ * tile index t = (layer * batch + b) * heads + h)
+ *   q, k   [layers][batch][heads][d_k]   qkv_dtype (f32 or bf16)
+ *   v      [layers][batch][heads][d_v]   qkv_dtype
+ *   gates  [layers][batch][heads][n_gate] gate_dtype, n_gate = 0 (RetNet),
+ *          1 (Mamba2: alpha), d_k (GLA: alpha_i), 2 (GDN: alpha, beta)
+ *   out    [layers][batch][heads][d_v]   float32
+ *   codes (library-owned): per tile d_k*d_v*bits/8 bytes, two's complement,
+ *          packed along d_v: 8-bit one byte per code; 4-bit code 2m in the
+ *          low nibble of byte m; 2-bit code 4m+s in bits 2s..2s+1 of byte m;
+ *          6-bit a low-nibble plane (4-bit layout of code & 15) for the whole
+ *          tile followed by a high plane (2-bit layout of (code >> 4) & 3);
+ *          32-bit: the fp32 state itself.  Tiles are contiguous in tile order;
+ *          with per-head bit widths the tile (layer, b, h) starts at
+ *          (layer*batch + b) * sum_h(tile_bytes_h) + sum_{h'<h} tile_bytes_h'.
+ *   scales (library-owned): [tiles][d_k][d_v/group] (group > 0) or [tiles],
+ *          binary16 or binary32.
+ *   ref   (library-owned, yoked only): [tiles][d_k][d_v] float32.
+ * q, k, v, gates and out must be 16-byte aligned.
+ *
+ * ERRORS AND OWNERSHIP
+ * Every call returns QSTATE_OK (0) or a negative code; nothing throws across
+ * the ABI.  Invalid arguments are rejected before any CUDA call.  Kernels
+ * never trap: non-finite inputs and binary16 scale overflow are counted in
+ * sticky device counters read by qstate_status().  A qstate object owns its
+ * device memory; its calls are asynchronous on the stream passed and an
+ * object must not be stepped from two streams at once.  All pointers other
+ * than the object are borrowed for the duration of the call's device work.
+ */
+#ifndef QSTATE_H
+#define QSTATE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Compatible with cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st* qstate_stream;
+
+enum {
+    QSTATE_OK = 0,
+    QSTATE_EINVAL = -1,       /* invalid argument or layout */
+    QSTATE_ENOMEM = -2,       /* device or host allocation failed */
+    QSTATE_ECUDA = -3,        /* a CUDA runtime call failed */
+    QSTATE_EUNSUPPORTED = -4  /* valid but not built (e.g. d_k outside {64,128}) */
+};
+
+typedef enum { QSTATE_RETNET = 0, QSTATE_MAMBA2 = 1, QSTATE_GLA = 2, QSTATE_GDN = 3 } qstate_kind;
+typedef enum { QSTATE_DYNAMIC = 0, QSTATE_PERSISTENT = 1, QSTATE_YOKED = 2 } qstate_scale_mode;
+typedef enum { QSTATE_RTN = 0, QSTATE_BDR = 1 } qstate_round_mode;
+typedef enum { QSTATE_F32 = 0, QSTATE_BF16 = 1, QSTATE_F16 = 2 } qstate_dtype;
+
+typedef struct qstate_layout {
+    int32_t batch;            /* >= 0 (0: an empty object, steps are no-ops) */
+    int32_t heads;            /* >= 1 */
+    int32_t d_k, d_v;         /* each 64 or 128 */
+    int32_t layers;           /* independent layers held by the object, >= 1 */
+    int32_t kind;             /* qstate_kind */
+    float gamma;              /* RetNet decay (ignored for the other kinds) */
+    int32_t qkv_dtype;        /* QSTATE_F32 or QSTATE_BF16 */
+    int32_t gate_dtype;       /* QSTATE_F32 or QSTATE_BF16 */
+    int32_t scale_dtype;      /* QSTATE_F16 or QSTATE_F32 */
+    const uint8_t* head_bits; /* NULL, or host array [heads] of 2/4/6/8 (copied);
+                                 overrides `bits` of qstate_create */
+} qstate_layout;
+
+typedef struct qstate qstate;
+
+typedef struct qstate_counters {
+    uint64_t nonfinite;       /* tile-steps with a non-finite input or group max */
+    uint64_t saturated;       /* binary16 scale conversions that overflowed */
+} qstate_counters;
+
+typedef struct qstate_sizes {
+    int64_t tiles;            /* layers * batch * heads */
+    int64_t code_bytes;       /* packed codes (or fp32 state) of all tiles */
+    int64_t scale_bytes;      /* all scales */
+    int64_t ref_bytes;        /* yoked reference state (0 otherwise) */
+    int64_t n_scales;         /* scales per tile */
+    int64_t n_gate;           /* gate values per tile */
+    int64_t q_bytes, v_bytes, gate_bytes, out_bytes;  /* step operand sizes */
+} qstate_sizes;
+
+/* Create a zero state (codes, scales and reference all zero).
+ * bits: 2, 4, 6, 8, or 32 (quantization disabled, fp32 state); ignored when
+ *   L->head_bits is given.
+ * group: columns per scale group along d_v, a multiple of 8 dividing d_v, or
+ *   0 for one scale per tile per step (per-token).
+ * sm / rm / eps_b: scale mode, rounding mode, BDR threshold (>= 0, in grid
+ *   steps of the new scale).  YOKED needs bits < 32.
+ * On success *out owns the device memory; free it with qstate_destroy. */
+int qstate_create(const qstate_layout* L, int bits, int group, qstate_scale_mode sm,
+                  qstate_round_mode rm, float eps_b, qstate** out);
+int qstate_destroy(qstate* s);
+
+/* Zero the state again (asynchronous on stream). */
+int qstate_reset(qstate* s, qstate_stream stream);
+
+/* One decode step of every tile (one kernel launch), asynchronous on stream.
+ * q, k, v, gates, out: caller-owned DEVICE buffers in the layouts above
+ * (gates may be NULL for RetNet).  Returns after the launch. */
+int qstate_step(qstate* s, const void* q, const void* k, const void* v, const void* gates,
+                float* out, qstate_stream stream);
+
+/* The same step from HOST buffers: copies q, k, v, gates host->device into
+ * library-owned staging buffers, launches the step and copies out
+ * device->host, all asynchronous on stream (synchronise the stream before
+ * reading out).  Pinned host memory makes the copies asynchronous. */
+int qstate_step_host(qstate* s, const void* q, const void* k, const void* v,
+                     const void* gates, float* out, qstate_stream stream);
+
+/* Dequantized state S_hat = code * scale, float32 [tiles][d_k][d_v] (device). */
+int qstate_dequant(const qstate* s, float* S_out, qstate_stream stream);
+
+/* Copy the raw state out to / in from caller device buffers of
+ * qstate_sizes() bytes (codes, scales, ref; ref may be NULL if not yoked).
+ * Used for checkpoints and teacher-forced parity. */
+int qstate_export(const qstate* s, void* codes, void* scales, float* ref,
+                  qstate_stream stream);
+int qstate_import(qstate* s, const void* codes, const void* scales, const float* ref,
+                  qstate_stream stream);
+
+int qstate_get_sizes(const qstate* s, qstate_sizes* out);
+
+/* Algorithmic bytes one step must move: packed state read + write, scales
+ * read + write, q, k, v and gates read, out written, and in yoked mode the
+ * float32 reference state read + write.  Returns -1 on a NULL object. */
+int64_t qstate_bytes_per_step(const qstate* s);
+
+/* Read the sticky counters: copies them device->host on stream and
+ * synchronises that stream. */
+int qstate_status(qstate* s, qstate_counters* out, qstate_stream stream);
+
+/* Static, human-readable name of a return code. */
+const char* qstate_error_string(int code);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* QSTATE_H */

@@ -215,7 +215,10 @@ class State:
     def ntiles(self):
         return len(self.tile_bits)
 
-    def step(self, q, k, v, alpha=None, beta=None):
+    def step(self, q, k, v, alpha=None, beta=None, threads: int = 1):
+        """One step of every tile; ``threads`` > 1 splits the tiles over host
+        threads (the tiles are independent; each thread runs the same scalar
+        code on its own slice)."""
         cfg = self.cfg
         T = self.ntiles
         q, k, v = _f32(q).reshape(T, -1), _f32(k).reshape(T, -1), _f32(v).reshape(T, -1)
@@ -224,12 +227,32 @@ class State:
         if beta is not None:
             beta = _f32(beta).reshape(T)
         out = np.zeros((T, cfg.d_v), np.float32)
-        rc = lib().or_step(ctypes.byref(cfg.c), T, _ptr(self.tile_bits), _ptr(self.codes),
-                           _ptr(self.S), _ptr(self.scales), _ptr(self.ref), _ptr(q), _ptr(k),
-                           _ptr(v), _ptr(alpha), _ptr(beta), _ptr(out),
-                           ctypes.byref(self.counts))
-        if rc != 0:
-            raise ValueError("oracle rejected the configuration")
+
+        def run(lo, hi):
+            cnt = Counts()
+            sl = slice(lo, hi)
+            rc = lib().or_step(ctypes.byref(cfg.c), hi - lo, _ptr(self.tile_bits[sl]),
+                               _ptr(self.codes[sl]), _ptr(self.S[sl]), _ptr(self.scales[sl]),
+                               _ptr(None if self.ref is None else self.ref[sl]), _ptr(q[sl]),
+                               _ptr(k[sl]), _ptr(v[sl]),
+                               _ptr(None if alpha is None else alpha[sl]),
+                               _ptr(None if beta is None else beta[sl]), _ptr(out[sl]),
+                               ctypes.byref(cnt))
+            if rc != 0:
+                raise ValueError("oracle rejected the configuration")
+            return cnt
+
+        threads = max(1, min(int(threads), T))
+        if threads == 1:
+            parts = [run(0, T)]
+        else:
+            import concurrent.futures
+            bounds = np.linspace(0, T, threads + 1).astype(int)
+            with concurrent.futures.ThreadPoolExecutor(threads) as ex:
+                parts = list(ex.map(lambda i: run(bounds[i], bounds[i + 1]), range(threads)))
+        for c in parts:
+            for name, _ in Counts._fields_:
+                setattr(self.counts, name, getattr(self.counts, name) + getattr(c, name))
         return out
 
     def dequant(self) -> np.ndarray:

@@ -1,0 +1,198 @@
+"""Helpers of the GPU parity tests: run the CUDA path (through the C ABI) and
+the CPU oracle on the same seeded synthetic inputs and compare them.
+
+Bars (the decode-step contract):
+  - packed codes bit-exact, allowing at most 1e-5 of the codes to differ by
+    one level (a round-half tie flipped by a different fp32 FMA order);
+  - scales bit-exact;
+  - outputs and dequantized state within a max relative error of 1e-3 per
+    tile, measured as max|y - y_oracle| / max|y_oracle|.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+from bit_recurrent_state_decode_b200 import qstate as Q
+from bit_recurrent_state_decode_b200 import synth
+
+CODE_FLIP_FRACTION = 1e-5
+REL_TOL = 1e-3
+
+
+def to_device(x: np.ndarray | None, bf16: bool):
+    if x is None:
+        return None
+    if bf16:
+        return torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16).cuda()
+    return torch.from_numpy(np.ascontiguousarray(x, np.float32)).cuda()
+
+
+def gpu_object(wl: synth.Workload, mode: int, batch: int, layers: int) -> Q.QState:
+    hb = wl.head_bits()
+    return Q.QState(batch, wl.heads, wl.d_k, wl.d_v, wl.kind, bits=wl.bits or 4, group=wl.group,
+                    scale_mode=mode, round_mode=wl.round_mode, eps_b=wl.eps_b, layers=layers,
+                    gamma=wl.gamma, qkv_dtype=wl.qkv_dtype, gate_dtype=wl.gate_dtype,
+                    scale_dtype=wl.scale_dtype, head_bits=hb)
+
+
+def oracle_state(wl: synth.Workload, mode: int, tile_heads: np.ndarray, bits=None):
+    cfg = oracle.Config(wl.d_k, wl.d_v, wl.kind, wl.group, scale_mode=mode,
+                        round_mode=wl.round_mode, scale_f32=wl.scale_dtype == synth.F32,
+                        gamma=wl.gamma, eps_b=wl.eps_b)
+    hb = wl.head_bits()
+    if bits is None:
+        bits = wl.bits
+    tile_bits = hb[tile_heads] if hb is not None else np.full(len(tile_heads), bits)
+    return oracle.State(cfg, tile_bits)
+
+
+def oracle_inputs(wl, x: synth.StepInputs):
+    q, k, v, g = x.as_f32(wl)
+    alpha = beta = None
+    if wl.kind == synth.MAMBA2:
+        alpha = g
+    elif wl.kind == synth.GLA:
+        alpha = g
+    elif wl.kind == synth.GDN:
+        alpha, beta = g[:, :1], g[:, 1]
+    return q, k, v, alpha, beta
+
+
+def concat_inputs(parts):
+    def cat(name):
+        arrs = [getattr(p, name) for p in parts]
+        return None if arrs[0] is None else np.concatenate(arrs, axis=0)
+    return synth.StepInputs(cat("q"), cat("k"), cat("v"), cat("gates"))
+
+
+def gpu_inputs(wl, x: synth.StepInputs):
+    bf = wl.qkv_dtype == synth.BF16
+    gbf = wl.gate_dtype == synth.BF16
+    return (to_device(x.q, bf), to_device(x.k, bf), to_device(x.v, bf),
+            to_device(x.gates, gbf))
+
+
+class GpuView:
+    """Exported GPU state of one object, indexable per tile."""
+
+    def __init__(self, obj: Q.QState):
+        self.obj = obj
+        codes, scales, ref = obj.export()
+        torch.cuda.synchronize()
+        self.codes = codes.cpu().numpy()
+        self.scales = scales.float().cpu().numpy().reshape(obj.tiles, -1) if scales.numel() else None
+        self.ref = None if ref is None else ref.cpu().numpy().reshape(obj.tiles, obj.d_k, obj.d_v)
+        hb = obj.head_bits
+        self.tile_bits = ([hb[t % obj.heads] for t in range(obj.tiles)] if hb
+                          else [obj.bits] * obj.tiles)
+        tb = [oracle.tile_bytes(b, obj.d_k, obj.d_v) for b in (hb or [obj.bits] * obj.heads)]
+        self.head_off = np.concatenate([[0], np.cumsum(tb)[:-1]]).astype(np.int64)
+        self.row_bytes = int(np.sum(tb))
+
+    def tile_codes(self, t: int) -> np.ndarray:
+        o = self.obj
+        b = self.tile_bits[t]
+        nb = oracle.tile_bytes(b, o.d_k, o.d_v)
+        start = (t // o.heads) * self.row_bytes + int(self.head_off[t % o.heads])
+        raw = self.codes[start:start + nb]
+        if b == 32:
+            return raw.view(np.float32).reshape(o.d_k, o.d_v)
+        return oracle.unpack(b, o.d_k, o.d_v, raw)
+
+
+def rel_err(y, ref):
+    y = np.asarray(y, np.float64)
+    ref = np.asarray(ref, np.float64)
+    den = np.abs(ref).max()
+    num = np.abs(y - ref).max()
+    if den == 0:
+        return float(num)
+    return float(num / den)
+
+
+def compare(view: GpuView, out_gpu: np.ndarray, st: oracle.State, out_orc: np.ndarray,
+            gpu_tiles, orc_tiles, check_dequant=None):
+    """Compare sampled tiles; returns a stats dict and raises AssertionError on
+    a breach of the bars."""
+    n_codes = n_flip = n_big = 0
+    worst_out = 0.0
+    scale_mismatch = 0
+    for gt, ot in zip(gpu_tiles, orc_tiles):
+        b = int(st.tile_bits[ot])
+        got = view.tile_codes(gt)
+        if b == 32:
+            assert np.array_equal(got.view(np.uint32), st.S[ot].view(np.uint32)), \
+                f"fp32 state differs at tile {gt}"
+        else:
+            d = np.abs(got.astype(np.int32) - st.codes[ot].astype(np.int32))
+            n_codes += d.size
+            n_flip += int(np.count_nonzero(d))
+            n_big += int(np.count_nonzero(d > 1))
+            if view.scales is not None:
+                scale_mismatch += int(np.count_nonzero(view.scales[gt] != st.scales[ot]))
+            if view.ref is not None and st.ref is not None:
+                assert np.array_equal(view.ref[gt].view(np.uint32), st.ref[ot].view(np.uint32)), \
+                    f"yoked reference differs at tile {gt}"
+        worst_out = max(worst_out, rel_err(out_gpu[gt], out_orc[ot]))
+    stats = dict(codes=n_codes, flips=n_flip, big=n_big, scale_mismatch=scale_mismatch,
+                 out_rel=worst_out)
+    assert n_big == 0, stats
+    assert n_flip <= CODE_FLIP_FRACTION * max(n_codes, 1) + 0, stats
+    assert scale_mismatch == 0, stats
+    assert worst_out <= REL_TOL, stats
+    return stats
+
+
+def run_pair(wl: synth.Workload, modes=None, batch_sel=None, layers=1, steps=8, start_step=0,
+             check_every=1, teacher_forced=False):
+    """Step the GPU and the oracle side by side on batch rows ``batch_sel`` of
+    ``layers`` layers; compare every ``check_every`` steps.  Returns stats."""
+    modes = modes or wl.scale_modes
+    batch_sel = np.arange(wl.batch) if batch_sel is None else np.asarray(batch_sel)
+    H = wl.heads
+    B = len(batch_sel)
+    orig_tiles = (batch_sel[:, None] * H + np.arange(H)[None, :]).reshape(-1)
+    tile_heads = np.tile(np.arange(H), B * layers)
+    gpu = {m: gpu_object(wl, m, B, layers) for m in modes}
+    orc = {m: oracle_state(wl, m, tile_heads) for m in modes}
+    T = B * H * layers
+    all_stats = []
+    for step in range(start_step, start_step + steps):
+        x = concat_inputs([synth.gen_step(wl, step, layer=l, tiles=orig_tiles)
+                           for l in range(layers)])
+        qd, kd, vd, gd = gpu_inputs(wl, x)
+        oq, ok_, ov, oa, ob = oracle_inputs(wl, x)
+        for m in modes:
+            if teacher_forced:
+                import_oracle_state(gpu[m], orc[m])
+            out = torch.empty((T, wl.d_v), dtype=torch.float32, device="cuda")
+            gpu[m].step(qd, kd, vd, gd, out)
+            o_orc = orc[m].step(oq, ok_, ov, oa, ob)
+            if (step - start_step + 1) % check_every == 0 or step == start_step + steps - 1:
+                view = GpuView(gpu[m])
+                s = compare(view, out.cpu().numpy(), orc[m], o_orc, range(T), range(T))
+                s.update(step=step, mode=m)
+                all_stats.append(s)
+    status = {m: gpu[m].status() for m in modes}
+    for m in modes:
+        gpu[m].close()
+    return all_stats, status, {m: orc[m].counts.as_dict() for m in modes}
+
+
+def import_oracle_state(obj: Q.QState, st: oracle.State):
+    """Pack the oracle state into the GPU layout and import it."""
+    view_bits = [obj.head_bits[t % obj.heads] for t in range(obj.tiles)] if obj.head_bits \
+        else [obj.bits] * obj.tiles
+    chunks = []
+    for t in range(obj.tiles):
+        if view_bits[t] == 32:
+            chunks.append(st.S[t].view(np.uint8).reshape(-1))
+        else:
+            chunks.append(oracle.pack(view_bits[t], st.codes[t]))
+    codes = torch.from_numpy(np.concatenate(chunks)).cuda()
+    sdt = np.float32 if obj.scale_dtype == Q.F32 else np.float16
+    scales = torch.from_numpy(st.scales.astype(sdt).reshape(-1)).cuda()
+    ref = None if st.ref is None else torch.from_numpy(st.ref.reshape(-1)).cuda()
+    obj.import_(codes, scales, ref)
