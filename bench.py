@@ -48,6 +48,10 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--replicas", type=int, default=0,
                     help="independent layer replicas (0: enough to exceed 4x L2)")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="override the number of layers stepped (small profiling cases)")
+    ap.add_argument("--launch-samples", type=int, default=200,
+                    help="launches timed one by one for the roofline figure")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     return ap.parse_args()
@@ -193,6 +197,8 @@ def run_ours(args, rank, world, local_rank):
     probe.close()
     replicas = args.replicas or pick_replicas(wl0, props.L2_cache_size, per_layer)
     layers = wl0.layers * replicas
+    if args.layers:
+        layers, replicas = args.layers, max(1, args.layers // wl0.layers)
     objs = [make(m, layers) for m in wl0.scale_modes]
     T = objs[0].tiles
     bytes_per_step = sum(o.bytes_per_step() for o in objs)
@@ -269,7 +275,8 @@ def run_ours(args, rank, world, local_rank):
 
     # per-launch durations of the dominant kernel, events on its stream
     dom = max(objs, key=lambda o: o.bytes_per_step())
-    nlaunch = min(K, 200)
+    dom_bytes = dom.bytes_per_step()
+    nlaunch = max(1, min(K, args.launch_samples))
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(nlaunch)]
     for i in range(nlaunch):
@@ -322,7 +329,6 @@ def run_ours(args, rank, world, local_rank):
         o.close()
 
     peak, peak_kind = measured_peaks()
-    dom_bytes = dom.bytes_per_step()
     achieved = dom_bytes / (launch_ms / 1e3) / 1e9
     traffic = read_traffic(args.workload)
     result = {
@@ -340,7 +346,7 @@ def run_ours(args, rank, world, local_rank):
         "data": "synthetic (seeded Philox4x32-10 decode streams)",
         "config": {
             "workload": wl0.name, "description": wl0.description, "batch": wl0.batch,
-            "heads": wl0.heads, "d_k": wl0.d_k, "d_v": wl0.d_v, "layers": wl0.layers,
+            "heads": wl0.heads, "d_k": wl0.d_k, "d_v": wl0.d_v, "layers": layers,
             "layer_replicas": replicas, "tiles_per_gpu": T,
             "objects": len(objs), "scale_modes": list(wl0.scale_modes),
             "l2": f"cold: state + inputs of {layers} layers ({(per_layer * layers) / 1e6:.0f} MB) "
