@@ -124,6 +124,24 @@ def pick_replicas(wl, l2_bytes, per_layer_bytes):
     return max(1, math.ceil(4 * l2_bytes / per_layer_bytes))
 
 
+def rank_layer_ids(rank, layers):
+    """Layer seeds of one rank's shard: disjoint across ranks, so every rank
+    steps its own independent tiles (no data-path exchange)."""
+    return [rank * layers + l for l in range(layers)]
+
+
+def max_over_ranks(value, device=None):
+    """Max of a per-rank float over the process group (identity when not
+    distributed).  Used only outside the timed region."""
+    import torch
+    import torch.distributed as tdist
+    if not (tdist.is_available() and tdist.is_initialized()):
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def default_steps(step_seconds_estimate):
     # about 3 s of timed work, never fewer than 50 steps
     return max(50, int(3.0 / max(step_seconds_estimate, 1e-7)))
@@ -218,7 +236,7 @@ def run_ours(args, rank, world, local_rank):
     ring = []
     host_ring = []
     for s in range(ring_n):
-        parts = [synth.gen_step(wl0, s, layer=rank * layers + l) for l in range(layers)]
+        parts = [synth.gen_step(wl0, s, layer=lid) for lid in rank_layer_ids(rank, layers)]
         cat = lambda name: (None if getattr(parts[0], name) is None
                             else np.concatenate([getattr(p, name) for p in parts]))
         x = synth.StepInputs(cat("q"), cat("k"), cat("v"), cat("gates"))
@@ -265,11 +283,8 @@ def run_ours(args, rank, world, local_rank):
     e1.record(stream)
     torch.cuda.synchronize()
     clk = clocks.stop()
-    ms_total = e0.elapsed_time(e1)
+    ms_total = max_over_ranks(e0.elapsed_time(e1), dev)
     if dist:
-        t = torch.tensor([ms_total], device=dev)
-        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
-        ms_total = float(t.item())
         tdist.barrier()
     ms_step = ms_total / K
 
@@ -315,11 +330,7 @@ def run_ours(args, rank, world, local_rank):
                 o.step_host(*pin[i % len(pin)], hout, stream)
         e1.record(stream)
         torch.cuda.synchronize()
-        ems = e0.elapsed_time(e1)
-        if dist:
-            t = torch.tensor([ems], device=dev)
-            tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
-            ems = float(t.item())
+        ems = max_over_ranks(e0.elapsed_time(e1), dev)
         e2e = {"value": world * T * Ke / (ems / 1e3), "unit": "state-updates/s",
                "h2d_bytes_per_step": int(h2d * len(objs)), "d2h_bytes_per_step": int(d2h),
                "steps": Ke}
