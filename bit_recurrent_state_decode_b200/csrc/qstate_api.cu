@@ -43,6 +43,8 @@ struct qstate {
     unsigned char* d_head_bits = nullptr;
     const qs::StepEntry* entry = nullptr;
     int grid = 1;
+    int dyn_smem = 0;                 // bytes of pipeline stages per CTA
+    qs::StepParams stage{};           // stage layout fields only
     // staging buffers of qstate_step_host (allocated by its first call)
     void* st_q = nullptr;
     void* st_k = nullptr;
@@ -80,6 +82,15 @@ qs::StepParams params_of(const qstate* s) {
     p.scale_f32 = s->L.scale_dtype == QSTATE_F32;
     p.gamma = s->L.gamma;
     p.eps_b = s->eps_b;
+    p.nstages = s->stage.nstages;
+    p.stage_bytes = s->stage.stage_bytes;
+    p.off_codes = s->stage.off_codes;
+    p.off_scales = s->stage.off_scales;
+    p.off_q = s->stage.off_q;
+    p.off_k = s->stage.off_k;
+    p.off_v = s->stage.off_v;
+    p.off_ga = s->stage.off_ga;
+    p.off_ref = s->stage.off_ref;
     return p;
 }
 
@@ -107,7 +118,7 @@ int zero_state(qstate* s, cudaStream_t st) {
         return QSTATE_ECUDA;
     if (s->ref_bytes && cudaMemsetAsync(s->d_ref, 0, s->ref_bytes, st) != cudaSuccess)
         return QSTATE_ECUDA;
-    if (cudaMemsetAsync(s->d_counters, 0, 2 * sizeof(unsigned long long), st) != cudaSuccess)
+    if (cudaMemsetAsync(s->d_counters, 0, 3 * sizeof(unsigned long long), st) != cudaSuccess)
         return QSTATE_ECUDA;
     return QSTATE_OK;
 }
@@ -202,7 +213,7 @@ int qstate_create(const qstate_layout* L, int bits, int group, qstate_scale_mode
     bool ok = alloc((void**)&s->d_codes, s->code_bytes) &&
               alloc(&s->d_scales, s->scale_bytes) &&
               alloc((void**)&s->d_ref, s->ref_bytes) &&
-              alloc((void**)&s->d_counters, 2 * sizeof(unsigned long long));
+              alloc((void**)&s->d_counters, 3 * sizeof(unsigned long long));
     if (ok && !hb.empty()) {
         ok = alloc((void**)&s->d_head_off, head_off.size() * sizeof(long long)) &&
              alloc((void**)&s->d_head_bits, hb.size()) &&
@@ -220,10 +231,43 @@ int qstate_create(const qstate_layout* L, int bits, int group, qstate_scale_mode
     const qs::StepEntry* tab = dk == 64 ? (dv == 64 ? qs::step_table_64_64() : qs::step_table_64_128())
                                         : (dv == 64 ? qs::step_table_128_64() : qs::step_table_128_128());
     s->entry = &tab[(L->kind == QSTATE_GDN) * 4 + (sm == QSTATE_YOKED) * 2 + (rm == QSTATE_BDR)];
+
+    // pipeline stage: codes | scales | q | k | v | GLA gate vector | reference
+    {
+        auto up16 = [](int64_t x) { return (x + 15) & ~int64_t(15); };
+        int maxbits = hb.empty() ? bits : 0;
+        for (uint8_t b : hb) maxbits = b > maxbits ? b : maxbits;
+        qs::StepParams& g = s->stage;
+        int64_t off = 0;
+        g.off_codes = 0;
+        off = up16(tile_bytes_of(maxbits, dk, dv));
+        g.off_scales = -1;
+        if (quantized && group) {
+            g.off_scales = (int)off;
+            off = up16(off + s->n_scales * s->scale_size);
+        }
+        g.off_q = (int)off;  off = up16(off + dk * s->in_size);
+        g.off_k = (int)off;  off = up16(off + dk * s->in_size);
+        g.off_v = (int)off;  off = up16(off + dv * s->in_size);
+        g.off_ga = -1;
+        if (L->kind == QSTATE_GLA) { g.off_ga = (int)off; off = up16(off + dk * s->gate_size); }
+        g.off_ref = -1;
+        if (sm == QSTATE_YOKED) { g.off_ref = (int)off; off = up16(off + (int64_t)dk * dv * 4); }
+        g.stage_bytes = (int)off;
+        // as many stages (2..4) as fit in ~200 KB of shared memory
+        int ns = (int)(200 * 1024 / off);
+        g.nstages = ns < 2 ? 2 : ns > qs::kMaxStages ? qs::kMaxStages : ns;
+        s->dyn_smem = g.nstages * g.stage_bytes;
+    }
     int sms = 0;
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, s->device);
-    int per_sm = s->entry->blocks_per_sm();
-    if (per_sm < 1) per_sm = 1;
+    int per_sm = s->entry->blocks_per_sm(s->dyn_smem);
+    if (per_sm < 1) {
+        cudaGetLastError();
+        free_all(s);
+        delete s;
+        return QSTATE_EUNSUPPORTED;
+    }
     long long g = (long long)sms * per_sm;
     if (g < 1) g = 1;
     if (s->tiles < g) g = s->tiles > 0 ? s->tiles : 1;
@@ -268,7 +312,7 @@ int qstate_step(qstate* s, const void* q, const void* k, const void* v, const vo
     p.v = v;
     p.gates = gates;
     p.out = out;
-    s->entry->launch(p, s->grid, (cudaStream_t)stream);
+    s->entry->launch(p, s->grid, s->dyn_smem, (cudaStream_t)stream);
     return cudaGetLastError() == cudaSuccess ? QSTATE_OK : QSTATE_ECUDA;
 }
 
@@ -375,13 +419,14 @@ int64_t qstate_bytes_per_step(const qstate* s) {
 
 int qstate_status(qstate* s, qstate_counters* o, qstate_stream stream) {
     if (!s || !o) return QSTATE_EINVAL;
-    unsigned long long h[2] = {0, 0};
+    unsigned long long h[3] = {0, 0, 0};
     cudaStream_t st = (cudaStream_t)stream;
     if (cudaMemcpyAsync(h, s->d_counters, sizeof(h), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
         cudaStreamSynchronize(st) != cudaSuccess)
         return QSTATE_ECUDA;
     o->nonfinite = h[0];
     o->saturated = h[1];
+    o->pipeline_timeouts = h[2];
     return QSTATE_OK;
 }
 

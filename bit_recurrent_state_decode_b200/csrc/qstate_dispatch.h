@@ -8,8 +8,10 @@
 namespace qs {
 
 struct StepEntry {
-    void (*launch)(const StepParams&, int grid, cudaStream_t);
-    int (*blocks_per_sm)();
+    void (*launch)(const StepParams&, int grid, int dyn_smem, cudaStream_t);
+    // resident CTAs per SM with `dyn_smem` bytes of dynamic shared memory
+    // (also raises the kernel's dynamic shared-memory limit to that size)
+    int (*blocks_per_sm)(int dyn_smem);
     int threads;
 };
 

@@ -5,15 +5,17 @@ namespace qs {
 namespace {
 
 template <bool GDN, bool YOKED, bool BDR>
-void launch(const StepParams& p, int grid, cudaStream_t st) {
-    step_kernel<64, 128, GDN, YOKED, BDR><<<grid, Geo<64, 128>::NT, 0, st>>>(p);
+void launch(const StepParams& p, int grid, int dyn_smem, cudaStream_t st) {
+    step_kernel<64, 128, GDN, YOKED, BDR><<<grid, Geo<64, 128>::NT, dyn_smem, st>>>(p);
 }
 
 template <bool GDN, bool YOKED, bool BDR>
-int blocks_per_sm() {
+int blocks_per_sm(int dyn_smem) {
+    auto* k = step_kernel<64, 128, GDN, YOKED, BDR>;
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn_smem) != cudaSuccess)
+        return 0;
     int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-            &n, step_kernel<64, 128, GDN, YOKED, BDR>, Geo<64, 128>::NT, 0) != cudaSuccess)
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, Geo<64, 128>::NT, dyn_smem) != cudaSuccess)
         return 0;
     return n;
 }

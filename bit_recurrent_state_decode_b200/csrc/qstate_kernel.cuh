@@ -4,22 +4,33 @@
 // Table 1; scale modes: "When Dynamic Scaling Fails", Abstract; BDR: the
 // Abstract and Figure 4 of the first page).
 //
-// Work decomposition.  One CTA steps one (layer, batch, head) tile at a time
-// and walks tiles with a grid stride (the grid is sized to the SM count times
-// the resident CTAs per SM).  Each thread owns an 8 x 8 block of the tile:
-// 8 consecutive rows (one "row block" of the canonical reduction) and 8
-// consecutive columns.  A warp covers all d_v columns of 32/(d_v/8) row
-// blocks, so
-//   - the column sums r_j, o_j are an in-thread fma chain over the block
-//     (exactly the canonical block sum), an xor butterfly across the row
-//     blocks of the warp (adjacent blocks first), and a pairwise tree across
-//     warps through shared memory;
-//   - the group maximum along d_v is an in-thread max plus an xor butterfly
-//     across the lanes that share the group;
-// and every load of a warp is a set of fully used 32-byte sectors.  The
-// state is read once and written once per step; nothing spills to global
-// scratch.  No tensor cores: the step is a rank-1 update plus two
-// matrix-vector products per tile.
+// Work decomposition.  Persistent CTAs (grid = SMs x resident CTAs) walk the
+// (layer, batch, head) tiles with a grid stride, one tile per CTA at a time.
+// Each CTA runs an NSTAGE-deep pipeline: one elected thread issues 1-D bulk
+// copies (the TMA engine, cp.async.bulk) of a tile's packed codes, scales,
+// q / k / v, GLA gate vector and yoked reference state into a shared-memory
+// stage, completing on an mbarrier; the CTA computes the tile from shared
+// memory and writes the new codes, scales and output straight to global
+// memory.  Every wait on an mbarrier is bounded: on expiry the kernel counts a
+// pipeline timeout, drains its own copies (again bounded) and returns.
+//
+// Each thread owns an 8 x 8 block of the tile: 8 consecutive rows (one row
+// block of the canonical reduction) and 8 consecutive columns.  A warp covers
+// all d_v columns of 32/(d_v/8) row blocks, so
+//   - the column sums r_j, o_j are an in-thread fma chain over the block (the
+//     canonical block sum), an xor butterfly across the warp's row blocks
+//     (adjacent blocks first) and a pairwise tree across warps in shared
+//     memory;
+//   - the group maxima along d_v are an in-thread max plus a reduce-scatter
+//     across the lanes sharing the group, so each lane derives the scale of
+//     one (row, group) and broadcasts its reciprocal with shuffles.
+// Element arithmetic is branch-free and uses the packed fp32x2 instructions
+// of sm_100 (each lane of a pair rounds exactly as the scalar instruction).
+// Codes are decoded with exponent-bias tricks (a masked field ORed into the
+// significand of 2^23 is an exact float, no int->float conversion) and
+// rounded with one fma against 1.5 * 2^23 (the exact product x * inv rounded
+// half to even).  No tensor cores: per tile the step is a rank-1 update and
+// two matrix-vector products with no reuse.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -32,6 +43,11 @@ namespace qs {
 enum { K_RETNET = 0, K_MAMBA2 = 1, K_GLA = 2, K_GDN = 3 };
 enum { M_DYNAMIC = 0, M_PERSISTENT = 1, M_YOKED = 2 };
 
+constexpr int kMaxStages = 4;
+// try_wait polls before a wait is declared lost (each poll may suspend the
+// thread for a hardware-defined interval; this bound is several seconds).
+constexpr uint32_t kWaitPolls = 1u << 24;
+
 struct StepParams {
     uint8_t* codes;                 // packed codes, or the fp32 state (32-bit tiles)
     void* scales;                   // [tiles][n_scales] binary16 or binary32
@@ -41,7 +57,8 @@ struct StepParams {
     const void* v;
     const void* gates;
     float* out;
-    unsigned long long* counters;   // [0] non-finite tile-steps, [1] saturated scales
+    unsigned long long* counters;   // [0] non-finite tile-steps, [1] saturated scales,
+                                    // [2] pipeline wait timeouts
     const long long* head_off;      // per-head byte offset in a (layer, batch) row, or null
     const unsigned char* head_bits; // per-head bit width, or null (uniform)
     long long row_bytes;            // code bytes of one (layer, batch) row (mixed bits)
@@ -56,6 +73,9 @@ struct StepParams {
     int n_gate;
     int qkv_bf16, gate_bf16, scale_f32;
     float gamma, eps_b;
+    // pipeline stage layout (byte offsets inside one stage; -1 = not staged)
+    int nstages, stage_bytes;
+    int off_codes, off_scales, off_q, off_k, off_v, off_ga, off_ref;
 };
 
 template <int DK, int DV>
@@ -68,37 +88,80 @@ struct Geo {
     static_assert(NWARPS >= 1 && (NWARPS & (NWARPS - 1)) == 0, "warps must be a power of two");
 };
 
-constexpr float kMagic = 12582912.0f;          // 1.5 * 2^23: rounds to integers in [2^23, 2^24)
-constexpr int kMagicBits = 0x4B400000;
+constexpr float kMagic = 12582912.0f;          // 1.5 * 2^23: integers in [2^23, 2^24)
+constexpr uint32_t kMagicBits = 0x4B400000u;
 
-// ------------------------------------------------------------------ loads
+// ------------------------------------------------------------------ PTX helpers
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(smem_addr(bar)), "r"(count)
+                 : "memory");
+}
+
+__device__ __forceinline__ void fence_barrier_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
+                 :: "r"(smem_addr(bar)), "r"(bytes) : "memory");
+}
+
+// 1-D bulk copy global -> shared, completing `bytes` of transaction on bar.
+// dst, src 16-byte aligned; bytes a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        :: "r"(smem_addr(dst)), "l"(src), "r"(bytes), "r"(smem_addr(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok) : "r"(smem_addr(bar)), "r"(parity) : "memory");
+    return ok != 0;
+}
+
+// Bounded wait for the phase with the given parity; false if it never came.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
+    for (uint32_t i = 0; i < kWaitPolls; i++)
+        if (mbar_try_wait(bar, parity)) return true;
+    return false;
+}
+
+// ------------------------------------------------------------------ small loads
 __device__ __forceinline__ void bf16x2_to_f32(uint32_t w, float& lo, float& hi) {
     lo = __uint_as_float(w << 16);
     hi = __uint_as_float(w & 0xFFFF0000u);
 }
 
-// 8 consecutive values (element index idx, a multiple of 8) as float.
-__device__ __forceinline__ void load8(const void* base, long long idx, bool bf16, float (&o)[8]) {
+// 8 consecutive values at byte address p (16-byte aligned), f32 or bf16.
+__device__ __forceinline__ void ld8(const uint8_t* p, bool bf16, float (&o)[8]) {
     if (bf16) {
-        const uint4 u = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(base) + idx));
+        const uint4 u = *reinterpret_cast<const uint4*>(p);
         bf16x2_to_f32(u.x, o[0], o[1]);
         bf16x2_to_f32(u.y, o[2], o[3]);
         bf16x2_to_f32(u.z, o[4], o[5]);
         bf16x2_to_f32(u.w, o[6], o[7]);
     } else {
-        const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(base) + idx);
-        const float4 a = __ldg(p), b = __ldg(p + 1);
+        const float4 a = reinterpret_cast<const float4*>(p)[0];
+        const float4 b = reinterpret_cast<const float4*>(p)[1];
         o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w;
         o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
     }
 }
 
-__device__ __forceinline__ float load1(const void* base, long long idx, bool bf16) {
+__device__ __forceinline__ float ldg1(const void* base, long long idx, bool bf16) {
     if (bf16) return __uint_as_float(uint32_t(__ldg(static_cast<const uint16_t*>(base) + idx)) << 16);
     return __ldg(static_cast<const float*>(base) + idx);
 }
 
-__device__ __forceinline__ float load_scale(const void* base, long long idx, bool f32) {
+__device__ __forceinline__ float scale_at(const void* base, long long idx, bool f32) {
     if (f32) return static_cast<const float*>(base)[idx];
     return __half2float(static_cast<const __half*>(base)[idx]);
 }
@@ -106,12 +169,9 @@ __device__ __forceinline__ float load_scale(const void* base, long long idx, boo
 // Convert a scale to its stored precision; returns the stored value widened.
 __device__ __forceinline__ float to_stored(float v, bool f32, bool& saturated) {
     if (f32) return v;
-    __half h = __float2half_rn(v);
-    if (__hisinf(h)) {
-        saturated = true;
-        return 65504.0f;
-    }
-    return __half2float(h);
+    const __half h = __float2half_rn(v);
+    saturated = __hisinf(h);
+    return saturated ? 65504.0f : __half2float(h);
 }
 
 __device__ __forceinline__ void store_scale(void* base, long long idx, bool f32, float v) {
@@ -119,122 +179,191 @@ __device__ __forceinline__ void store_scale(void* base, long long idx, bool f32,
     else static_cast<__half*>(base)[idx] = __float2half_rn(v);   // exact: v is a binary16 value
 }
 
-// ------------------------------------------------------------------ codes
-// One thread's 8 codes of one row, for each bit width.  `t` is the tile base.
-template <int BITS, int DK, int DV>
-struct Codec;
+// ------------------------------------------------------------------ float2 math
+__device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) { return __fadd2_rn(a, b); }
 
-template <int DK, int DV>
-struct Codec<4, DK, DV> {
-    struct W { uint32_t w; };
-    static __device__ __forceinline__ W load(const uint8_t* t, int i, int cb) {
-        return W{*reinterpret_cast<const uint32_t*>(t + i * (DV / 2) + cb * 4)};
-    }
-    static __device__ __forceinline__ int get(const W& w, int c) {
-        return int(w.w << (28 - 4 * c)) >> 28;
-    }
-    static __device__ __forceinline__ void store(uint8_t* t, int i, int cb, const int (&c)[8]) {
-        uint32_t w = 0;
-#pragma unroll
-        for (int e = 0; e < 8; e++) w |= (uint32_t(c[e]) & 15u) << (4 * e);
-        *reinterpret_cast<uint32_t*>(t + i * (DV / 2) + cb * 4) = w;
+// ------------------------------------------------------------------ code decode
+// Exact float code values c[8] of one thread's 8 codes of a row.  A field
+// masked into place and XORed with 0x4B000000 plus its sign bit is the float
+// 2^23 + (field ^ signbit) * 2^pos; one fma scales by 2^-pos and removes the
+// bias exactly.
+template <int BITS>
+struct Decode;
+
+template <>
+struct Decode<4> {
+    static __device__ __forceinline__ void run(const uint8_t* row, int cb, float (&c)[8]) {
+        const uint32_t w = *reinterpret_cast<const uint32_t*>(row + cb * 4);
+        const uint32_t h = w >> 12;
+        const float f0 = __uint_as_float((w & 0xFu) ^ 0x4B000008u);
+        const float f1 = __uint_as_float((w & 0xF0u) ^ 0x4B000080u);
+        const float f2_ = __uint_as_float((w & 0xF00u) ^ 0x4B000800u);
+        const float f3 = __uint_as_float((w & 0xF000u) ^ 0x4B008000u);
+        const float f4 = __uint_as_float((w & 0xF0000u) ^ 0x4B080000u);
+        const float f5 = __uint_as_float((h & 0xF00u) ^ 0x4B000800u);
+        const float f6 = __uint_as_float((h & 0xF000u) ^ 0x4B008000u);
+        const float f7 = __uint_as_float((h & 0xF0000u) ^ 0x4B080000u);
+        // pos 0 / 4 :  scale 1 / 2^-4,   bias 2^23 + 8 / 2^19 + 8
+        float2 r01 = ffma2(f2(f0, f1), f2(1.0f, 0x1p-4f), f2(-8388616.0f, -524296.0f));
+        // pos 8 (codes 2 and 5), 12 (3 and 6), 16 (4 and 7)
+        float2 r25 = ffma2(f2(f2_, f5), f2(0x1p-8f, 0x1p-8f), f2(-32776.0f, -32776.0f));
+        float2 r36 = ffma2(f2(f3, f6), f2(0x1p-12f, 0x1p-12f), f2(-2056.0f, -2056.0f));
+        float2 r47 = ffma2(f2(f4, f7), f2(0x1p-16f, 0x1p-16f), f2(-136.0f, -136.0f));
+        c[0] = r01.x; c[1] = r01.y; c[2] = r25.x; c[5] = r25.y;
+        c[3] = r36.x; c[6] = r36.y; c[4] = r47.x; c[7] = r47.y;
     }
 };
 
-template <int DK, int DV>
-struct Codec<8, DK, DV> {
-    struct W { uint2 w; };
-    static __device__ __forceinline__ W load(const uint8_t* t, int i, int cb) {
-        return W{*reinterpret_cast<const uint2*>(t + i * DV + cb * 8)};
+template <>
+struct Decode<8> {
+    static __device__ __forceinline__ void run(const uint8_t* row, int cb, float (&c)[8]) {
+        const uint2 w = *reinterpret_cast<const uint2*>(row + cb * 8);
+        const uint32_t hx = w.x >> 16, hy = w.y >> 16;
+        const float b0 = __uint_as_float((w.x & 0xFFu) ^ 0x4B000080u);
+        const float b1 = __uint_as_float((w.x & 0xFF00u) ^ 0x4B008000u);
+        const float b2 = __uint_as_float((hx & 0xFFu) ^ 0x4B000080u);
+        const float b3 = __uint_as_float((hx & 0xFF00u) ^ 0x4B008000u);
+        const float b4 = __uint_as_float((w.y & 0xFFu) ^ 0x4B000080u);
+        const float b5 = __uint_as_float((w.y & 0xFF00u) ^ 0x4B008000u);
+        const float b6 = __uint_as_float((hy & 0xFFu) ^ 0x4B000080u);
+        const float b7 = __uint_as_float((hy & 0xFF00u) ^ 0x4B008000u);
+        // pos 0: 2^23 + 128 ; pos 8: scale 2^-8, bias 2^15 + 128
+        const float2 s0 = f2(1.0f, 0x1p-8f), z0 = f2(-8388736.0f, -32896.0f);
+        float2 r01 = ffma2(f2(b0, b1), s0, z0);
+        float2 r23 = ffma2(f2(b2, b3), s0, z0);
+        float2 r45 = ffma2(f2(b4, b5), s0, z0);
+        float2 r67 = ffma2(f2(b6, b7), s0, z0);
+        c[0] = r01.x; c[1] = r01.y; c[2] = r23.x; c[3] = r23.y;
+        c[4] = r45.x; c[5] = r45.y; c[6] = r67.x; c[7] = r67.y;
     }
-    static __device__ __forceinline__ int get(const W& w, int c) {
-        const uint32_t v = c < 4 ? w.w.x : w.w.y;
-        return int(v << (24 - 8 * (c & 3))) >> 24;
-    }
-    static __device__ __forceinline__ void store(uint8_t* t, int i, int cb, const int (&c)[8]) {
-        uint2 w = make_uint2(0u, 0u);
+};
+
+template <>
+struct Decode<2> {
+    static __device__ __forceinline__ void run(const uint8_t* row, int cb, float (&c)[8]) {
+        const uint32_t w = *reinterpret_cast<const uint16_t*>(row + cb * 2);
 #pragma unroll
-        for (int e = 0; e < 4; e++) {
-            w.x |= (uint32_t(c[e]) & 255u) << (8 * e);
-            w.y |= (uint32_t(c[e + 4]) & 255u) << (8 * e);
+        for (int e = 0; e < 8; e += 2) {
+            const float fa = __uint_as_float((w & (3u << (2 * e))) ^ (0x4B000000u | (2u << (2 * e))));
+            const float fb = __uint_as_float((w & (3u << (2 * e + 2))) ^ (0x4B000000u | (2u << (2 * e + 2))));
+            const float sa = __uint_as_float((127u - 2u * e) << 23);        // 4^-e
+            const float sb = __uint_as_float((127u - 2u * e - 2u) << 23);   // 4^-(e+1)
+            const float za = -(__uint_as_float((150u - 2u * e) << 23) + 2.0f);       // -(2^(23-2e) + 2)
+            const float zb = -(__uint_as_float((150u - 2u * e - 2u) << 23) + 2.0f);
+            const float2 r = ffma2(f2(fa, fb), f2(sa, sb), f2(za, zb));
+            c[e] = r.x;
+            c[e + 1] = r.y;
         }
-        *reinterpret_cast<uint2*>(t + i * DV + cb * 8) = w;
     }
 };
 
+// 6-bit codes: a low-nibble plane (unsigned nibble u) and a high 2-bit plane
+// (signed s); code = u + 16 s.
 template <int DK, int DV>
-struct Codec<2, DK, DV> {
-    struct W { uint32_t w; };
-    static __device__ __forceinline__ W load(const uint8_t* t, int i, int cb) {
-        return W{*reinterpret_cast<const uint16_t*>(t + i * (DV / 4) + cb * 2)};
-    }
-    static __device__ __forceinline__ int get(const W& w, int c) {
-        return int(w.w << (30 - 2 * c)) >> 30;
-    }
-    static __device__ __forceinline__ void store(uint8_t* t, int i, int cb, const int (&c)[8]) {
-        uint32_t w = 0;
+struct Decode6 {
+    static __device__ __forceinline__ void run(const uint8_t* tile, int i, int cb, float (&c)[8]) {
+        const uint32_t wl = *reinterpret_cast<const uint32_t*>(tile + i * (DV / 2) + cb * 4);
+        const uint32_t wh = *reinterpret_cast<const uint16_t*>(tile + DK * DV / 2 + i * (DV / 4) + cb * 2);
 #pragma unroll
-        for (int e = 0; e < 8; e++) w |= (uint32_t(c[e]) & 3u) << (2 * e);
-        *reinterpret_cast<uint16_t*>(t + i * (DV / 4) + cb * 2) = uint16_t(w);
+        for (int e = 0; e < 8; e++) {
+            const uint32_t u = (wl >> (4 * e)) & 15u;
+            const float fh = __uint_as_float((wh & (3u << (2 * e))) ^ (0x4B000000u | (2u << (2 * e))));
+            const float sh = __fmaf_rn(fh, __uint_as_float((127u - 2u * e) << 23),
+                                       -(__uint_as_float((150u - 2u * e) << 23) + 2.0f));
+            c[e] = __fmaf_rn(sh, 16.0f, float(u));
+        }
+    }
+};
+
+// ------------------------------------------------------------------ code pack
+// t[e] = 1.5 * 2^23 + code (exact): the low bits of its pattern are the code's
+// two's complement.
+template <int BITS>
+struct Pack;
+
+template <>
+struct Pack<4> {
+    // offset code s = code + 8 in [0, 15]; sixteen-bit halves summed exactly in
+    // fp32, then the nibbles' sign bits flipped back to two's complement
+    static __device__ __forceinline__ void run(uint8_t* row, int cb, const float (&t)[8]) {
+        const float2 k = f2(-(kMagic - 8.0f), -(kMagic - 8.0f));
+        const float2 s01 = fadd2(f2(t[0], t[4]), k), s11 = fadd2(f2(t[1], t[5]), k);
+        const float2 s21 = fadd2(f2(t[2], t[6]), k), s31 = fadd2(f2(t[3], t[7]), k);
+        const float2 p01 = ffma2(s11, f2(16.0f, 16.0f), s01);     // (s0 + 16 s1, s4 + 16 s5)
+        const float2 p23 = ffma2(s31, f2(16.0f, 16.0f), s21);     // (s2 + 16 s3, s6 + 16 s7)
+        float2 z = ffma2(p23, f2(256.0f, 256.0f), p01);
+        z = fadd2(z, f2(8388608.0f, 8388608.0f));                  // 2^23 + 16-bit value
+        const uint32_t w = __byte_perm(__float_as_uint(z.x), __float_as_uint(z.y), 0x5410) ^ 0x88888888u;
+        *reinterpret_cast<uint32_t*>(row + cb * 4) = w;
+    }
+};
+
+template <>
+struct Pack<8> {
+    static __device__ __forceinline__ void run(uint8_t* row, int cb, const float (&t)[8]) {
+        const uint32_t a = __byte_perm(__float_as_uint(t[0]), __float_as_uint(t[1]), 0x0040);
+        const uint32_t b = __byte_perm(__float_as_uint(t[2]), __float_as_uint(t[3]), 0x0040);
+        const uint32_t c = __byte_perm(__float_as_uint(t[4]), __float_as_uint(t[5]), 0x0040);
+        const uint32_t d = __byte_perm(__float_as_uint(t[6]), __float_as_uint(t[7]), 0x0040);
+        *reinterpret_cast<uint2*>(row + cb * 8) =
+            make_uint2(__byte_perm(a, b, 0x5410), __byte_perm(c, d, 0x5410));
+    }
+};
+
+template <>
+struct Pack<2> {
+    // offset code s = code + 2 in [0, 3]
+    static __device__ __forceinline__ void run(uint8_t* row, int cb, const float (&t)[8]) {
+        const float2 k = f2(-(kMagic - 2.0f), -(kMagic - 2.0f));
+        const float2 s0 = fadd2(f2(t[0], t[4]), k), s1 = fadd2(f2(t[1], t[5]), k);
+        const float2 s2 = fadd2(f2(t[2], t[6]), k), s3 = fadd2(f2(t[3], t[7]), k);
+        const float2 p01 = ffma2(s1, f2(4.0f, 4.0f), s0);
+        const float2 p23 = ffma2(s3, f2(4.0f, 4.0f), s2);
+        float2 z = ffma2(p23, f2(16.0f, 16.0f), p01);              // 8-bit halves
+        z = fadd2(z, f2(8388608.0f, 8388608.0f));
+        const uint32_t w = __byte_perm(__float_as_uint(z.x), __float_as_uint(z.y), 0x0040) ^ 0xAAAAu;
+        *reinterpret_cast<uint16_t*>(row + cb * 2) = uint16_t(w);
     }
 };
 
 template <int DK, int DV>
-struct Codec<6, DK, DV> {
-    // low-nibble plane (4-bit layout) then high 2-bit plane (2-bit layout)
-    struct W { uint32_t lo, hi; };
-    static __device__ __forceinline__ W load(const uint8_t* t, int i, int cb) {
-        return W{*reinterpret_cast<const uint32_t*>(t + i * (DV / 2) + cb * 4),
-                 *reinterpret_cast<const uint16_t*>(t + DK * DV / 2 + i * (DV / 4) + cb * 2)};
-    }
-    static __device__ __forceinline__ int get(const W& w, int c) {
-        const uint32_t u = ((w.lo >> (4 * c)) & 15u) | (((w.hi >> (2 * c)) & 3u) << 4);
-        return int(u << 26) >> 26;
-    }
-    static __device__ __forceinline__ void store(uint8_t* t, int i, int cb, const int (&c)[8]) {
+struct Pack6 {
+    static __device__ __forceinline__ void run(uint8_t* tile, int i, int cb, const float (&t)[8]) {
         uint32_t lo = 0, hi = 0;
 #pragma unroll
         for (int e = 0; e < 8; e++) {
-            lo |= (uint32_t(c[e]) & 15u) << (4 * e);
-            hi |= ((uint32_t(c[e]) >> 4) & 3u) << (2 * e);
+            const uint32_t u = __float_as_uint(t[e]);
+            lo |= (u & 15u) << (4 * e);
+            hi |= ((u >> 4) & 3u) << (2 * e);
         }
-        *reinterpret_cast<uint32_t*>(t + i * (DV / 2) + cb * 4) = lo;
-        *reinterpret_cast<uint16_t*>(t + DK * DV / 2 + i * (DV / 4) + cb * 2) = uint16_t(hi);
+        *reinterpret_cast<uint32_t*>(tile + i * (DV / 2) + cb * 4) = lo;
+        *reinterpret_cast<uint16_t*>(tile + DK * DV / 2 + i * (DV / 4) + cb * 2) = uint16_t(hi);
     }
 };
 
 // ------------------------------------------------------------------ reductions
-// Canonical column sums of a thread-owned 8x8 block: sum_i val[r][c] * w[r].
-// The in-thread chain is the block sum, the xor butterfly over offsets
-// CBW, 2*CBW, ... joins adjacent row blocks of the warp, and the pairwise tree
-// over warps finishes the balanced tree.  Every thread receives its 8 column
-// totals.  red: shared [NWARPS][DV]; tot: shared [DV].
+// Column sums: p[8] holds this thread's canonical block sums (rows i0..i0+7)
+// for its columns j0..j0+7.  Adjacent row blocks of the warp are joined by the
+// xor butterfly over offsets CBW, 2*CBW, ..; warps by a pairwise tree.  When
+// `broadcast`, every thread gets its 8 column totals in res; otherwise the
+// totals are written to dst[j] (threads j < DV) and res is untouched.
 template <int DK, int DV>
-__device__ __forceinline__ void colsum(const float (&val)[8][8], const float (&w)[8],
-                                       float (&res)[8], float* red, float* tot,
-                                       int warp, int rbl, int j0) {
+__device__ __forceinline__ void colsum_finish(float (&p)[8], float* red, float* tot, int warp,
+                                              int rbl, int j0, bool broadcast, float (&res)[8],
+                                              float* dst) {
     using G = Geo<DK, DV>;
-    float p[8];
-#pragma unroll
-    for (int c = 0; c < 8; c++) {
-        float s = 0.0f;
-#pragma unroll
-        for (int r = 0; r < 8; r++) s = __fmaf_rn(val[r][c], w[r], s);
-        p[c] = s;
-    }
 #pragma unroll
     for (int off = G::CBW; off < 32; off <<= 1) {
 #pragma unroll
         for (int c = 0; c < 8; c++) p[c] = __fadd_rn(p[c], __shfl_xor_sync(0xFFFFFFFFu, p[c], off));
     }
-    if (G::NWARPS == 1) {
-#pragma unroll
-        for (int c = 0; c < 8; c++) res[c] = p[c];
-        return;
-    }
     if (rbl == 0) {
-#pragma unroll
-        for (int c = 0; c < 8; c++) red[warp * DV + j0 + c] = p[c];
+        float4* r4 = reinterpret_cast<float4*>(red + warp * DV + j0);
+        r4[0] = make_float4(p[0], p[1], p[2], p[3]);
+        r4[1] = make_float4(p[4], p[5], p[6], p[7]);
     }
     __syncthreads();
     if (threadIdx.x < DV) {
@@ -246,300 +375,615 @@ __device__ __forceinline__ void colsum(const float (&val)[8][8], const float (&w
 #pragma unroll
             for (int u = 0; u < n / 2; u++) t[u] = __fadd_rn(t[2 * u], t[2 * u + 1]);
         }
-        tot[threadIdx.x] = t[0];
+        if (broadcast) tot[threadIdx.x] = t[0];
+        else dst[threadIdx.x] = t[0];
     }
-    __syncthreads();
-#pragma unroll
-    for (int c = 0; c < 8; c++) res[c] = tot[j0 + c];
-    __syncthreads();   // red/tot are reused by the next reduction
+    if (broadcast) {
+        __syncthreads();
+        const float4 a = reinterpret_cast<const float4*>(tot + j0)[0];
+        const float4 b = reinterpret_cast<const float4*>(tot + j0)[1];
+        res[0] = a.x; res[1] = a.y; res[2] = a.z; res[3] = a.w;
+        res[4] = b.x; res[5] = b.y; res[6] = b.z; res[7] = b.w;
+    }
 }
 
-// Row-group maxima: in-thread over 8 columns then across the lanes of a group
-// (group > 0), or over the whole tile (group == 0, result in every m[r]).
+// Reduce-scatter of 8 per-row maxima across the L lanes of a group (L a power
+// of two, 2..16): afterwards lane lp (= lane mod L) holds the group maxima of
+// rows (lp mod L') * (8/L') + k, k < 8/L', L' = min(L, 8), in v[k].
+template <int L>
+__device__ __forceinline__ void max_scatter(float (&v)[8], int lp) {
+    constexpr int Lp = L < 8 ? L : 8;
+    if constexpr (Lp >= 8) {
+        const bool hi = (lp & 4) != 0;
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+            const float send = hi ? v[i] : v[i + 4];
+            const float keep = hi ? v[i + 4] : v[i];
+            v[i] = fmaxf(keep, __shfl_xor_sync(0xFFFFFFFFu, send, 4));
+        }
+    }
+    if constexpr (Lp >= 4) {
+        constexpr int half = Lp == 8 ? 2 : 4;       // values left to split at this level
+        const bool hi = (lp & 2) != 0;
+#pragma unroll
+        for (int i = 0; i < half; i++) {
+            const float send = hi ? v[i] : v[i + half];
+            const float keep = hi ? v[i + half] : v[i];
+            v[i] = fmaxf(keep, __shfl_xor_sync(0xFFFFFFFFu, send, 2));
+        }
+    }
+    if constexpr (Lp >= 2) {
+        constexpr int half = 8 / Lp;                 // 1, 2 or 4 values left to split
+        const bool hi = (lp & 1) != 0;
+#pragma unroll
+        for (int i = 0; i < half; i++) {
+            const float send = hi ? v[i] : v[i + half];
+            const float keep = hi ? v[i + half] : v[i];
+            v[i] = fmaxf(keep, __shfl_xor_sync(0xFFFFFFFFu, send, 1));
+        }
+    }
+    if constexpr (L == 16) v[0] = fmaxf(v[0], __shfl_xor_sync(0xFFFFFFFFu, v[0], 8));
+}
+
+// ------------------------------------------------------------------ rounding
+// RTN in the biased domain: t = 1.5 * 2^23 + round_half_even(x * inv).
+__device__ __forceinline__ float2 rtn2(float2 x, float inv) {
+    return ffma2(x, f2(inv, inv), f2(kMagic, kMagic));
+}
+
+// BDR correction of one element (branch-free).  s = a*inv - code rounded once;
+// the element is reversed when sign(d) * s > eps (d = x - a != 0) and then
+// moves one grid step toward its update.
+__device__ __forceinline__ float bdr1(float t, float s, float d, float eps) {
+    const uint32_t sg = __float_as_uint(d) & 0x80000000u;
+    const float ss = __uint_as_float(__float_as_uint(s) ^ sg);
+    const float step = __uint_as_float(sg | 0x3F800000u);
+    const bool rev = (ss > eps) & (d != 0.0f);
+    return rev ? __fadd_rn(t, step) : t;
+}
+
+// ------------------------------------------------------------------ shared state
 template <int DK, int DV>
-__device__ __forceinline__ void groupmax(float (&m)[8], int group, float* wred, int warp) {
+struct Shared {
     using G = Geo<DK, DV>;
-    if (group > 0) {
-        const int lanes = group / 8;
-        for (int off = 1; off < lanes; off <<= 1) {
+    float red_r[G::NWARPS * DV];
+    float tot_r[DV];
+    float red_q[G::NWARPS * DV];   // reference-state column sums (yoked GDN)
+    float tot_q[DV];
+    float red_o[G::NWARPS * DV];
+    float wred[2][G::NWARPS];
+};
+
+// Round (RTN, then BDR) and repack a thread's 8 x 8 block.  a holds the
+// decayed state (BDR) or the updated state (RTN); with BDR the update
+// x = fma(ur, wc, a) is formed again here.  CLAMP: some element may leave the
+// code range, so codes are clamped to [-Qmax, Qmax].
+template <int DK, int DV, int BITS, bool BDR, bool CLAMP, class URow>
+__device__ __forceinline__ void round_pack(const float (&a)[8][8], URow urow,
+                                           const float (&wc)[8], const float (&inv)[8],
+                                           float eps_b, uint8_t* ct, int i0, int cb) {
+    constexpr float fq = float((1 << (BITS - 1)) - 1);
 #pragma unroll
-            for (int r = 0; r < 8; r++) m[r] = fmaxf(m[r], __shfl_xor_sync(0xFFFFFFFFu, m[r], off));
+    for (int r = 0; r < 8; r++) {
+        float t8[8];
+        float ur = 0.0f;
+        if constexpr (BDR) ur = urow(r);
+#pragma unroll
+        for (int c = 0; c < 8; c += 2) {
+            const float2 a2 = f2(a[r][c], a[r][c + 1]);
+            const float2 x2 = BDR ? ffma2(f2(ur, ur), f2(wc[c], wc[c + 1]), a2) : a2;
+            float2 t2 = rtn2(x2, inv[r]);
+            if constexpr (CLAMP) {
+                t2.x = fminf(fmaxf(t2.x, kMagic - fq), kMagic + fq);
+                t2.y = fminf(fmaxf(t2.y, kMagic - fq), kMagic + fq);
+            }
+            if constexpr (BDR) {
+                const float2 d2 = fadd2(x2, f2(-a2.x, -a2.y));
+                const float2 cn = fadd2(f2(kMagic, kMagic), f2(-t2.x, -t2.y));   // -code
+                const float2 s2 = ffma2(a2, f2(inv[r], inv[r]), cn);
+                t2.x = bdr1(t2.x, s2.x, d2.x, eps_b);
+                t2.y = bdr1(t2.y, s2.y, d2.y, eps_b);
+                if constexpr (CLAMP) {
+                    t2.x = fminf(fmaxf(t2.x, kMagic - fq), kMagic + fq);
+                    t2.y = fminf(fmaxf(t2.y, kMagic - fq), kMagic + fq);
+                }
+            }
+            t8[c] = t2.x;
+            t8[c + 1] = t2.y;
         }
-        return;
+        if constexpr (BITS == 4) Pack<4>::run(ct + (i0 + r) * (DV / 2), cb, t8);
+        else if constexpr (BITS == 8) Pack<8>::run(ct + (i0 + r) * DV, cb, t8);
+        else if constexpr (BITS == 2) Pack<2>::run(ct + (i0 + r) * (DV / 4), cb, t8);
+        else Pack6<DK, DV>::run(ct, i0 + r, cb, t8);
     }
-    float t = m[0];
-#pragma unroll
-    for (int r = 1; r < 8; r++) t = fmaxf(t, m[r]);
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) t = fmaxf(t, __shfl_xor_sync(0xFFFFFFFFu, t, off));
-    if ((threadIdx.x & 31) == 0) wred[warp] = t;
-    __syncthreads();
-    t = wred[0];
-#pragma unroll
-    for (int w2 = 1; w2 < G::NWARPS; w2++) t = fmaxf(t, wred[w2]);
-    __syncthreads();
-#pragma unroll
-    for (int r = 0; r < 8; r++) m[r] = t;
 }
 
-// Round one element (RTN, then BDR when enabled).  Returns the code.
-template <bool BDR>
-__device__ __forceinline__ int round_code(float a, float x, float inv, int qmax, float eps_b) {
-    float t = __fmaf_rn(x, inv, kMagic);                  // one rounding of the exact product
-    t = fminf(fmaxf(t, kMagic - float(qmax)), kMagic + float(qmax));
-    int c = __float_as_int(t) - kMagicBits;
-    if (BDR) {
-        const float d = __fsub_rn(x, a);
-        if (d != 0.0f) {
-            const float s = __fmaf_rn(a, inv, -float(c));
-            if (d > 0.0f && s > eps_b) c = min(c + 1, qmax);
-            else if (d < 0.0f && s < -eps_b) c = max(c - 1, -qmax);
+// Scales of the (row, group) pairs of a thread's 8 rows for a group of L
+// lanes: reduce-scatter of the row maxima, one scale per lane, reciprocal
+// broadcast back with shuffles.  One lane of each pair stores the scale.
+template <int L, class NewScale, class PrevScale>
+__device__ __forceinline__ void group_scales(int cb, int lane, int i0, const float (&m)[8],
+                                             const float (&mref)[8], float (&inv)[8],
+                                             unsigned& nsat, float& chk2, NewScale new_scale,
+                                             PrevScale prev_scale, const StepParams& p,
+                                             long long sbase, int ng, int gcol) {
+    constexpr int Lp = L < 8 ? L : 8, nv = 8 / Lp;
+    const int lp = cb % L;
+    const bool sf32 = p.scale_f32 != 0;
+    float mv[8], rv[8];
+#pragma unroll
+    for (int r = 0; r < 8; r++) { mv[r] = m[r]; rv[r] = mref[r]; }
+    if constexpr (L > 1) {
+        max_scatter<L>(mv, lp);
+        if (p.scale_mode == M_YOKED) max_scatter<L>(rv, lp);
+    }
+    const int rbase = (lp % Lp) * nv;
+    float invm[nv];
+#pragma unroll
+    for (int k = 0; k < nv; k++) {
+        const int row = i0 + rbase + k;
+        bool sat;
+        const float d = new_scale(mv[k], rv[k], prev_scale(row), sat);
+        invm[k] = d == 0.0f ? 0.0f : __frcp_rn(d);
+        chk2 = __fmaf_rn(mv[k], 0x1p-64f, __fmaf_rn(rv[k], 0x1p-64f, chk2));
+        if (lp < 8) {
+            store_scale(p.scales, sbase + (long long)row * ng + gcol, sf32, d);
+            nsat += sat ? 1u : 0u;
         }
     }
-    return c;
-}
-
-__device__ __forceinline__ bool all_finite8(const float (&v)[8]) {
-    bool ok = true;
+    if constexpr (L == 1) {
 #pragma unroll
-    for (int e = 0; e < 8; e++) ok &= isfinite(v[e]);
-    return ok;
+        for (int r = 0; r < 8; r++) inv[r] = invm[r];
+    } else {
+        const int gbase = lane - lp;
+#pragma unroll
+        for (int r = 0; r < 8; r++) inv[r] = __shfl_sync(0xFFFFFFFFu, invm[r % nv], gbase + r / nv);
+    }
 }
 
 // ------------------------------------------------------------------ one tile
-template <int DK, int DV, int BITS, bool GDN, bool YOKED, bool BDR>
-__device__ __forceinline__ void step_tile(const StepParams& p, long long tile, uint8_t* ct,
-                                          float* red, float* tot, float* wred) {
+// st: the tile's shared-memory stage; ct: its codes in global memory.
+// g0, g1: scalar gates (alpha, beta) and pts: per-token previous scale,
+// prefetched by the caller.
+template <int DK, int DV, int BITS, bool GDN, bool YOKED, bool BDR, bool BF>
+__device__ __forceinline__ void step_tile(const StepParams& p, long long tile, const uint8_t* st,
+                                          uint8_t* ct, float g0, float g1, float pts,
+                                          Shared<DK, DV>& sh, volatile int* badflag) {
     using G = Geo<DK, DV>;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int cb = lane % G::CBW, rbl = lane / G::CBW;
     const int i0 = (warp * G::RBW + rbl) * 8, j0 = cb * 8;
     constexpr int QMAX = BITS == 32 ? 0 : (1 << (BITS - 1)) - 1;
-    const bool bf = p.qkv_bf16 != 0, gbf = p.gate_bf16 != 0, sf32 = p.scale_f32 != 0;
+    const bool sf32 = p.scale_f32 != 0;
+    constexpr int isz = BF ? 2 : 4;
+    const int group = p.group;
 
-    // step inputs
-    float kk[8], qq[8], vv[8], al[8];
-    load8(p.k, tile * DK + i0, bf, kk);
-    load8(p.q, tile * DK + i0, bf, qq);
-    load8(p.v, tile * DV + j0, bf, vv);
-    bool bad = !(all_finite8(kk) && all_finite8(qq) && all_finite8(vv));
+    // step inputs (shared-memory stage); q and k are read row by row where
+    // they are used, which keeps them out of the register file
+    const uint8_t* sk = st + p.off_k + i0 * isz;
+    const uint8_t* sq = st + p.off_q + i0 * isz;
+    auto row_in = [](const uint8_t* base, int r) -> float {
+        if constexpr (BF) return __uint_as_float(uint32_t(reinterpret_cast<const uint16_t*>(base)[r]) << 16);
+        else return reinterpret_cast<const float*>(base)[r];
+    };
+    float vv[8], al[8];
+    ld8(st + p.off_v + j0 * isz, BF, vv);
     if (p.kind == K_GLA) {
-        load8(p.gates, tile * p.n_gate + i0, gbf, al);
-        bad |= !all_finite8(al);
+        ld8(st + p.off_ga + i0 * (p.gate_bf16 ? 2 : 4), p.gate_bf16 != 0, al);
     } else {
-        const float s = p.kind == K_RETNET ? p.gamma : load1(p.gates, tile * p.n_gate, gbf);
-        bad |= !isfinite(s);
+        const float s = p.kind == K_RETNET ? p.gamma : g0;
 #pragma unroll
         for (int r = 0; r < 8; r++) al[r] = s;
     }
-    float beta = 0.0f;
-    if (GDN) {
-        beta = load1(p.gates, tile * p.n_gate + 1, gbf);
-        bad |= !isfinite(beta);
+    const float beta = GDN ? g1 : 0.0f;
+    // non-finite inputs: a scaled sum propagates inf / NaN without overflowing
+    float chk = 0.0f;
+    {
+        float kk[8], qq[8];
+        ld8(sk, BF, kk);
+        ld8(sq, BF, qq);
+#pragma unroll
+        for (int r = 0; r < 8; r++)
+            chk = __fmaf_rn(kk[r], 0x1p-64f, __fmaf_rn(qq[r], 0x1p-64f, __fmaf_rn(vv[r], 0x1p-64f,
+                  __fmaf_rn(al[r], 0x1p-64f, chk))));
     }
+    if (GDN) chk = __fmaf_rn(beta, 0x1p-64f, chk);
 
-    const int group = p.group;
-    const int ng = group ? DV / group : 1;                 // groups per row
+    const int ng = group ? DV / group : 1;
     const long long sbase = tile * (long long)p.n_scales;
-    auto sidx = [&](int r) -> long long {
-        return group ? sbase + (long long)(i0 + r) * ng + j0 / group : sbase;
+    const int gcol = group ? j0 / group : 0;
+    auto prev_scale = [&](int row) -> float {
+        if (!group) return pts;
+        const int idx = row * ng + gcol;
+        return sf32 ? reinterpret_cast<const float*>(st + p.off_scales)[idx]
+                    : __half2float(reinterpret_cast<const __half*>(st + p.off_scales)[idx]);
     };
 
-    // 1. decay
-    float a[8][8];
-    float dprev[8];
-    if (BITS == 32) {
-#pragma unroll
-        for (int r = 0; r < 8; r++) {
-            const float4* sp = reinterpret_cast<const float4*>(
-                reinterpret_cast<const float*>(ct) + (i0 + r) * DV + j0);
-            const float4 u0 = sp[0], u1 = sp[1];
-            const float s8[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-#pragma unroll
-            for (int c = 0; c < 8; c++) a[r][c] = __fmul_rn(s8[c], al[r]);
-            dprev[r] = 0.0f;
-        }
-    } else {
-        using CD = Codec<(BITS == 32 ? 8 : BITS), DK, DV>;
-#pragma unroll
-        for (int r = 0; r < 8; r++) {
-            dprev[r] = load_scale(p.scales, sidx(r), sf32);
-            const float eta = __fmul_rn(al[r], dprev[r]);
-            const auto w = CD::load(ct, i0 + r, cb);
-#pragma unroll
-            for (int c = 0; c < 8; c++) a[r][c] = __fmul_rn(float(CD::get(w, c)), eta);
-        }
-    }
-
-    // yoked reference state: stepped first, only its group maxima are kept
+    // ---- yoked reference state: stepped first; only its group maxima stay
     float mref[8];
-    if (YOKED) {
+#pragma unroll
+    for (int r = 0; r < 8; r++) mref[r] = 0.0f;
+    if constexpr (YOKED) {
         float ar[8][8];
 #pragma unroll
         for (int r = 0; r < 8; r++) {
-            const float4* sp = reinterpret_cast<const float4*>(
-                p.ref + (tile * DK + i0 + r) * (long long)DV + j0);
-            const float4 u0 = sp[0], u1 = sp[1];
-            const float s8[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+            float s8[8];
+            ld8(st + p.off_ref + ((i0 + r) * DV + j0) * 4, false, s8);
 #pragma unroll
-            for (int c = 0; c < 8; c++) ar[r][c] = __fmul_rn(s8[c], al[r]);
-        }
-        if (GDN) {
-            float rr[8];
-            colsum<DK, DV>(ar, kk, rr, red, tot, warp, rbl, j0);
-#pragma unroll
-            for (int c = 0; c < 8; c++) rr[c] = __fsub_rn(vv[c], rr[c]);
-#pragma unroll
-            for (int r = 0; r < 8; r++) {
-                const float kap = __fmul_rn(beta, kk[r]);
-#pragma unroll
-                for (int c = 0; c < 8; c++) ar[r][c] = __fmaf_rn(kap, rr[c], ar[r][c]);
+            for (int c = 0; c < 8; c += 2) {
+                const float2 v2 = fmul2(f2(s8[c], s8[c + 1]), f2(al[r], al[r]));
+                ar[r][c] = v2.x;
+                ar[r][c + 1] = v2.y;
             }
-        } else {
+        }
+        float e2[8];
+        if constexpr (GDN) {
+            float pr[8];
+#pragma unroll
+            for (int c = 0; c < 8; c++) pr[c] = 0.0f;
 #pragma unroll
             for (int r = 0; r < 8; r++)
 #pragma unroll
-                for (int c = 0; c < 8; c++) ar[r][c] = __fmaf_rn(kk[r], vv[c], ar[r][c]);
+                for (int c = 0; c < 8; c += 2) {
+                    const float kr = row_in(sk, r);
+                    const float2 v2 = ffma2(f2(ar[r][c], ar[r][c + 1]), f2(kr, kr),
+                                            f2(pr[c], pr[c + 1]));
+                    pr[c] = v2.x;
+                    pr[c + 1] = v2.y;
+                }
+            colsum_finish<DK, DV>(pr, sh.red_q, sh.tot_q, warp, rbl, j0, true, e2, nullptr);
+#pragma unroll
+            for (int c = 0; c < 8; c++) e2[c] = __fsub_rn(vv[c], e2[c]);
         }
+        float* gref = p.ref + (tile * DK) * (long long)DV;
 #pragma unroll
         for (int r = 0; r < 8; r++) {
-            float4* sp = reinterpret_cast<float4*>(p.ref + (tile * DK + i0 + r) * (long long)DV + j0);
-            sp[0] = make_float4(ar[r][0], ar[r][1], ar[r][2], ar[r][3]);
-            sp[1] = make_float4(ar[r][4], ar[r][5], ar[r][6], ar[r][7]);
+            const float kap = GDN ? __fmul_rn(beta, row_in(sk, r)) : row_in(sk, r);
             float mm = 0.0f;
 #pragma unroll
-            for (int c = 0; c < 8; c++) mm = fmaxf(mm, fabsf(ar[r][c]));
+            for (int c = 0; c < 8; c += 2) {
+                float2 w2;
+                if constexpr (GDN) w2 = f2(e2[c], e2[c + 1]);
+                else w2 = f2(vv[c], vv[c + 1]);
+                const float2 v2 = ffma2(f2(kap, kap), w2, f2(ar[r][c], ar[r][c + 1]));
+                ar[r][c] = v2.x;
+                ar[r][c + 1] = v2.y;
+                mm = fmaxf(mm, fmaxf(fabsf(v2.x), fabsf(v2.y)));
+            }
+            float4* dst = reinterpret_cast<float4*>(gref + (i0 + r) * DV + j0);
+            dst[0] = make_float4(ar[r][0], ar[r][1], ar[r][2], ar[r][3]);
+            dst[1] = make_float4(ar[r][4], ar[r][5], ar[r][6], ar[r][7]);
             mref[r] = mm;
         }
-        groupmax<DK, DV>(mref, group, wred, warp);
     }
 
-    // 2. update
-    float x[8][8];
-    if (GDN) {
-        float e[8];
-        colsum<DK, DV>(a, kk, e, red, tot, warp, rbl, j0);
+    // ---- 1. decay: a = code * (alpha * scale)   (32-bit state: S * alpha)
+    float a[8][8];
+    float dprev[8];
 #pragma unroll
-        for (int c = 0; c < 8; c++) e[c] = __fsub_rn(vv[c], e[c]);
-#pragma unroll
-        for (int r = 0; r < 8; r++) {
-            const float kap = __fmul_rn(beta, kk[r]);
-#pragma unroll
-            for (int c = 0; c < 8; c++) x[r][c] = __fmaf_rn(kap, e[c], a[r][c]);
+    for (int r = 0; r < 8; r++) {
+        float c8[8];
+        float eta;
+        if constexpr (BITS == 32) {
+            ld8(st + p.off_codes + ((i0 + r) * DV + j0) * 4, false, c8);
+            eta = al[r];
+            dprev[r] = 0.0f;
+        } else {
+            dprev[r] = prev_scale(i0 + r);
+            eta = __fmul_rn(al[r], dprev[r]);
+            const uint8_t* srow = st + p.off_codes;
+            if constexpr (BITS == 4) Decode<4>::run(srow + (i0 + r) * (DV / 2), cb, c8);
+            else if constexpr (BITS == 8) Decode<8>::run(srow + (i0 + r) * DV, cb, c8);
+            else if constexpr (BITS == 2) Decode<2>::run(srow + (i0 + r) * (DV / 4), cb, c8);
+            else Decode6<DK, DV>::run(srow, i0 + r, cb, c8);
         }
-    } else {
+#pragma unroll
+        for (int c = 0; c < 8; c += 2) {
+            const float2 v2 = fmul2(f2(c8[c], c8[c + 1]), f2(eta, eta));
+            a[r][c] = v2.x;
+            a[r][c + 1] = v2.y;
+        }
+    }
+
+    // ---- 2. update coefficients: x = fma(u_r, w_c, a), u_r = beta k_r (GDN)
+    // or k_r, formed row by row
+    auto urow = [&](int r) -> float {
+        if constexpr (GDN) return __fmul_rn(beta, row_in(sk, r));
+        else return row_in(sk, r);
+    };
+    float wc[8];
+    if constexpr (GDN) {
+        float pr[8];
+#pragma unroll
+        for (int c = 0; c < 8; c++) pr[c] = 0.0f;
 #pragma unroll
         for (int r = 0; r < 8; r++)
 #pragma unroll
-            for (int c = 0; c < 8; c++) x[r][c] = __fmaf_rn(kk[r], vv[c], a[r][c]);
+            for (int c = 0; c < 8; c += 2) {
+                const float kr = row_in(sk, r);
+                const float2 v2 = ffma2(f2(a[r][c], a[r][c + 1]), f2(kr, kr), f2(pr[c], pr[c + 1]));
+                pr[c] = v2.x;
+                pr[c + 1] = v2.y;
+            }
+        colsum_finish<DK, DV>(pr, sh.red_r, sh.tot_r, warp, rbl, j0, true, wc, nullptr);
+#pragma unroll
+        for (int c = 0; c < 8; c++) wc[c] = __fsub_rn(vv[c], wc[c]);       // e = v - r
+    } else {
+#pragma unroll
+        for (int c = 0; c < 8; c++) wc[c] = vv[c];
     }
 
-    // 3. output from the updated, not yet rounded state
+    // ---- 3. output o = x^T q and row maxima, x formed on the fly
+    float m[8];
     {
-        float o[8];
-        colsum<DK, DV>(x, qq, o, red, tot, warp, rbl, j0);
-        if (rbl == 0 && warp == 0) {
-            float4* op = reinterpret_cast<float4*>(p.out + tile * DV + j0);
-            op[0] = make_float4(o[0], o[1], o[2], o[3]);
-            op[1] = make_float4(o[4], o[5], o[6], o[7]);
-        }
-    }
-
-    if (BITS == 32) {
+        float po[8];
+#pragma unroll
+        for (int c = 0; c < 8; c++) po[c] = 0.0f;
 #pragma unroll
         for (int r = 0; r < 8; r++) {
-            float4* sp = reinterpret_cast<float4*>(reinterpret_cast<float*>(ct) + (i0 + r) * DV + j0);
-            sp[0] = make_float4(x[r][0], x[r][1], x[r][2], x[r][3]);
-            sp[1] = make_float4(x[r][4], x[r][5], x[r][6], x[r][7]);
+            float mm = 0.0f;
+            const float ur = urow(r), qr = row_in(sq, r);
+#pragma unroll
+            for (int c = 0; c < 8; c += 2) {
+                const float2 x2 = ffma2(f2(ur, ur), f2(wc[c], wc[c + 1]), f2(a[r][c], a[r][c + 1]));
+                const float2 o2 = ffma2(x2, f2(qr, qr), f2(po[c], po[c + 1]));
+                po[c] = o2.x;
+                po[c + 1] = o2.y;
+                mm = fmaxf(mm, fmaxf(fabsf(x2.x), fabsf(x2.y)));
+                if constexpr (!BDR) {        // the decayed state is not needed again
+                    a[r][c] = x2.x;
+                    a[r][c + 1] = x2.y;
+                }
+            }
+            m[r] = mm;
+        }
+        float dummy[8];
+        colsum_finish<DK, DV>(po, sh.red_o, nullptr, warp, rbl, j0, false, dummy,
+                              p.out + tile * DV);
+    }
+
+    if constexpr (BITS == 32) {
+        uint8_t* gs = ct;
+#pragma unroll
+        for (int r = 0; r < 8; r++) {
+            float x8[8];
+#pragma unroll
+            const float ur = urow(r);
+            for (int c = 0; c < 8; c += 2) {
+                float2 x2 = f2(a[r][c], a[r][c + 1]);
+                if constexpr (BDR)
+                    x2 = ffma2(f2(ur, ur), f2(wc[c], wc[c + 1]), x2);
+                x8[c] = x2.x;
+                x8[c + 1] = x2.y;
+            }
+            float4* dst = reinterpret_cast<float4*>(gs + ((i0 + r) * DV + j0) * 4);
+            dst[0] = make_float4(x8[0], x8[1], x8[2], x8[3]);
+            dst[1] = make_float4(x8[4], x8[5], x8[6], x8[7]);
         }
         return;
-    }
-
-    // 4. scale
-    float m[8];
-#pragma unroll
-    for (int r = 0; r < 8; r++) {
-        float mm = 0.0f;
-#pragma unroll
-        for (int c = 0; c < 8; c++) mm = fmaxf(mm, fabsf(x[r][c]));
-        m[r] = mm;
-    }
-    groupmax<DK, DV>(m, group, wred, warp);
-    const float fq = float(QMAX);
-    float inv[8];
-    // one lane per (row, group) stores the scale and counts its overflow
-    const bool writer = group ? (cb % (group / 8)) == 0 : threadIdx.x == 0;
-    unsigned nsat = 0;
-#pragma unroll
-    for (int r = 0; r < 8; r++) {
-        bad |= !isfinite(m[r]);
-        bool sat = false;
-        float d;
-        if (YOKED) {
-            bad |= !isfinite(mref[r]);
-            d = to_stored(__fdiv_rn(mref[r], fq), sf32, sat);
-        } else if (p.scale_mode == M_PERSISTENT) {
-            d = (m[r] > __fmul_rn(fq, dprev[r])) ? to_stored(__fdiv_rn(m[r], fq), sf32, sat)
-                                                  : dprev[r];
+    } else {
+        // ---- 4. scales
+        const float fq = float(QMAX);
+        float inv[8];
+        unsigned nsat = 0;
+        auto new_scale = [&](float mm, float mr, float dp, bool& sat) -> float {
+            sat = false;
+            if constexpr (YOKED) return to_stored(__fdiv_rn(mr, fq), sf32, sat);
+            if (p.scale_mode == M_PERSISTENT)
+                return (mm > __fmul_rn(fq, dp)) ? to_stored(__fdiv_rn(mm, fq), sf32, sat) : dp;
+            return to_stored(__fdiv_rn(mm, fq), sf32, sat);
+        };
+        float chk2 = 0.0f;
+        if (group) {
+            switch (group / 8) {
+                case 1: group_scales<1>(cb, lane, i0, m, mref, inv, nsat, chk2, new_scale, prev_scale, p, sbase, ng, gcol); break;
+                case 2: group_scales<2>(cb, lane, i0, m, mref, inv, nsat, chk2, new_scale, prev_scale, p, sbase, ng, gcol); break;
+                case 4: group_scales<4>(cb, lane, i0, m, mref, inv, nsat, chk2, new_scale, prev_scale, p, sbase, ng, gcol); break;
+                case 8: group_scales<8>(cb, lane, i0, m, mref, inv, nsat, chk2, new_scale, prev_scale, p, sbase, ng, gcol); break;
+                default: group_scales<16>(cb, lane, i0, m, mref, inv, nsat, chk2, new_scale, prev_scale, p, sbase, ng, gcol); break;
+            }
         } else {
-            d = to_stored(__fdiv_rn(m[r], fq), sf32, sat);
+            // one scale per tile
+            float t = m[0], tr = YOKED ? mref[0] : 0.0f;
+#pragma unroll
+            for (int r = 1; r < 8; r++) { t = fmaxf(t, m[r]); if (YOKED) tr = fmaxf(tr, mref[r]); }
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                t = fmaxf(t, __shfl_xor_sync(0xFFFFFFFFu, t, off));
+                if (YOKED) tr = fmaxf(tr, __shfl_xor_sync(0xFFFFFFFFu, tr, off));
+            }
+            if (lane == 0) { sh.wred[0][warp] = t; sh.wred[1][warp] = tr; }
+            __syncthreads();
+            t = sh.wred[0][0];
+            tr = sh.wred[1][0];
+#pragma unroll
+            for (int w2 = 1; w2 < G::NWARPS; w2++) { t = fmaxf(t, sh.wred[0][w2]); tr = fmaxf(tr, sh.wred[1][w2]); }
+            bool sat;
+            const float d = new_scale(t, tr, pts, sat);
+            const float iv = d == 0.0f ? 0.0f : __frcp_rn(d);
+#pragma unroll
+            for (int r = 0; r < 8; r++) inv[r] = iv;
+            chk2 = __fmaf_rn(t, 0x1p-64f, __fmaf_rn(tr, 0x1p-64f, chk2));
+            if (threadIdx.x == 0) {
+                store_scale(p.scales, sbase, sf32, d);
+                nsat += sat ? 1u : 0u;
+            }
         }
-        inv[r] = d == 0.0f ? 0.0f : __frcp_rn(d);
-        if (writer && (group || r == 0)) {
-            store_scale(p.scales, sidx(r), sf32, d);
-            nsat += sat ? 1u : 0u;
-        }
-    }
-    if (nsat) atomicAdd(p.counters + 1, (unsigned long long)nsat);
+        if (nsat) atomicAdd(p.counters + 1, (unsigned long long)nsat);
 
-    // 5-6. round and repack
-    using CD = Codec<(BITS == 32 ? 8 : BITS), DK, DV>;
+        // clamping is needed only where some |x * inv| may exceed Qmax
+        bool clamp = false;
 #pragma unroll
-    for (int r = 0; r < 8; r++) {
-        int c8[8];
-#pragma unroll
-        for (int c = 0; c < 8; c++) c8[c] = round_code<BDR>(a[r][c], x[r][c], inv[r], QMAX, p.eps_b);
-        CD::store(ct, i0 + r, cb, c8);
+        for (int r = 0; r < 8; r++) clamp |= __fmaf_rn(m[r], inv[r], -fq) > 0.0f;
+        clamp = __any_sync(0xFFFFFFFFu, clamp);
+
+        // ---- 5-6. round and repack
+        if (clamp)
+            round_pack<DK, DV, BITS, BDR, true>(a, urow, wc, inv, p.eps_b, ct, i0, cb);
+        else
+            round_pack<DK, DV, BITS, BDR, false>(a, urow, wc, inv, p.eps_b, ct, i0, cb);
+        // a tile-step is counted once if any input or group maximum was not
+        // finite (the flag is collected at the next tile's barrier)
+        if (!isfinite(chk) || !isfinite(chk2)) *badflag = 1;
     }
-    if (__syncthreads_or(bad) && threadIdx.x == 0) atomicAdd(p.counters, 1ull);
 }
+
+template <int DK, int DV, int BITS, bool GDN, bool YOKED, bool BDR>
+__device__ __forceinline__ void run_tile(const StepParams& p, long long tile, const uint8_t* st,
+                                         uint8_t* ct, float g0, float g1, float pts,
+                                         Shared<DK, DV>& sh, volatile int* badflag) {
+    if (p.qkv_bf16) step_tile<DK, DV, BITS, GDN, YOKED, BDR, true>(p, tile, st, ct, g0, g1, pts, sh, badflag);
+    else step_tile<DK, DV, BITS, GDN, YOKED, BDR, false>(p, tile, st, ct, g0, g1, pts, sh, badflag);
+}
+
+// ------------------------------------------------------------------ producer
+__device__ __forceinline__ void tile_codes(const StepParams& p, long long tile, uint8_t*& ptr,
+                                           int& bits, uint32_t& bytes, int dk, int dv) {
+    if (p.head_bits) {
+        const int h = int(tile % p.heads);
+        bits = p.head_bits[h];
+        ptr = p.codes + (tile / p.heads) * p.row_bytes + p.head_off[h];
+    } else {
+        bits = p.bits;
+        ptr = p.codes + tile * p.tile_bytes;
+    }
+    bytes = uint32_t((long long)dk * dv * bits / 8);
+}
+
+template <int DK, int DV, bool YOKED>
+__device__ __forceinline__ void issue_tile(const StepParams& p, long long tile, uint8_t* st,
+                                           uint64_t* bar) {
+    uint8_t* cp;
+    int bits;
+    uint32_t cbytes;
+    tile_codes(p, tile, cp, bits, cbytes, DK, DV);
+    const uint32_t isz = p.qkv_bf16 ? 2 : 4, gsz = p.gate_bf16 ? 2 : 4;
+    const uint32_t ssz = p.scale_f32 ? 4 : 2;
+    uint32_t total = cbytes + 2 * DK * isz + DV * isz;
+    const bool stage_scales = p.off_scales >= 0 && bits != 32;
+    if (stage_scales) total += uint32_t(p.n_scales) * ssz;
+    if (p.off_ga >= 0) total += DK * gsz;
+    if (YOKED) total += DK * DV * 4;
+    mbar_expect_tx(bar, total);
+    bulk_g2s(st + p.off_codes, cp, cbytes, bar);
+    if (stage_scales)
+        bulk_g2s(st + p.off_scales,
+                 static_cast<const uint8_t*>(p.scales) + tile * (long long)p.n_scales * ssz,
+                 uint32_t(p.n_scales) * ssz, bar);
+    bulk_g2s(st + p.off_q, static_cast<const uint8_t*>(p.q) + tile * DK * isz, DK * isz, bar);
+    bulk_g2s(st + p.off_k, static_cast<const uint8_t*>(p.k) + tile * DK * isz, DK * isz, bar);
+    bulk_g2s(st + p.off_v, static_cast<const uint8_t*>(p.v) + tile * DV * isz, DV * isz, bar);
+    if (p.off_ga >= 0)
+        bulk_g2s(st + p.off_ga, static_cast<const uint8_t*>(p.gates) + tile * DK * gsz, DK * gsz, bar);
+    if (YOKED)
+        bulk_g2s(st + p.off_ref, p.ref + tile * (long long)DK * DV, DK * DV * 4, bar);
+}
+
+// Scalar per-tile inputs that are too small for a bulk copy.
+__device__ __forceinline__ void load_scalars(const StepParams& p, long long tile, float& g0,
+                                             float& g1, float& pts) {
+    g0 = g1 = 0.0f;
+    pts = 0.0f;
+    if (tile >= p.ntiles) return;
+    if (p.kind == K_MAMBA2 || p.kind == K_GDN) g0 = ldg1(p.gates, tile * p.n_gate, p.gate_bf16 != 0);
+    if (p.kind == K_GDN) g1 = ldg1(p.gates, tile * p.n_gate + 1, p.gate_bf16 != 0);
+    if (p.group == 0) {
+        int bits = p.head_bits ? p.head_bits[tile % p.heads] : p.bits;
+        if (bits != 32) pts = scale_at(p.scales, tile, p.scale_f32 != 0);
+    }
+}
+
+// ------------------------------------------------------------------ kernel
+// Registers are capped so that several CTAs share an SM (their barriers and
+// pipeline waits then overlap); the yoked variant holds a second 8 x 8 block.
+template <int DK, int DV, bool YOKED>
+struct Occupancy {
+    static constexpr int MIN_BLOCKS = YOKED ? 1 : (Geo<DK, DV>::NT >= 256 ? 2 : 4);
+};
 
 template <int DK, int DV, bool GDN, bool YOKED, bool BDR>
-__global__ void __launch_bounds__(Geo<DK, DV>::NT)
+__global__ void __launch_bounds__(Geo<DK, DV>::NT, (Occupancy<DK, DV, YOKED>::MIN_BLOCKS))
 step_kernel(const StepParams p) {
-    using G = Geo<DK, DV>;
-    __shared__ __align__(16) float red[G::NWARPS * DV];
-    __shared__ __align__(16) float tot[DV];
-    __shared__ float wred[G::NWARPS];
-    for (long long tile = blockIdx.x; tile < p.ntiles; tile += gridDim.x) {
-        int bits = p.bits;
-        uint8_t* ct;
-        if (p.head_bits) {
-            const int h = int(tile % p.heads);
-            bits = p.head_bits[h];
-            ct = p.codes + (tile / p.heads) * p.row_bytes + p.head_off[h];
-        } else {
-            ct = p.codes + tile * p.tile_bytes;
-        }
-        // warm L2 with the next tile of this CTA (bulk prefetch, no completion)
-        if (threadIdx.x == 0 && !p.head_bits && tile + gridDim.x < p.ntiles) {
-            const uint8_t* nxt = p.codes + (tile + gridDim.x) * p.tile_bytes;
-            asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;"
-                         :: "l"(nxt), "r"(uint32_t(p.tile_bytes)) : "memory");
-        }
-        switch (bits) {
-            case 2: step_tile<DK, DV, 2, GDN, YOKED, BDR>(p, tile, ct, red, tot, wred); break;
-            case 4: step_tile<DK, DV, 4, GDN, YOKED, BDR>(p, tile, ct, red, tot, wred); break;
-            case 6: step_tile<DK, DV, 6, GDN, YOKED, BDR>(p, tile, ct, red, tot, wred); break;
-            case 8: step_tile<DK, DV, 8, GDN, YOKED, BDR>(p, tile, ct, red, tot, wred); break;
-            default:
-                if (!YOKED) step_tile<DK, DV, 32, GDN, false, BDR>(p, tile, ct, red, tot, wred);
-                break;
+    extern __shared__ __align__(128) uint8_t dsmem[];
+    __shared__ Shared<DK, DV> sh;
+    __shared__ __align__(8) uint64_t bars[kMaxStages];
+    __shared__ volatile int badf[2];
+    const int S = p.nstages;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; s++) mbar_init(&bars[s], 1);
+        fence_barrier_init();
+        badf[0] = badf[1] = 0;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; s++) {
+            const long long t = blockIdx.x + (long long)s * gridDim.x;
+            if (t < p.ntiles) issue_tile<DK, DV, YOKED>(p, t, dsmem + s * p.stage_bytes, &bars[s]);
         }
     }
+    float g0, g1, pts;
+    load_scalars(p, blockIdx.x, g0, g1, pts);
+
+    int it = 0;
+    for (long long tile = blockIdx.x; tile < p.ntiles; tile += gridDim.x, it++) {
+        const int s = it % S;
+        const uint32_t parity = (it / S) & 1;
+        float n0, n1, nts;
+        load_scalars(p, tile + gridDim.x, n0, n1, nts);    // next tile's scalars
+        const bool ok = mbar_wait_bounded(&bars[s], parity);
+        // One barrier per tile: every thread has its stage (or has given up),
+        // and every thread has finished the previous tile, so its stage and the
+        // shared reduction buffers are free again.
+        if (!__syncthreads_and(ok)) {
+            if (threadIdx.x == 0) {
+                atomicAdd(p.counters + 2, 1ull);
+                // drain this CTA's copies still in flight (tiles it .. it+S-1
+                // before the first refill, it .. it+S-2 after), each wait bounded
+                const int pending = it == 0 ? S : S - 1;
+                for (int k = 0; k < pending; k++) {
+                    const long long t2 = tile + (long long)k * gridDim.x;
+                    if (t2 < p.ntiles)
+                        (void)mbar_wait_bounded(&bars[(it + k) % S], ((it + k) / S) & 1);
+                }
+            }
+            return;
+        }
+        if (threadIdx.x == 0 && it > 0 && badf[(it - 1) & 1]) {
+            badf[(it - 1) & 1] = 0;
+            atomicAdd(p.counters, 1ull);
+        }
+        if (threadIdx.x == 0 && it > 0) {
+            // refill the previous tile's stage with the tile S strides ahead of it
+            const long long nt = tile + (long long)(S - 1) * gridDim.x;
+            const int sp = (it - 1) % S;
+            if (nt < p.ntiles) issue_tile<DK, DV, YOKED>(p, nt, dsmem + sp * p.stage_bytes, &bars[sp]);
+        }
+        uint8_t* st = dsmem + s * p.stage_bytes;
+        uint8_t* ct;
+        int bits;
+        uint32_t cbytes;
+        tile_codes(p, tile, ct, bits, cbytes, DK, DV);
+        switch (bits) {
+            case 2: run_tile<DK, DV, 2, GDN, YOKED, BDR>(p, tile, st, ct, g0, g1, pts, sh, &badf[it & 1]); break;
+            case 4: run_tile<DK, DV, 4, GDN, YOKED, BDR>(p, tile, st, ct, g0, g1, pts, sh, &badf[it & 1]); break;
+            case 6: run_tile<DK, DV, 6, GDN, YOKED, BDR>(p, tile, st, ct, g0, g1, pts, sh, &badf[it & 1]); break;
+            case 8: run_tile<DK, DV, 8, GDN, YOKED, BDR>(p, tile, st, ct, g0, g1, pts, sh, &badf[it & 1]); break;
+            default:
+                if constexpr (!YOKED)
+                    run_tile<DK, DV, 32, GDN, false, BDR>(p, tile, st, ct, g0, g1, pts, sh, &badf[it & 1]);
+                break;
+        }
+        g0 = n0;
+        g1 = n1;
+        pts = nts;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && it > 0 && badf[(it - 1) & 1]) atomicAdd(p.counters, 1ull);
 }
 
-// Dequantized state S_hat = code * scale, one thread per 8-column block.
+// ------------------------------------------------------------------ dequant
+// S_hat = code * scale, one thread per 8-column block (reads global memory).
 template <int DK, int DV>
 __global__ void dequant_kernel(const StepParams p, float* S) {
     const long long nblk = p.ntiles * DK * (DV / 8);
@@ -548,16 +992,12 @@ __global__ void dequant_kernel(const StepParams p, float* S) {
         const long long tile = b / (DK * (DV / 8));
         const int rem = int(b % (DK * (DV / 8)));
         const int i = rem / (DV / 8), cb = rem % (DV / 8);
-        int bits = p.bits;
-        const uint8_t* ct;
-        if (p.head_bits) {
-            const int h = int(tile % p.heads);
-            bits = p.head_bits[h];
-            ct = p.codes + (tile / p.heads) * p.row_bytes + p.head_off[h];
-        } else {
-            ct = p.codes + tile * p.tile_bytes;
-        }
+        uint8_t* ct;
+        int bits;
+        uint32_t cbytes;
+        tile_codes(p, tile, ct, bits, cbytes, DK, DV);
         float* dst = S + (tile * DK + i) * (long long)DV + cb * 8;
+        float c8[8];
         if (bits == 32) {
             const float* src = reinterpret_cast<const float*>(ct) + i * DV + cb * 8;
 #pragma unroll
@@ -566,20 +1006,15 @@ __global__ void dequant_kernel(const StepParams p, float* S) {
         }
         const int group = p.group, ng = group ? DV / group : 1;
         const long long si = tile * (long long)p.n_scales + (group ? (long long)i * ng + cb * 8 / group : 0);
-        const float d = load_scale(p.scales, si, p.scale_f32 != 0);
-        int c8[8];
+        const float d = scale_at(p.scales, si, p.scale_f32 != 0);
         switch (bits) {
-            case 2: { auto w = Codec<2, DK, DV>::load(ct, i, cb);
-                      for (int c = 0; c < 8; c++) c8[c] = Codec<2, DK, DV>::get(w, c); } break;
-            case 4: { auto w = Codec<4, DK, DV>::load(ct, i, cb);
-                      for (int c = 0; c < 8; c++) c8[c] = Codec<4, DK, DV>::get(w, c); } break;
-            case 6: { auto w = Codec<6, DK, DV>::load(ct, i, cb);
-                      for (int c = 0; c < 8; c++) c8[c] = Codec<6, DK, DV>::get(w, c); } break;
-            default: { auto w = Codec<8, DK, DV>::load(ct, i, cb);
-                       for (int c = 0; c < 8; c++) c8[c] = Codec<8, DK, DV>::get(w, c); } break;
+            case 2: Decode<2>::run(ct + i * (DV / 4), cb, c8); break;
+            case 4: Decode<4>::run(ct + i * (DV / 2), cb, c8); break;
+            case 6: Decode6<DK, DV>::run(ct, i, cb, c8); break;
+            default: Decode<8>::run(ct + i * DV, cb, c8); break;
         }
 #pragma unroll
-        for (int c = 0; c < 8; c++) dst[c] = __fmul_rn(float(c8[c]), d);
+        for (int c = 0; c < 8; c++) dst[c] = __fmul_rn(c8[c], d);
     }
 }
 

@@ -43,7 +43,8 @@ class Layout(ctypes.Structure):
 
 
 class Counters(ctypes.Structure):
-    _fields_ = [("nonfinite", ctypes.c_uint64), ("saturated", ctypes.c_uint64)]
+    _fields_ = [("nonfinite", ctypes.c_uint64), ("saturated", ctypes.c_uint64),
+                ("pipeline_timeouts", ctypes.c_uint64)]
 
 
 class Sizes(ctypes.Structure):
@@ -215,7 +216,8 @@ class QState:
     def status(self, stream=None) -> dict:
         c = Counters()
         _check("qstate_status", lib().qstate_status(self._h, ctypes.byref(c), _stream(stream)))
-        return {"nonfinite": int(c.nonfinite), "saturated": int(c.saturated)}
+        return {"nonfinite": int(c.nonfinite), "saturated": int(c.saturated),
+                "pipeline_timeouts": int(c.pipeline_timeouts)}
 
     # ------------------------------------------------------------ helpers
     def alloc_inputs(self, device="cuda"):

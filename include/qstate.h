@@ -122,6 +122,8 @@ typedef struct qstate qstate;
 typedef struct qstate_counters {
     uint64_t nonfinite;       /* tile-steps with a non-finite input or group max */
     uint64_t saturated;       /* binary16 scale conversions that overflowed */
+    uint64_t pipeline_timeouts; /* CTAs that gave up a bounded wait for their input
+                                   copies (the step's results are then undefined) */
 } qstate_counters;
 
 typedef struct qstate_sizes {
