@@ -44,6 +44,8 @@ struct qstate {
     const qs::StepEntry* entry = nullptr;
     int grid = 1;
     int dyn_smem = 0;                 // bytes of pipeline stages per CTA
+    unsigned wait_polls = qs::kWaitPolls;
+    long long drop_from = -1;
     qs::StepParams stage{};           // stage layout fields only
     // staging buffers of qstate_step_host (allocated by its first call)
     void* st_q = nullptr;
@@ -91,6 +93,8 @@ qs::StepParams params_of(const qstate* s) {
     p.off_v = s->stage.off_v;
     p.off_ga = s->stage.off_ga;
     p.off_ref = s->stage.off_ref;
+    p.wait_polls = s->wait_polls;
+    p.drop_from = s->drop_from;
     return p;
 }
 
@@ -415,6 +419,13 @@ int64_t qstate_bytes_per_step(const qstate* s) {
     int64_t b = 2 * s->code_bytes + 2 * s->scale_bytes + 2 * s->ref_bytes;
     b += s->tiles * ((2 * dk + dv) * s->in_size + s->n_gate * s->gate_size + dv * 4);
     return b;
+}
+
+int qstate_debug_set(qstate* s, int64_t drop_from_tile, uint32_t wait_polls) {
+    if (!s || wait_polls == 0 || drop_from_tile < -1) return QSTATE_EINVAL;
+    s->drop_from = drop_from_tile;
+    s->wait_polls = wait_polls;
+    return QSTATE_OK;
 }
 
 int qstate_status(qstate* s, qstate_counters* o, qstate_stream stream) {

@@ -44,8 +44,9 @@ enum { K_RETNET = 0, K_MAMBA2 = 1, K_GLA = 2, K_GDN = 3 };
 enum { M_DYNAMIC = 0, M_PERSISTENT = 1, M_YOKED = 2 };
 
 constexpr int kMaxStages = 4;
-// try_wait polls before a wait is declared lost (each poll may suspend the
-// thread for a hardware-defined interval; this bound is several seconds).
+// Default number of try_wait polls before a wait is declared lost (each poll
+// may suspend the thread for a hardware-defined interval; this bound is
+// several seconds).
 constexpr uint32_t kWaitPolls = 1u << 24;
 
 struct StepParams {
@@ -76,6 +77,10 @@ struct StepParams {
     // pipeline stage layout (byte offsets inside one stage; -1 = not staged)
     int nstages, stage_bytes;
     int off_codes, off_scales, off_q, off_k, off_v, off_ga, off_ref;
+    // bounded waits: polls per wait; fault injection: tiles >= drop_from are
+    // never copied (their waits run out), -1 = off
+    unsigned wait_polls;
+    long long drop_from;
 };
 
 template <int DK, int DV>
@@ -128,8 +133,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Bounded wait for the phase with the given parity; false if it never came.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
-    for (uint32_t i = 0; i < kWaitPolls; i++)
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint32_t polls) {
+    for (uint32_t i = 0; i < polls; i++)
         if (mbar_try_wait(bar, parity)) return true;
     return false;
 }
@@ -853,6 +858,7 @@ __device__ __forceinline__ void tile_codes(const StepParams& p, long long tile, 
 template <int DK, int DV, bool YOKED>
 __device__ __forceinline__ void issue_tile(const StepParams& p, long long tile, uint8_t* st,
                                            uint64_t* bar) {
+    if (p.drop_from >= 0 && tile >= p.drop_from) return;   // injected fault: never arrives
     uint8_t* cp;
     int bits;
     uint32_t cbytes;
@@ -931,7 +937,7 @@ step_kernel(const StepParams p) {
         const uint32_t parity = (it / S) & 1;
         float n0, n1, nts;
         load_scalars(p, tile + gridDim.x, n0, n1, nts);    // next tile's scalars
-        const bool ok = mbar_wait_bounded(&bars[s], parity);
+        const bool ok = mbar_wait_bounded(&bars[s], parity, p.wait_polls);
         // One barrier per tile: every thread has its stage (or has given up),
         // and every thread has finished the previous tile, so its stage and the
         // shared reduction buffers are free again.
@@ -944,7 +950,8 @@ step_kernel(const StepParams p) {
                 for (int k = 0; k < pending; k++) {
                     const long long t2 = tile + (long long)k * gridDim.x;
                     if (t2 < p.ntiles)
-                        (void)mbar_wait_bounded(&bars[(it + k) % S], ((it + k) / S) & 1);
+                        (void)mbar_wait_bounded(&bars[(it + k) % S], ((it + k) / S) & 1,
+                                                p.wait_polls);
                 }
             }
             return;

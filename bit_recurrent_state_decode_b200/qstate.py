@@ -25,7 +25,7 @@ F32, BF16, F16 = 0, 1, 2
 # every symbol include/qstate.h declares
 EXPORTS = ("qstate_create", "qstate_destroy", "qstate_reset", "qstate_step", "qstate_step_host",
            "qstate_dequant", "qstate_export", "qstate_import", "qstate_get_sizes",
-           "qstate_bytes_per_step", "qstate_status", "qstate_error_string")
+           "qstate_bytes_per_step", "qstate_status", "qstate_debug_set", "qstate_error_string")
 
 
 class QStateError(RuntimeError):
@@ -78,6 +78,7 @@ def lib():
         L.qstate_bytes_per_step.argtypes = [P]
         L.qstate_bytes_per_step.restype = ctypes.c_int64
         L.qstate_status.argtypes = [P, ctypes.POINTER(Counters), S]
+        L.qstate_debug_set.argtypes = [P, ctypes.c_int64, ctypes.c_uint32]
         L.qstate_error_string.argtypes = [I]
         L.qstate_error_string.restype = ctypes.c_char_p
         for name in EXPORTS:
@@ -218,6 +219,11 @@ class QState:
         _check("qstate_status", lib().qstate_status(self._h, ctypes.byref(c), _stream(stream)))
         return {"nonfinite": int(c.nonfinite), "saturated": int(c.saturated),
                 "pipeline_timeouts": int(c.pipeline_timeouts)}
+
+    def debug_set(self, drop_from_tile=-1, wait_polls=1 << 24):
+        """Fault injection for the bounded pipeline waits (see qstate_debug_set)."""
+        _check("qstate_debug_set", lib().qstate_debug_set(self._h, int(drop_from_tile),
+                                                          int(wait_polls)))
 
     # ------------------------------------------------------------ helpers
     def alloc_inputs(self, device="cuda"):

@@ -186,6 +186,16 @@ int64_t qstate_bytes_per_step(const qstate* s);
  * synchronises that stream. */
 int qstate_status(qstate* s, qstate_counters* out, qstate_stream stream);
 
+/* Fault injection for tests of the bounded waits (no counterpart on the
+ * pages).  The step kernel stages each tile's inputs with asynchronous bulk
+ * copies and waits for them with at most `wait_polls` polls (default 2^24,
+ * several seconds).  With drop_from_tile >= 0 the copies of every tile with
+ * index >= drop_from_tile are never issued, so those waits run out: the
+ * affected CTAs count a pipeline timeout and return, the step's results are
+ * undefined, and the CUDA context stays usable.  drop_from_tile = -1 restores
+ * normal operation.  Returns QSTATE_EINVAL for wait_polls == 0. */
+int qstate_debug_set(qstate* s, int64_t drop_from_tile, uint32_t wait_polls);
+
 /* Static, human-readable name of a return code. */
 const char* qstate_error_string(int code);
 

@@ -178,6 +178,7 @@ def run_pair(wl: synth.Workload, modes=None, batch_sel=None, layers=1, steps=8, 
     status = {m: gpu[m].status() for m in modes}
     for m in modes:
         gpu[m].close()
+        assert status[m]["pipeline_timeouts"] == 0, status
     return all_stats, status, {m: orc[m].counts.as_dict() for m in modes}
 
 

@@ -51,7 +51,7 @@ def test_fp32_recurrence_bit_exact(kind, dk, dv, dt):
 def test_retnet_full_horizon():
     stats, status, _ = run_pair(C1, steps=C1.steps, check_every=16)
     assert all(s["flips"] == 0 for s in stats)
-    assert status[synth.DYNAMIC] == {"nonfinite": 0, "saturated": 0}
+    assert status[synth.DYNAMIC] == {"nonfinite": 0, "saturated": 0, "pipeline_timeouts": 0}
 
 
 @pytest.mark.parametrize("name,batch_sel,layers,steps", [
@@ -66,7 +66,7 @@ def test_workload_reduced_batch(name, batch_sel, layers, steps):
                                       check_every=8)
     assert all(s["flips"] == 0 for s in stats), [s for s in stats if s["flips"]]
     for m in status:
-        assert status[m]["nonfinite"] == 0
+        assert status[m]["nonfinite"] == 0 and status[m]["pipeline_timeouts"] == 0
         assert status[m]["saturated"] == ocounts[m]["saturated"]
 
 
@@ -239,3 +239,27 @@ def test_invalid_pointer_alignment_rejected():
     with pytest.raises(Q.QStateError):
         obj.step(buf[1:], k, v, g, out)
     obj.close()
+
+
+def test_bounded_wait_runs_out_and_context_survives():
+    """Fault injection on the host: the copies of tiles >= 100 are never
+    issued, so their bounded waits run out.  The kernel reports pipeline
+    timeouts instead of hanging, and the device stays usable."""
+    wl = C4.scaled(batch=8, heads=32, layers=1)              # 256 tiles
+    obj = gpu_object(wl, synth.PERSISTENT, 8, 1)
+    obj.debug_set(drop_from_tile=100, wait_polls=4096)
+    x = synth.gen_step(wl, 0)
+    qd, kd, vd, gd = gpu_inputs(wl, x)
+    out = torch.empty((obj.tiles, wl.d_v), dtype=torch.float32, device="cuda")
+    obj.step(qd, kd, vd, gd, out)
+    torch.cuda.synchronize()
+    st = obj.status()
+    assert st["pipeline_timeouts"] > 0
+    obj.debug_set(-1, 1 << 24)
+    obj.reset()
+    obj.step(qd, kd, vd, gd, out)
+    torch.cuda.synchronize()
+    assert obj.status()["pipeline_timeouts"] == 0
+    obj.close()
+    stats, status, _ = run_pair(wl.scaled(batch=1), steps=4)
+    assert all(s["flips"] == 0 for s in stats)
