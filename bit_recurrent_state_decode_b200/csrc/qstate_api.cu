@@ -232,9 +232,20 @@ int qstate_create(const qstate_layout* L, int bits, int group, qstate_scale_mode
         return QSTATE_ENOMEM;
     }
 
-    const qs::StepEntry* tab = dk == 64 ? (dv == 64 ? qs::step_table_64_64() : qs::step_table_64_128())
-                                        : (dv == 64 ? qs::step_table_128_64() : qs::step_table_128_128());
-    s->entry = &tab[(L->kind == QSTATE_GDN) * 4 + (sm == QSTATE_YOKED) * 2 + (rm == QSTATE_BDR)];
+    const qs::StepEntry* tab;
+    const bool gdn = L->kind == QSTATE_GDN;
+    if (dk == 64 && dv == 64) tab = gdn ? qs::step_table_64_64_1() : qs::step_table_64_64_0();
+    else if (dk == 64) tab = gdn ? qs::step_table_64_128_1() : qs::step_table_64_128_0();
+    else if (dv == 64) tab = gdn ? qs::step_table_128_64_1() : qs::step_table_128_64_0();
+    else tab = gdn ? qs::step_table_128_128_1() : qs::step_table_128_128_0();
+    const int bidx = qs::bits_index(hb.empty() ? bits : 0);
+    const int yk = sm == QSTATE_YOKED, bd = rm == QSTATE_BDR, bf = L->qkv_dtype == QSTATE_BF16;
+    s->entry = &tab[((yk * 2 + bd) * 2 + bf) * 6 + bidx];
+    if (!s->entry->launch) {
+        free_all(s);
+        delete s;
+        return QSTATE_EUNSUPPORTED;
+    }
 
     // pipeline stage: codes | scales | q | k | v | GLA gate vector | reference
     {

@@ -15,11 +15,29 @@ struct StepEntry {
     int threads;
 };
 
-// One table per (d_k, d_v), indexed by gdn * 4 + yoked * 2 + bdr.
-const StepEntry* step_table_64_64();
-const StepEntry* step_table_64_128();
-const StepEntry* step_table_128_64();
-const StepEntry* step_table_128_128();
+// One table per (d_k, d_v, GDN?) with 48 entries, indexed by
+// ((yoked * 2 + bdr) * 2 + bf16) * 6 + bits_index (see gen_instances.py).
+const StepEntry* step_table_64_64_0();
+const StepEntry* step_table_64_64_1();
+const StepEntry* step_table_64_128_0();
+const StepEntry* step_table_64_128_1();
+const StepEntry* step_table_128_64_0();
+const StepEntry* step_table_128_64_1();
+const StepEntry* step_table_128_128_0();
+const StepEntry* step_table_128_128_1();
+
+// 0 = per-head widths, then 2, 4, 6, 8, 32 bits; -1 if invalid
+inline int bits_index(int bits) {
+    switch (bits) {
+        case 0: return 0;
+        case 2: return 1;
+        case 4: return 2;
+        case 6: return 3;
+        case 8: return 4;
+        case 32: return 5;
+        default: return -1;
+    }
+}
 
 void launch_dequant(int dk, int dv, const StepParams& p, float* S, cudaStream_t st);
 

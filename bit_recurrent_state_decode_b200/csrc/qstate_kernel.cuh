@@ -291,18 +291,18 @@ struct Pack;
 
 template <>
 struct Pack<4> {
-    // offset code s = code + 8 in [0, 15]; sixteen-bit halves summed exactly in
-    // fp32, then the nibbles' sign bits flipped back to two's complement
+    // byte m = nibble of code 2m | nibble of code 2m+1 << 4, then the low bytes
+    // of the four pairs gathered into one word
     static __device__ __forceinline__ void run(uint8_t* row, int cb, const float (&t)[8]) {
-        const float2 k = f2(-(kMagic - 8.0f), -(kMagic - 8.0f));
-        const float2 s01 = fadd2(f2(t[0], t[4]), k), s11 = fadd2(f2(t[1], t[5]), k);
-        const float2 s21 = fadd2(f2(t[2], t[6]), k), s31 = fadd2(f2(t[3], t[7]), k);
-        const float2 p01 = ffma2(s11, f2(16.0f, 16.0f), s01);     // (s0 + 16 s1, s4 + 16 s5)
-        const float2 p23 = ffma2(s31, f2(16.0f, 16.0f), s21);     // (s2 + 16 s3, s6 + 16 s7)
-        float2 z = ffma2(p23, f2(256.0f, 256.0f), p01);
-        z = fadd2(z, f2(8388608.0f, 8388608.0f));                  // 2^23 + 16-bit value
-        const uint32_t w = __byte_perm(__float_as_uint(z.x), __float_as_uint(z.y), 0x5410) ^ 0x88888888u;
-        *reinterpret_cast<uint32_t*>(row + cb * 4) = w;
+        uint32_t b[4];
+#pragma unroll
+        for (int m = 0; m < 4; m++) {
+            const uint32_t lo = __float_as_uint(t[2 * m]), hi = __float_as_uint(t[2 * m + 1]) << 4;
+            b[m] = (lo & 0x0Fu) | (hi & ~0x0Fu);
+        }
+        const uint32_t w01 = __byte_perm(b[0], b[1], 0x0040);
+        const uint32_t w23 = __byte_perm(b[2], b[3], 0x0040);
+        *reinterpret_cast<uint32_t*>(row + cb * 4) = __byte_perm(w01, w23, 0x5410);
     }
 };
 
@@ -459,14 +459,27 @@ struct Shared {
     float wred[2][G::NWARPS];
 };
 
-// Round (RTN, then BDR) and repack a thread's 8 x 8 block.  a holds the
-// decayed state (BDR) or the updated state (RTN); with BDR the update
-// x = fma(ur, wc, a) is formed again here.  CLAMP: some element may leave the
-// code range, so codes are clamped to [-Qmax, Qmax].
-template <int DK, int DV, int BITS, bool BDR, bool CLAMP, class URow>
-__device__ __forceinline__ void round_pack(const float (&a)[8][8], URow urow,
-                                           const float (&wc)[8], const float (&inv)[8],
-                                           float eps_b, uint8_t* ct, int i0, int cb) {
+__device__ __forceinline__ float sgnf(float x) {
+    return x > 0.0f ? 1.0f : (x < 0.0f ? -1.0f : 0.0f);
+}
+
+template <int DK, int DV, int BITS>
+__device__ __forceinline__ void pack_row(uint8_t* ct, int i, int cb, const float (&t8)[8]) {
+    if constexpr (BITS == 4) Pack<4>::run(ct + i * (DV / 2), cb, t8);
+    else if constexpr (BITS == 8) Pack<8>::run(ct + i * DV, cb, t8);
+    else if constexpr (BITS == 2) Pack<2>::run(ct + i * (DV / 4), cb, t8);
+    else Pack6<DK, DV>::run(ct, i, cb, t8);
+}
+
+// Round and repack a thread's 8 x 8 block, exact general path: full clamping
+// of the RTN code and of the BDR step, and the update's sign taken from
+// d = x - a element by element.  a holds the decayed state (BDR) or the
+// updated state (RTN); with BDR the update x = fma(u_r, w_c, a) is formed
+// again here.
+template <int DK, int DV, int BITS, bool BDR, class URow>
+__device__ __forceinline__ void round_pack_exact(const float (&a)[8][8], URow urow,
+                                                 const float (&wc)[8], const float (&inv)[8],
+                                                 float eps_b, uint8_t* ct, int i0, int cb) {
     constexpr float fq = float((1 << (BITS - 1)) - 1);
 #pragma unroll
     for (int r = 0; r < 8; r++) {
@@ -478,28 +491,70 @@ __device__ __forceinline__ void round_pack(const float (&a)[8][8], URow urow,
             const float2 a2 = f2(a[r][c], a[r][c + 1]);
             const float2 x2 = BDR ? ffma2(f2(ur, ur), f2(wc[c], wc[c + 1]), a2) : a2;
             float2 t2 = rtn2(x2, inv[r]);
-            if constexpr (CLAMP) {
-                t2.x = fminf(fmaxf(t2.x, kMagic - fq), kMagic + fq);
-                t2.y = fminf(fmaxf(t2.y, kMagic - fq), kMagic + fq);
-            }
+            t2.x = fminf(fmaxf(t2.x, kMagic - fq), kMagic + fq);
+            t2.y = fminf(fmaxf(t2.y, kMagic - fq), kMagic + fq);
             if constexpr (BDR) {
-                const float2 d2 = fadd2(x2, f2(-a2.x, -a2.y));
-                const float2 cn = fadd2(f2(kMagic, kMagic), f2(-t2.x, -t2.y));   // -code
+                const float2 d2 = ffma2(a2, f2(-1.0f, -1.0f), x2);                  // x - a
+                const float2 cn = ffma2(t2, f2(-1.0f, -1.0f), f2(kMagic, kMagic));  // -code
                 const float2 s2 = ffma2(a2, f2(inv[r], inv[r]), cn);
                 t2.x = bdr1(t2.x, s2.x, d2.x, eps_b);
                 t2.y = bdr1(t2.y, s2.y, d2.y, eps_b);
-                if constexpr (CLAMP) {
-                    t2.x = fminf(fmaxf(t2.x, kMagic - fq), kMagic + fq);
-                    t2.y = fminf(fmaxf(t2.y, kMagic - fq), kMagic + fq);
-                }
+                t2.x = fminf(fmaxf(t2.x, kMagic - fq), kMagic + fq);
+                t2.y = fminf(fmaxf(t2.y, kMagic - fq), kMagic + fq);
             }
             t8[c] = t2.x;
             t8[c + 1] = t2.y;
         }
-        if constexpr (BITS == 4) Pack<4>::run(ct + (i0 + r) * (DV / 2), cb, t8);
-        else if constexpr (BITS == 8) Pack<8>::run(ct + (i0 + r) * DV, cb, t8);
-        else if constexpr (BITS == 2) Pack<2>::run(ct + (i0 + r) * (DV / 4), cb, t8);
-        else Pack6<DK, DV>::run(ct, i0 + r, cb, t8);
+        pack_row<DK, DV, BITS>(ct, i0 + r, cb, t8);
+    }
+}
+
+// Fast path, taken by a warp when no element can round past the code range
+// (|x * inv| < Qmax + 1/2 everywhere) and, with BDR, when every update is large
+// enough that x != a exactly where u_r * w_c != 0: the sign of d = x - a is
+// then sign(u_r) * sign(w_c), a rank-1 sign pattern.  A BDR step can still
+// leave the range where |x * inv| > Qmax; rows flagged in `clampmask` are
+// clamped after the step.
+template <int DK, int DV, int BITS, bool BDR, class URow>
+__device__ __forceinline__ void round_pack_fast(const float (&a)[8][8], URow urow,
+                                                const float (&wc)[8], const float (&inv)[8],
+                                                float eps_b, uint32_t clampmask, uint8_t* ct,
+                                                int i0, int cb) {
+    constexpr float fq = float((1 << (BITS - 1)) - 1);
+    float sgc[8];
+    if constexpr (BDR) {
+#pragma unroll
+        for (int c = 0; c < 8; c++) sgc[c] = sgnf(wc[c]);
+    }
+#pragma unroll
+    for (int r = 0; r < 8; r++) {
+        float t8[8];
+        float ur = 0.0f, sgr = 0.0f;
+        if constexpr (BDR) {
+            ur = urow(r);
+            sgr = sgnf(ur);
+        }
+#pragma unroll
+        for (int c = 0; c < 8; c += 2) {
+            const float2 a2 = f2(a[r][c], a[r][c + 1]);
+            const float2 x2 = BDR ? ffma2(f2(ur, ur), f2(wc[c], wc[c + 1]), a2) : a2;
+            float2 t2 = rtn2(x2, inv[r]);
+            if constexpr (BDR) {
+                const float2 cn = ffma2(t2, f2(-1.0f, -1.0f), f2(kMagic, kMagic));  // -code
+                const float2 s2 = ffma2(a2, f2(inv[r], inv[r]), cn);                // u - code
+                const float2 sg = fmul2(f2(sgr, sgr), f2(sgc[c], sgc[c + 1]));      // sign(d)
+                const float2 ss = fmul2(s2, sg);
+                const float2 add = f2(ss.x > eps_b ? sg.x : 0.0f, ss.y > eps_b ? sg.y : 0.0f);
+                t2 = fadd2(t2, add);
+            }
+            t8[c] = t2.x;
+            t8[c + 1] = t2.y;
+        }
+        if (BDR && ((clampmask >> r) & 1u)) {
+#pragma unroll
+            for (int c = 0; c < 8; c++) t8[c] = fminf(fmaxf(t8[c], kMagic - fq), kMagic + fq);
+        }
+        pack_row<DK, DV, BITS>(ct, i0 + r, cb, t8);
     }
 }
 
@@ -718,8 +773,11 @@ __device__ __forceinline__ void step_tile(const StepParams& p, long long tile, c
         for (int c = 0; c < 8; c++) wc[c] = vv[c];
     }
 
-    // ---- 3. output o = x^T q and row maxima, x formed on the fly
+    // ---- 3. output o = x^T q and row maxima, x formed on the fly.  With one
+    // scale per tile the warp maxima travel with the output partials, so the
+    // tile maximum needs no barrier of its own.
     float m[8];
+    float tmax = 0.0f, tref = 0.0f;
     {
         float po[8];
 #pragma unroll
@@ -742,9 +800,48 @@ __device__ __forceinline__ void step_tile(const StepParams& p, long long tile, c
             }
             m[r] = mm;
         }
-        float dummy[8];
-        colsum_finish<DK, DV>(po, sh.red_o, nullptr, warp, rbl, j0, false, dummy,
-                              p.out + tile * DV);
+#pragma unroll
+        for (int off = G::CBW; off < 32; off <<= 1) {
+#pragma unroll
+            for (int c = 0; c < 8; c++) po[c] = __fadd_rn(po[c], __shfl_xor_sync(0xFFFFFFFFu, po[c], off));
+        }
+        if (rbl == 0) {
+            float4* r4 = reinterpret_cast<float4*>(sh.red_o + warp * DV + j0);
+            r4[0] = make_float4(po[0], po[1], po[2], po[3]);
+            r4[1] = make_float4(po[4], po[5], po[6], po[7]);
+        }
+        if (group == 0 && BITS != 32) {
+            float t = m[0], tr = mref[0];
+#pragma unroll
+            for (int r = 1; r < 8; r++) { t = fmaxf(t, m[r]); tr = fmaxf(tr, mref[r]); }
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                t = fmaxf(t, __shfl_xor_sync(0xFFFFFFFFu, t, off));
+                if (YOKED) tr = fmaxf(tr, __shfl_xor_sync(0xFFFFFFFFu, tr, off));
+            }
+            if (lane == 0) { sh.wred[0][warp] = t; sh.wred[1][warp] = tr; }
+        }
+        __syncthreads();
+        if (threadIdx.x < DV) {
+            float t[G::NWARPS];
+#pragma unroll
+            for (int w2 = 0; w2 < G::NWARPS; w2++) t[w2] = sh.red_o[w2 * DV + threadIdx.x];
+#pragma unroll
+            for (int n = G::NWARPS; n > 1; n >>= 1) {
+#pragma unroll
+                for (int u = 0; u < n / 2; u++) t[u] = __fadd_rn(t[2 * u], t[2 * u + 1]);
+            }
+            p.out[tile * DV + threadIdx.x] = t[0];
+        }
+        if (group == 0 && BITS != 32) {
+            tmax = sh.wred[0][0];
+            tref = sh.wred[1][0];
+#pragma unroll
+            for (int w2 = 1; w2 < G::NWARPS; w2++) {
+                tmax = fmaxf(tmax, sh.wred[0][w2]);
+                tref = fmaxf(tref, sh.wred[1][w2]);
+            }
+        }
     }
 
     if constexpr (BITS == 32) {
@@ -752,8 +849,8 @@ __device__ __forceinline__ void step_tile(const StepParams& p, long long tile, c
 #pragma unroll
         for (int r = 0; r < 8; r++) {
             float x8[8];
-#pragma unroll
             const float ur = urow(r);
+#pragma unroll
             for (int c = 0; c < 8; c += 2) {
                 float2 x2 = f2(a[r][c], a[r][c + 1]);
                 if constexpr (BDR)
@@ -788,27 +885,12 @@ __device__ __forceinline__ void step_tile(const StepParams& p, long long tile, c
                 default: group_scales<16>(cb, lane, i0, m, mref, inv, nsat, chk2, new_scale, prev_scale, p, sbase, ng, gcol); break;
             }
         } else {
-            // one scale per tile
-            float t = m[0], tr = YOKED ? mref[0] : 0.0f;
-#pragma unroll
-            for (int r = 1; r < 8; r++) { t = fmaxf(t, m[r]); if (YOKED) tr = fmaxf(tr, mref[r]); }
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                t = fmaxf(t, __shfl_xor_sync(0xFFFFFFFFu, t, off));
-                if (YOKED) tr = fmaxf(tr, __shfl_xor_sync(0xFFFFFFFFu, tr, off));
-            }
-            if (lane == 0) { sh.wred[0][warp] = t; sh.wred[1][warp] = tr; }
-            __syncthreads();
-            t = sh.wred[0][0];
-            tr = sh.wred[1][0];
-#pragma unroll
-            for (int w2 = 1; w2 < G::NWARPS; w2++) { t = fmaxf(t, sh.wred[0][w2]); tr = fmaxf(tr, sh.wred[1][w2]); }
             bool sat;
-            const float d = new_scale(t, tr, pts, sat);
+            const float d = new_scale(tmax, tref, pts, sat);
             const float iv = d == 0.0f ? 0.0f : __frcp_rn(d);
 #pragma unroll
             for (int r = 0; r < 8; r++) inv[r] = iv;
-            chk2 = __fmaf_rn(t, 0x1p-64f, __fmaf_rn(tr, 0x1p-64f, chk2));
+            chk2 = __fmaf_rn(tmax, 0x1p-64f, __fmaf_rn(tref, 0x1p-64f, chk2));
             if (threadIdx.x == 0) {
                 store_scale(p.scales, sbase, sf32, d);
                 nsat += sat ? 1u : 0u;
@@ -816,29 +898,35 @@ __device__ __forceinline__ void step_tile(const StepParams& p, long long tile, c
         }
         if (nsat) atomicAdd(p.counters + 1, (unsigned long long)nsat);
 
-        // clamping is needed only where some |x * inv| may exceed Qmax
-        bool clamp = false;
+        // ---- 5-6. round and repack.  The fast path needs every |x * inv| below
+        // Qmax + 1/2 (no RTN clamp) and, with BDR, updates large enough that
+        // the sign of x - a is the sign of u_r * w_c.
+        bool slow = false;
+        uint32_t clampmask = 0;
+        float wmin = 0.0f;
+        if constexpr (BDR) {
+            wmin = fabsf(wc[0]);
 #pragma unroll
-        for (int r = 0; r < 8; r++) clamp |= __fmaf_rn(m[r], inv[r], -fq) > 0.0f;
-        clamp = __any_sync(0xFFFFFFFFu, clamp);
-
-        // ---- 5-6. round and repack
-        if (clamp)
-            round_pack<DK, DV, BITS, BDR, true>(a, urow, wc, inv, p.eps_b, ct, i0, cb);
+            for (int c = 1; c < 8; c++) wmin = fminf(wmin, fabsf(wc[c]));
+        }
+#pragma unroll
+        for (int r = 0; r < 8; r++) {
+            slow |= !(__fmaf_rn(m[r], inv[r], -(fq + 0.5f)) < 0.0f);
+            if constexpr (BDR) {
+                const float eta = __fmul_rn(al[r], dprev[r]);
+                const float floor_ = fmaxf(__fmul_rn(eta, float(1 << (BITS - 1)) * 0x1p-21f), 0x1p-120f);
+                slow |= !(__fmaf_rn(fabsf(urow(r)), wmin, -floor_) > 0.0f);
+                if (__any_sync(0xFFFFFFFFu, __fmaf_rn(m[r], inv[r], -fq) > 0.0f)) clampmask |= 1u << r;
+            }
+        }
+        if (__any_sync(0xFFFFFFFFu, slow))
+            round_pack_exact<DK, DV, BITS, BDR>(a, urow, wc, inv, p.eps_b, ct, i0, cb);
         else
-            round_pack<DK, DV, BITS, BDR, false>(a, urow, wc, inv, p.eps_b, ct, i0, cb);
+            round_pack_fast<DK, DV, BITS, BDR>(a, urow, wc, inv, p.eps_b, clampmask, ct, i0, cb);
         // a tile-step is counted once if any input or group maximum was not
         // finite (the flag is collected at the next tile's barrier)
         if (!isfinite(chk) || !isfinite(chk2)) *badflag = 1;
     }
-}
-
-template <int DK, int DV, int BITS, bool GDN, bool YOKED, bool BDR>
-__device__ __forceinline__ void run_tile(const StepParams& p, long long tile, const uint8_t* st,
-                                         uint8_t* ct, float g0, float g1, float pts,
-                                         Shared<DK, DV>& sh, volatile int* badflag) {
-    if (p.qkv_bf16) step_tile<DK, DV, BITS, GDN, YOKED, BDR, true>(p, tile, st, ct, g0, g1, pts, sh, badflag);
-    else step_tile<DK, DV, BITS, GDN, YOKED, BDR, false>(p, tile, st, ct, g0, g1, pts, sh, badflag);
 }
 
 // ------------------------------------------------------------------ producer
@@ -883,6 +971,13 @@ __device__ __forceinline__ void issue_tile(const StepParams& p, long long tile, 
         bulk_g2s(st + p.off_ga, static_cast<const uint8_t*>(p.gates) + tile * DK * gsz, DK * gsz, bar);
     if (YOKED)
         bulk_g2s(st + p.off_ref, p.ref + tile * (long long)DK * DV, DK * DV * 4, bar);
+    // the tile's scalar inputs (gates, per-token scale) are read with plain
+    // loads one tile ahead; warm L2 with them now
+    if (p.kind == K_MAMBA2 || p.kind == K_GDN)
+        asm volatile("prefetch.global.L2 [%0];" :: "l"(static_cast<const uint8_t*>(p.gates) +
+                                                       tile * p.n_gate * gsz));
+    if (p.group == 0 && bits != 32)
+        asm volatile("prefetch.global.L2 [%0];" :: "l"(static_cast<const uint8_t*>(p.scales) + tile * ssz));
 }
 
 // Scalar per-tile inputs that are too small for a bulk copy.
@@ -907,7 +1002,9 @@ struct Occupancy {
     static constexpr int MIN_BLOCKS = YOKED ? 1 : (Geo<DK, DV>::NT >= 256 ? 2 : 4);
 };
 
-template <int DK, int DV, bool GDN, bool YOKED, bool BDR>
+// BITS: the uniform code width of the object (2, 4, 6, 8, 32), or 0 when the
+// width varies per head (dispatched per tile).  BF: q, k, v are bf16.
+template <int DK, int DV, int BITS, bool GDN, bool YOKED, bool BDR, bool BF>
 __global__ void __launch_bounds__(Geo<DK, DV>::NT, (Occupancy<DK, DV, YOKED>::MIN_BLOCKS))
 step_kernel(const StepParams p) {
     extern __shared__ __align__(128) uint8_t dsmem[];
@@ -971,15 +1068,16 @@ step_kernel(const StepParams p) {
         int bits;
         uint32_t cbytes;
         tile_codes(p, tile, ct, bits, cbytes, DK, DV);
-        switch (bits) {
-            case 2: run_tile<DK, DV, 2, GDN, YOKED, BDR>(p, tile, st, ct, g0, g1, pts, sh, &badf[it & 1]); break;
-            case 4: run_tile<DK, DV, 4, GDN, YOKED, BDR>(p, tile, st, ct, g0, g1, pts, sh, &badf[it & 1]); break;
-            case 6: run_tile<DK, DV, 6, GDN, YOKED, BDR>(p, tile, st, ct, g0, g1, pts, sh, &badf[it & 1]); break;
-            case 8: run_tile<DK, DV, 8, GDN, YOKED, BDR>(p, tile, st, ct, g0, g1, pts, sh, &badf[it & 1]); break;
-            default:
-                if constexpr (!YOKED)
-                    run_tile<DK, DV, 32, GDN, false, BDR>(p, tile, st, ct, g0, g1, pts, sh, &badf[it & 1]);
-                break;
+        if constexpr (BITS == 0) {
+            switch (bits) {
+                case 2: step_tile<DK, DV, 2, GDN, YOKED, BDR, BF>(p, tile, st, ct, g0, g1, pts, sh, &badf[it & 1]); break;
+                case 4: step_tile<DK, DV, 4, GDN, YOKED, BDR, BF>(p, tile, st, ct, g0, g1, pts, sh, &badf[it & 1]); break;
+                case 6: step_tile<DK, DV, 6, GDN, YOKED, BDR, BF>(p, tile, st, ct, g0, g1, pts, sh, &badf[it & 1]); break;
+                default: step_tile<DK, DV, 8, GDN, YOKED, BDR, BF>(p, tile, st, ct, g0, g1, pts, sh, &badf[it & 1]); break;
+            }
+        } else {
+            (void)bits;
+            step_tile<DK, DV, BITS, GDN, YOKED, BDR, BF>(p, tile, st, ct, g0, g1, pts, sh, &badf[it & 1]);
         }
         g0 = n0;
         g1 = n1;
