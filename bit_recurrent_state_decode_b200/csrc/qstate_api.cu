@@ -9,7 +9,7 @@
 #include <new>
 #include <vector>
 
-#include "../../include/qstate.h"
+#include "qstate.h"
 #include "qstate_dispatch.h"
 
 namespace qs {

@@ -392,44 +392,6 @@ __device__ __forceinline__ void colsum_finish(float (&p)[8], float* red, float* 
     }
 }
 
-// Reduce-scatter of 8 per-row maxima across the L lanes of a group (L a power
-// of two, 2..16): afterwards lane lp (= lane mod L) holds the group maxima of
-// rows (lp mod L') * (8/L') + k, k < 8/L', L' = min(L, 8), in v[k].
-template <int L>
-__device__ __forceinline__ void max_scatter(float (&v)[8], int lp) {
-    constexpr int Lp = L < 8 ? L : 8;
-    if constexpr (Lp >= 8) {
-        const bool hi = (lp & 4) != 0;
-#pragma unroll
-        for (int i = 0; i < 4; i++) {
-            const float send = hi ? v[i] : v[i + 4];
-            const float keep = hi ? v[i + 4] : v[i];
-            v[i] = fmaxf(keep, __shfl_xor_sync(0xFFFFFFFFu, send, 4));
-        }
-    }
-    if constexpr (Lp >= 4) {
-        constexpr int half = Lp == 8 ? 2 : 4;       // values left to split at this level
-        const bool hi = (lp & 2) != 0;
-#pragma unroll
-        for (int i = 0; i < half; i++) {
-            const float send = hi ? v[i] : v[i + half];
-            const float keep = hi ? v[i + half] : v[i];
-            v[i] = fmaxf(keep, __shfl_xor_sync(0xFFFFFFFFu, send, 2));
-        }
-    }
-    if constexpr (Lp >= 2) {
-        constexpr int half = 8 / Lp;                 // 1, 2 or 4 values left to split
-        const bool hi = (lp & 1) != 0;
-#pragma unroll
-        for (int i = 0; i < half; i++) {
-            const float send = hi ? v[i] : v[i + half];
-            const float keep = hi ? v[i + half] : v[i];
-            v[i] = fmaxf(keep, __shfl_xor_sync(0xFFFFFFFFu, send, 1));
-        }
-    }
-    if constexpr (L == 16) v[0] = fmaxf(v[0], __shfl_xor_sync(0xFFFFFFFFu, v[0], 8));
-}
-
 // ------------------------------------------------------------------ rounding
 // RTN in the biased domain: t = 1.5 * 2^23 + round_half_even(x * inv).
 __device__ __forceinline__ float2 rtn2(float2 x, float inv) {
@@ -457,6 +419,9 @@ struct Shared {
     float tot_q[DV];
     float red_o[G::NWARPS * DV];
     float wred[2][G::NWARPS];
+    // per-row maxima of each 8-column block, column-block major: [DV/8][DK]
+    float rmax[DV / 8][DK];
+    float rmaxr[DV / 8][DK];       // of the yoked reference state
 };
 
 __device__ __forceinline__ float sgnf(float x) {
@@ -558,34 +523,35 @@ __device__ __forceinline__ void round_pack_fast(const float (&a)[8][8], URow uro
     }
 }
 
-// Scales of the (row, group) pairs of a thread's 8 rows for a group of L
-// lanes: reduce-scatter of the row maxima, one scale per lane, reciprocal
-// broadcast back with shuffles.  One lane of each pair stores the scale.
-template <int L, class NewScale, class PrevScale>
-__device__ __forceinline__ void group_scales(int cb, int lane, int i0, const float (&m)[8],
-                                             const float (&mref)[8], float (&inv)[8],
-                                             unsigned& nsat, float& chk2, NewScale new_scale,
-                                             PrevScale prev_scale, const StepParams& p,
-                                             long long sbase, int ng, int gcol) {
+// Scales of the (row, group) pairs of a thread's 8 rows, for a group of L
+// lanes (L = group / 8 column blocks).  The per-row maxima of every 8-column
+// block are in shared memory; lane lp of a group derives the scales of
+// rows lp*nv .. lp*nv + nv - 1 of its row block (nv = 8 / min(L, 8)), stores
+// them, and the reciprocals go back to the group's lanes with shuffles.
+template <int DK, int DV, int L, class NewScale, class PrevScale>
+__device__ __forceinline__ void group_scales(int cb, int lane, int i0, const Shared<DK, DV>& sh,
+                                             bool yoked, float (&inv)[8], unsigned& nsat,
+                                             bool& bad, NewScale new_scale, PrevScale prev_scale,
+                                             const StepParams& p, long long sbase, int ng, int gcol) {
     constexpr int Lp = L < 8 ? L : 8, nv = 8 / Lp;
     const int lp = cb % L;
+    const int cb0 = cb - lp;                 // first column block of the group
     const bool sf32 = p.scale_f32 != 0;
-    float mv[8], rv[8];
-#pragma unroll
-    for (int r = 0; r < 8; r++) { mv[r] = m[r]; rv[r] = mref[r]; }
-    if constexpr (L > 1) {
-        max_scatter<L>(mv, lp);
-        if (p.scale_mode == M_YOKED) max_scatter<L>(rv, lp);
-    }
     const int rbase = (lp % Lp) * nv;
     float invm[nv];
 #pragma unroll
     for (int k = 0; k < nv; k++) {
         const int row = i0 + rbase + k;
+        float mm = 0.0f, mr = 0.0f;
+#pragma unroll
+        for (int b = 0; b < L; b++) {
+            mm = fmaxf(mm, sh.rmax[cb0 + b][row]);
+            if (yoked) mr = fmaxf(mr, sh.rmaxr[cb0 + b][row]);
+        }
         bool sat;
-        const float d = new_scale(mv[k], rv[k], prev_scale(row), sat);
+        const float d = new_scale(mm, mr, prev_scale(row), sat);
         invm[k] = d == 0.0f ? 0.0f : __frcp_rn(d);
-        chk2 = __fmaf_rn(mv[k], 0x1p-64f, __fmaf_rn(rv[k], 0x1p-64f, chk2));
+        bad |= !isfinite(mm) || !isfinite(mr);
         if (lp < 8) {
             store_scale(p.scales, sbase + (long long)row * ng + gcol, sf32, d);
             nsat += sat ? 1u : 0u;
@@ -636,18 +602,9 @@ __device__ __forceinline__ void step_tile(const StepParams& p, long long tile, c
         for (int r = 0; r < 8; r++) al[r] = s;
     }
     const float beta = GDN ? g1 : 0.0f;
-    // non-finite inputs: a scaled sum propagates inf / NaN without overflowing
-    float chk = 0.0f;
-    {
-        float kk[8], qq[8];
-        ld8(sk, BF, kk);
-        ld8(sq, BF, qq);
-#pragma unroll
-        for (int r = 0; r < 8; r++)
-            chk = __fmaf_rn(kk[r], 0x1p-64f, __fmaf_rn(qq[r], 0x1p-64f, __fmaf_rn(vv[r], 0x1p-64f,
-                  __fmaf_rn(al[r], 0x1p-64f, chk))));
-    }
-    if (GDN) chk = __fmaf_rn(beta, 0x1p-64f, chk);
+    // Non-finite inputs are not checked one by one: any NaN or infinity in q,
+    // k, v or the gates reaches the output o or a group maximum (0 * inf and
+    // inf - inf are NaN), where it is counted.
 
     const int ng = group ? DV / group : 1;
     const long long sbase = tile * (long long)p.n_scales;
@@ -810,6 +767,16 @@ __device__ __forceinline__ void step_tile(const StepParams& p, long long tile, c
             r4[0] = make_float4(po[0], po[1], po[2], po[3]);
             r4[1] = make_float4(po[4], po[5], po[6], po[7]);
         }
+        if (group != 0 && BITS != 32) {
+            float4* r4 = reinterpret_cast<float4*>(&sh.rmax[cb][i0]);
+            r4[0] = make_float4(m[0], m[1], m[2], m[3]);
+            r4[1] = make_float4(m[4], m[5], m[6], m[7]);
+            if (YOKED) {
+                float4* q4 = reinterpret_cast<float4*>(&sh.rmaxr[cb][i0]);
+                q4[0] = make_float4(mref[0], mref[1], mref[2], mref[3]);
+                q4[1] = make_float4(mref[4], mref[5], mref[6], mref[7]);
+            }
+        }
         if (group == 0 && BITS != 32) {
             float t = m[0], tr = mref[0];
 #pragma unroll
@@ -832,6 +799,7 @@ __device__ __forceinline__ void step_tile(const StepParams& p, long long tile, c
                 for (int u = 0; u < n / 2; u++) t[u] = __fadd_rn(t[2 * u], t[2 * u + 1]);
             }
             p.out[tile * DV + threadIdx.x] = t[0];
+            if (BITS != 32 && !isfinite(t[0])) *badflag = 1;
         }
         if (group == 0 && BITS != 32) {
             tmax = sh.wred[0][0];
@@ -875,14 +843,14 @@ __device__ __forceinline__ void step_tile(const StepParams& p, long long tile, c
                 return (mm > __fmul_rn(fq, dp)) ? to_stored(__fdiv_rn(mm, fq), sf32, sat) : dp;
             return to_stored(__fdiv_rn(mm, fq), sf32, sat);
         };
-        float chk2 = 0.0f;
+        bool bad = false;
         if (group) {
             switch (group / 8) {
-                case 1: group_scales<1>(cb, lane, i0, m, mref, inv, nsat, chk2, new_scale, prev_scale, p, sbase, ng, gcol); break;
-                case 2: group_scales<2>(cb, lane, i0, m, mref, inv, nsat, chk2, new_scale, prev_scale, p, sbase, ng, gcol); break;
-                case 4: group_scales<4>(cb, lane, i0, m, mref, inv, nsat, chk2, new_scale, prev_scale, p, sbase, ng, gcol); break;
-                case 8: group_scales<8>(cb, lane, i0, m, mref, inv, nsat, chk2, new_scale, prev_scale, p, sbase, ng, gcol); break;
-                default: group_scales<16>(cb, lane, i0, m, mref, inv, nsat, chk2, new_scale, prev_scale, p, sbase, ng, gcol); break;
+                case 1: group_scales<DK, DV, 1>(cb, lane, i0, sh, YOKED, inv, nsat, bad, new_scale, prev_scale, p, sbase, ng, gcol); break;
+                case 2: group_scales<DK, DV, 2>(cb, lane, i0, sh, YOKED, inv, nsat, bad, new_scale, prev_scale, p, sbase, ng, gcol); break;
+                case 4: group_scales<DK, DV, 4>(cb, lane, i0, sh, YOKED, inv, nsat, bad, new_scale, prev_scale, p, sbase, ng, gcol); break;
+                case 8: group_scales<DK, DV, 8>(cb, lane, i0, sh, YOKED, inv, nsat, bad, new_scale, prev_scale, p, sbase, ng, gcol); break;
+                default: group_scales<DK, DV, 16>(cb, lane, i0, sh, YOKED, inv, nsat, bad, new_scale, prev_scale, p, sbase, ng, gcol); break;
             }
         } else {
             bool sat;
@@ -890,7 +858,7 @@ __device__ __forceinline__ void step_tile(const StepParams& p, long long tile, c
             const float iv = d == 0.0f ? 0.0f : __frcp_rn(d);
 #pragma unroll
             for (int r = 0; r < 8; r++) inv[r] = iv;
-            chk2 = __fmaf_rn(tmax, 0x1p-64f, __fmaf_rn(tref, 0x1p-64f, chk2));
+            bad |= !isfinite(tmax) || !isfinite(tref);
             if (threadIdx.x == 0) {
                 store_scale(p.scales, sbase, sf32, d);
                 nsat += sat ? 1u : 0u;
@@ -923,9 +891,9 @@ __device__ __forceinline__ void step_tile(const StepParams& p, long long tile, c
             round_pack_exact<DK, DV, BITS, BDR>(a, urow, wc, inv, p.eps_b, ct, i0, cb);
         else
             round_pack_fast<DK, DV, BITS, BDR>(a, urow, wc, inv, p.eps_b, clampmask, ct, i0, cb);
-        // a tile-step is counted once if any input or group maximum was not
+        // a tile-step is counted once if an output or a group maximum was not
         // finite (the flag is collected at the next tile's barrier)
-        if (!isfinite(chk) || !isfinite(chk2)) *badflag = 1;
+        if (bad) *badflag = 1;
     }
 }
 

@@ -120,7 +120,8 @@ typedef struct qstate_layout {
 typedef struct qstate qstate;
 
 typedef struct qstate_counters {
-    uint64_t nonfinite;       /* tile-steps with a non-finite input or group max */
+    uint64_t nonfinite;       /* tile-steps with a non-finite output or group
+                                 maximum (any non-finite input produces one) */
     uint64_t saturated;       /* binary16 scale conversions that overflowed */
     uint64_t pipeline_timeouts; /* CTAs that gave up a bounded wait for their input
                                    copies (the step's results are then undefined) */

@@ -333,6 +333,7 @@ static void tile_step(const or_cfg* c, int bits, int8_t* codes, float* S, float*
     /* 3. output o_t = S_t^T q_t from the updated, not yet rounded state.
      * Reading: the output is taken before the scale and rounding steps. */
     for (int j = 0; j < dv; j++) out[j] = or_canon_dot(dk, x + j, dv, q);
+    int bad_out = !finite_all(out, dv);
 
     if (bits == 32) {                     /* quantization disabled */
         memcpy(S, x, sizeof(float) * (size_t)dk * dv);
@@ -343,6 +344,7 @@ static void tile_step(const or_cfg* c, int bits, int8_t* codes, float* S, float*
     if (c->kind == OR_GLA) bad |= !finite_all(alpha, dk);
     else if (c->kind != OR_RETNET) bad |= !isfinite(alpha[0]);
     if (c->kind == OR_GDN) bad |= !isfinite(beta);
+    bad |= bad_out;
 
     /* 4-6. scale and rounding, group by group (a group is gs consecutive
      * columns of one row, or the whole tile for a per-token scale). */

@@ -57,7 +57,7 @@ typedef struct {
 } or_cfg;
 
 typedef struct {
-    int64_t nonfinite;   /* tile-steps with a non-finite input or group maximum */
+    int64_t nonfinite;   /* tile-steps with a non-finite input, output or group maximum */
     int64_t saturated;   /* binary16 scale conversions that overflowed */
     int64_t lost, moved, reversed, bdr_applied;  /* rounding taxonomy counts */
 } or_counts;
