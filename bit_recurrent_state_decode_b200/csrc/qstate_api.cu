@@ -269,7 +269,7 @@ int qstate_create(const qstate_layout* L, int bits, int group, qstate_scale_mode
         g.off_ref = -1;
         if (sm == QSTATE_YOKED) { g.off_ref = (int)off; off = up16(off + (int64_t)dk * dv * 4); }
         g.stage_bytes = (int)off;
-        // as many stages (2..4) as fit in ~200 KB of shared memory
+        // as many stages (2..4) as fit next to the kernel's static shared memory
         int ns = (int)(200 * 1024 / off);
         g.nstages = ns < 2 ? 2 : ns > qs::kMaxStages ? qs::kMaxStages : ns;
         s->dyn_smem = g.nstages * g.stage_bytes;
@@ -277,6 +277,12 @@ int qstate_create(const qstate_layout* L, int bits, int group, qstate_scale_mode
     int sms = 0;
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, s->device);
     int per_sm = s->entry->blocks_per_sm(s->dyn_smem);
+    while (per_sm < 1 && s->stage.nstages > 2) {      // fewer stages if they do not fit
+        cudaGetLastError();
+        s->stage.nstages--;
+        s->dyn_smem = s->stage.nstages * s->stage.stage_bytes;
+        per_sm = s->entry->blocks_per_sm(s->dyn_smem);
+    }
     if (per_sm < 1) {
         cudaGetLastError();
         free_all(s);

@@ -224,23 +224,20 @@ struct Decode<4> {
 
 template <>
 struct Decode<8> {
+    // each byte (sign bit flipped) is permuted into the low byte of the float
+    // 2^23, giving 2^23 + code + 128 exactly; one add removes the bias
     static __device__ __forceinline__ void run(const uint8_t* row, int cb, float (&c)[8]) {
         const uint2 w = *reinterpret_cast<const uint2*>(row + cb * 8);
-        const uint32_t hx = w.x >> 16, hy = w.y >> 16;
-        const float b0 = __uint_as_float((w.x & 0xFFu) ^ 0x4B000080u);
-        const float b1 = __uint_as_float((w.x & 0xFF00u) ^ 0x4B008000u);
-        const float b2 = __uint_as_float((hx & 0xFFu) ^ 0x4B000080u);
-        const float b3 = __uint_as_float((hx & 0xFF00u) ^ 0x4B008000u);
-        const float b4 = __uint_as_float((w.y & 0xFFu) ^ 0x4B000080u);
-        const float b5 = __uint_as_float((w.y & 0xFF00u) ^ 0x4B008000u);
-        const float b6 = __uint_as_float((hy & 0xFFu) ^ 0x4B000080u);
-        const float b7 = __uint_as_float((hy & 0xFF00u) ^ 0x4B008000u);
-        // pos 0: 2^23 + 128 ; pos 8: scale 2^-8, bias 2^15 + 128
-        const float2 s0 = f2(1.0f, 0x1p-8f), z0 = f2(-8388736.0f, -32896.0f);
-        float2 r01 = ffma2(f2(b0, b1), s0, z0);
-        float2 r23 = ffma2(f2(b2, b3), s0, z0);
-        float2 r45 = ffma2(f2(b4, b5), s0, z0);
-        float2 r67 = ffma2(f2(b6, b7), s0, z0);
+        const uint32_t x = w.x ^ 0x80808080u, y = w.y ^ 0x80808080u;
+        const float2 z = f2(-8388736.0f, -8388736.0f);   // -(2^23 + 128)
+        const float2 r01 = fadd2(f2(__uint_as_float(__byte_perm(x, 0x4B000000u, 0x7540)),
+                                    __uint_as_float(__byte_perm(x, 0x4B000000u, 0x7541))), z);
+        const float2 r23 = fadd2(f2(__uint_as_float(__byte_perm(x, 0x4B000000u, 0x7542)),
+                                    __uint_as_float(__byte_perm(x, 0x4B000000u, 0x7543))), z);
+        const float2 r45 = fadd2(f2(__uint_as_float(__byte_perm(y, 0x4B000000u, 0x7540)),
+                                    __uint_as_float(__byte_perm(y, 0x4B000000u, 0x7541))), z);
+        const float2 r67 = fadd2(f2(__uint_as_float(__byte_perm(y, 0x4B000000u, 0x7542)),
+                                    __uint_as_float(__byte_perm(y, 0x4B000000u, 0x7543))), z);
         c[0] = r01.x; c[1] = r01.y; c[2] = r23.x; c[3] = r23.y;
         c[4] = r45.x; c[5] = r45.y; c[6] = r67.x; c[7] = r67.y;
     }
@@ -419,9 +416,10 @@ struct Shared {
     float tot_q[DV];
     float red_o[G::NWARPS * DV];
     float wred[2][G::NWARPS];
-    // per-row maxima of each 8-column block, column-block major: [DV/8][DK]
-    float rmax[DV / 8][DK];
-    float rmaxr[DV / 8][DK];       // of the yoked reference state
+    // per-row maxima of each 8-column block, column-block major; rows padded
+    // by 4 so the lanes of a warp (different column blocks) hit different banks
+    float rmax[DV / 8][DK + 4];
+    float rmaxr[DV / 8][DK + 4];   // of the yoked reference state
 };
 
 __device__ __forceinline__ float sgnf(float x) {
@@ -741,7 +739,8 @@ __device__ __forceinline__ void step_tile(const StepParams& p, long long tile, c
         for (int c = 0; c < 8; c++) po[c] = 0.0f;
 #pragma unroll
         for (int r = 0; r < 8; r++) {
-            float mm = 0.0f;
+            // max |x| of the row = max(max x, -min x): three-input max / min
+            float mx = 0.0f, mn = 0.0f;
             const float ur = urow(r), qr = row_in(sq, r);
 #pragma unroll
             for (int c = 0; c < 8; c += 2) {
@@ -749,13 +748,14 @@ __device__ __forceinline__ void step_tile(const StepParams& p, long long tile, c
                 const float2 o2 = ffma2(x2, f2(qr, qr), f2(po[c], po[c + 1]));
                 po[c] = o2.x;
                 po[c + 1] = o2.y;
-                mm = fmaxf(mm, fmaxf(fabsf(x2.x), fabsf(x2.y)));
+                mx = fmaxf(fmaxf(mx, x2.x), x2.y);
+                mn = fminf(fminf(mn, x2.x), x2.y);
                 if constexpr (!BDR) {        // the decayed state is not needed again
                     a[r][c] = x2.x;
                     a[r][c + 1] = x2.y;
                 }
             }
-            m[r] = mm;
+            m[r] = fmaxf(mx, -mn);
         }
 #pragma unroll
         for (int off = G::CBW; off < 32; off <<= 1) {
@@ -877,9 +877,15 @@ __device__ __forceinline__ void step_tile(const StepParams& p, long long tile, c
 #pragma unroll
             for (int c = 1; c < 8; c++) wmin = fminf(wmin, fabsf(wc[c]));
         }
+        if (group == 0) {
+            float mt = m[0];
+#pragma unroll
+            for (int r = 1; r < 8; r++) mt = fmaxf(mt, m[r]);
+            slow = !(__fmaf_rn(mt, inv[0], -(fq + 0.5f)) < 0.0f);
+        }
 #pragma unroll
         for (int r = 0; r < 8; r++) {
-            slow |= !(__fmaf_rn(m[r], inv[r], -(fq + 0.5f)) < 0.0f);
+            if (group != 0) slow |= !(__fmaf_rn(m[r], inv[r], -(fq + 0.5f)) < 0.0f);
             if constexpr (BDR) {
                 const float eta = __fmul_rn(al[r], dprev[r]);
                 const float floor_ = fmaxf(__fmul_rn(eta, float(1 << (BITS - 1)) * 0x1p-21f), 0x1p-120f);

@@ -183,21 +183,22 @@ BY_INDEX = {w.index: w for w in WORKLOADS.values()}
 
 
 def _draw16(seed, layer, step, tiles, field, n):
-    """uint16 draws [len(tiles), n] for one field."""
+    """uint16 draws [..., len(tiles), n] for one field; `step` may be an array
+    of steps (leading axis)."""
     tiles = np.asarray(tiles, np.uint32)
+    steps = np.atleast_1d(np.asarray(step, np.uint32))
     nchunk = (n + 7) // 8
     chunk = np.arange(nchunk, dtype=np.uint32)
-    c0 = np.uint32(step)
-    c1 = tiles[:, None]
-    c2 = np.uint32(field)
-    c3 = chunk[None, :]
-    w = philox4x32_10(np.full((1, 1), c0, np.uint32), c1, np.full((1, 1), c2, np.uint32), c3,
-                      np.uint32(seed & 0xFFFFFFFF), np.uint32(layer))
-    words = np.stack(w, axis=-1)                      # [T, nchunk, 4]
+    c0 = steps[:, None, None]
+    c1 = tiles[None, :, None]
+    c2 = np.full((1, 1, 1), field, np.uint32)
+    c3 = chunk[None, None, :]
+    w = philox4x32_10(c0, c1, c2, c3, np.uint32(seed & 0xFFFFFFFF), np.uint32(layer))
+    words = np.stack(w, axis=-1)                      # [S, T, nchunk, 4]
     lo = (words & np.uint32(0xFFFF)).astype(np.uint16)
     hi = (words >> np.uint32(16)).astype(np.uint16)
-    draws = np.stack([lo, hi], axis=-1).reshape(len(tiles), nchunk * 8)
-    return draws[:, :n]
+    draws = np.stack([lo, hi], axis=-1).reshape(len(steps), len(tiles), nchunk * 8)[..., :n]
+    return draws if np.ndim(step) else draws[0]
 
 
 def _normal(seed, layer, step, tiles, field, n, sigma):
@@ -209,10 +210,10 @@ def _normal(seed, layer, step, tiles, field, n, sigma):
 
 def _l2_normalised(z: np.ndarray) -> np.ndarray:
     """fp32: s = sum of squares in ascending order, then z / sqrt(s)."""
-    s = np.zeros(z.shape[0], np.float32)
-    for i in range(z.shape[1]):
-        s = s + z[:, i] * z[:, i]
-    return z / np.sqrt(s)[:, None]
+    s = np.zeros(z.shape[:-1], np.float32)
+    for i in range(z.shape[-1]):
+        s = s + z[..., i] * z[..., i]
+    return z / np.sqrt(s)[..., None]
 
 
 def _cast(x32: np.ndarray, dtype: int) -> np.ndarray:
@@ -242,9 +243,10 @@ class StepInputs:
                 f(self.gates, wl.gate_dtype))
 
 
-def gen_step(wl: Workload, step: int, layer: int = 0, tiles=None) -> StepInputs:
+def gen_step(wl: Workload, step, layer: int = 0, tiles=None) -> StepInputs:
     """Inputs of decode step ``step`` for the given tiles (default: all tiles
-    of one layer, tile = b * heads + h)."""
+    of one layer, tile = b * heads + h).  With an array of steps every field
+    gains a leading step axis (the values are those of the single steps)."""
     if tiles is None:
         tiles = np.arange(wl.tiles_per_layer)
     tiles = np.asarray(tiles)
@@ -267,7 +269,7 @@ def gen_step(wl: Workload, step: int, layer: int = 0, tiles=None) -> StepInputs:
         ua = _draw16(s, layer, step, tiles, FIELD_ALPHA, 1)
         ub = _draw16(s, layer, step, tiles, FIELD_BETA, 1)
         gates = np.concatenate([gate_table("gdn_alpha")[ua], gate_table("gdn_beta")[ub]],
-                               axis=1).astype(np.float32)
+                               axis=-1).astype(np.float32)
     if gates is not None:
         gates = _cast(gates, wl.gate_dtype)
     return StepInputs(_cast(q, wl.qkv_dtype), _cast(k, wl.qkv_dtype), _cast(v, wl.qkv_dtype),

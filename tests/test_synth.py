@@ -72,3 +72,19 @@ def test_mixed_head_bits_mean_four():
     hb = synth.WORKLOADS["gdn_b32_h16_d128_mixed_3modes"].head_bits()
     assert sorted(hb.tolist()) == [2] * 4 + [4] * 9 + [6] * 2 + [8]
     assert hb.mean() == 4.0
+
+
+@pytest.mark.parametrize("name", ["mamba2_b64_h32_dk128_dv64_int8tok", "gdn_b32_h16_d128_mixed_3modes",
+                                  "gla_b128_h16_d128_int4g32_persistent"])
+def test_multi_step_generation_matches_single_steps(name):
+    wl = synth.WORKLOADS[name]
+    tiles = np.arange(6)
+    many = synth.gen_step(wl, np.arange(10, 14), layer=2, tiles=tiles)
+    for i, s in enumerate(range(10, 14)):
+        one = synth.gen_step(wl, s, layer=2, tiles=tiles)
+        for f in ("q", "k", "v", "gates"):
+            a, b = getattr(many, f), getattr(one, f)
+            if b is None:
+                assert a is None
+            else:
+                assert np.array_equal(a[i], b), f
