@@ -36,6 +36,7 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
+#include <stddef.h>
 #include <stdint.h>
 
 namespace qs {
@@ -349,13 +350,11 @@ struct Pack6 {
 // ------------------------------------------------------------------ reductions
 // Column sums: p[8] holds this thread's canonical block sums (rows i0..i0+7)
 // for its columns j0..j0+7.  Adjacent row blocks of the warp are joined by the
-// xor butterfly over offsets CBW, 2*CBW, ..; warps by a pairwise tree.  When
-// `broadcast`, every thread gets its 8 column totals in res; otherwise the
-// totals are written to dst[j] (threads j < DV) and res is untouched.
+// xor butterfly over offsets CBW, 2*CBW, ..; warps by a pairwise tree.  Every
+// thread gets its 8 column totals in res.
 template <int DK, int DV>
 __device__ __forceinline__ void colsum_finish(float (&p)[8], float* red, float* tot, int warp,
-                                              int rbl, int j0, bool broadcast, float (&res)[8],
-                                              float* dst) {
+                                              int rbl, int j0, float (&res)[8]) {
     using G = Geo<DK, DV>;
 #pragma unroll
     for (int off = G::CBW; off < 32; off <<= 1) {
@@ -377,16 +376,26 @@ __device__ __forceinline__ void colsum_finish(float (&p)[8], float* red, float* 
 #pragma unroll
             for (int u = 0; u < n / 2; u++) t[u] = __fadd_rn(t[2 * u], t[2 * u + 1]);
         }
-        if (broadcast) tot[threadIdx.x] = t[0];
-        else dst[threadIdx.x] = t[0];
+        tot[threadIdx.x] = t[0];
     }
-    if (broadcast) {
-        __syncthreads();
-        const float4 a = reinterpret_cast<const float4*>(tot + j0)[0];
-        const float4 b = reinterpret_cast<const float4*>(tot + j0)[1];
-        res[0] = a.x; res[1] = a.y; res[2] = a.z; res[3] = a.w;
-        res[4] = b.x; res[5] = b.y; res[6] = b.z; res[7] = b.w;
-    }
+    __syncthreads();
+    const float4 a = reinterpret_cast<const float4*>(tot + j0)[0];
+    const float4 b = reinterpret_cast<const float4*>(tot + j0)[1];
+    res[0] = a.x; res[1] = a.y; res[2] = a.z; res[3] = a.w;
+    res[4] = b.x; res[5] = b.y; res[6] = b.z; res[7] = b.w;
+}
+
+// ------------------------------------------------------------------ scales
+// m / Qmax correctly rounded, for m >= 0 finite or +inf and rq = RN(1 / Qmax):
+// a product with the rounded reciprocal, then one correction by the exact
+// remainder (Markstein's scheme for division by a constant).  For every
+// non-negative binary32 m and Qmax in {1, 7, 31, 127} the result equals the
+// IEEE quotient bit for bit; +inf (remainder NaN) keeps the product.
+__device__ __forceinline__ float div_by_qmax(float m, float qmax, float rq) {
+    const float q0 = __fmul_rn(m, rq);
+    const float r = __fmaf_rn(-q0, qmax, m);
+    const float q1 = __fmaf_rn(r, rq, q0);
+    return r != r ? q0 : q1;
 }
 
 // ------------------------------------------------------------------ rounding
@@ -407,19 +416,40 @@ __device__ __forceinline__ float bdr1(float t, float s, float d, float eps) {
 }
 
 // ------------------------------------------------------------------ shared state
-template <int DK, int DV>
-struct Shared {
+// Partials that a tile writes before its exchange barrier and reads after it.
+// They are double-buffered by tile parity: a CTA has one barrier per tile, so
+// the next tile may write its partials while a slower warp still reads these.
+template <int DK, int DV, bool YOKED>
+struct __align__(16) Xchg {
     using G = Geo<DK, DV>;
-    float red_r[G::NWARPS * DV];
-    float tot_r[DV];
-    float red_q[G::NWARPS * DV];   // reference-state column sums (yoked GDN)
-    float tot_q[DV];
     float red_o[G::NWARPS * DV];
     float wred[2][G::NWARPS];
     // per-row maxima of each 8-column block, column-block major; rows padded
     // by 4 so the lanes of a warp (different column blocks) hit different banks
     float rmax[DV / 8][DK + 4];
-    float rmaxr[DV / 8][DK + 4];   // of the yoked reference state
+    float rmaxr[YOKED ? DV / 8 : 1][DK + 4];   // of the yoked reference state
+};
+
+template <int DK, int DV, bool GDN, bool YOKED>
+struct __align__(16) Shared {
+    using G = Geo<DK, DV>;
+    // Gated DeltaNet column sums r = a^T k, used before the exchange barrier
+    // only; the yoked reference state's sums use them first (the two sums are
+    // separated by the barriers inside each)
+    float red_r[GDN ? G::NWARPS * DV : 4];
+    float tot_r[GDN ? DV : 4];
+    Xchg<DK, DV, YOKED> x[2];
+};
+// the partials are written and read as float4: every array starts on 16 bytes
+template <int DK, int DV, bool GDN, bool YOKED>
+struct SharedLayoutCheck {
+    using X = Xchg<DK, DV, YOKED>;
+    using S = Shared<DK, DV, GDN, YOKED>;
+    static_assert(offsetof(X, red_o) % 16 == 0 && offsetof(X, rmax) % 16 == 0 &&
+                  offsetof(X, rmaxr) % 16 == 0 && sizeof(X) % 16 == 0, "exchange layout");
+    static_assert(offsetof(S, red_r) % 16 == 0 && offsetof(S, tot_r) % 16 == 0 &&
+                  offsetof(S, x) % 16 == 0, "shared layout");
+    static constexpr bool ok = true;
 };
 
 __device__ __forceinline__ float sgnf(float x) {
@@ -526,8 +556,8 @@ __device__ __forceinline__ void round_pack_fast(const float (&a)[8][8], URow uro
 // block are in shared memory; lane lp of a group derives the scales of
 // rows lp*nv .. lp*nv + nv - 1 of its row block (nv = 8 / min(L, 8)), stores
 // them, and the reciprocals go back to the group's lanes with shuffles.
-template <int DK, int DV, int L, class NewScale, class PrevScale>
-__device__ __forceinline__ void group_scales(int cb, int lane, int i0, const Shared<DK, DV>& sh,
+template <int DK, int DV, int L, class X, class NewScale, class PrevScale>
+__device__ __forceinline__ void group_scales(int cb, int lane, int i0, const X& sh,
                                              bool yoked, float (&inv)[8], unsigned& nsat,
                                              bool& bad, NewScale new_scale, PrevScale prev_scale,
                                              const StepParams& p, long long sbase, int ng, int gcol) {
@@ -568,11 +598,18 @@ __device__ __forceinline__ void group_scales(int cb, int lane, int i0, const Sha
 // ------------------------------------------------------------------ one tile
 // st: the tile's shared-memory stage; ct: its codes in global memory.
 // g0, g1: scalar gates (alpha, beta) and pts: per-token previous scale,
-// prefetched by the caller.
-template <int DK, int DV, int BITS, bool GDN, bool YOKED, bool BDR, bool BF>
-__device__ __forceinline__ void step_tile(const StepParams& p, long long tile, const uint8_t* st,
+// prefetched by the caller.  ok: this thread's stage arrived.  Without the delta
+// rule the tile has one CTA barrier, the exchange of output partials and
+// maxima; it votes on ok (false is returned by every thread, before any global
+// write of the tile, when one of them gave up) and at_barrier() runs right
+// after it.  Gated DeltaNet tiles vote at a barrier of their own at the top
+// (the caller's), before their column sums.
+template <int DK, int DV, int BITS, bool GDN, bool YOKED, bool BDR, bool BF, class AtBarrier>
+__device__ __forceinline__ bool step_tile(const StepParams& p, long long tile, const uint8_t* st,
                                           uint8_t* ct, float g0, float g1, float pts,
-                                          Shared<DK, DV>& sh, volatile int* badflag) {
+                                          Shared<DK, DV, GDN, YOKED>& sh,
+                                          Xchg<DK, DV, YOKED>& xs, volatile int* badflag,
+                                          bool ok, AtBarrier at_barrier) {
     using G = Geo<DK, DV>;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int cb = lane % G::CBW, rbl = lane / G::CBW;
@@ -646,7 +683,7 @@ __device__ __forceinline__ void step_tile(const StepParams& p, long long tile, c
                     pr[c] = v2.x;
                     pr[c + 1] = v2.y;
                 }
-            colsum_finish<DK, DV>(pr, sh.red_q, sh.tot_q, warp, rbl, j0, true, e2, nullptr);
+            colsum_finish<DK, DV>(pr, sh.red_r, sh.tot_r, warp, rbl, j0, e2);
 #pragma unroll
             for (int c = 0; c < 8; c++) e2[c] = __fsub_rn(vv[c], e2[c]);
         }
@@ -665,9 +702,11 @@ __device__ __forceinline__ void step_tile(const StepParams& p, long long tile, c
                 ar[r][c + 1] = v2.y;
                 mm = fmaxf(mm, fmaxf(fabsf(v2.x), fabsf(v2.y)));
             }
-            float4* dst = reinterpret_cast<float4*>(gref + (i0 + r) * DV + j0);
-            dst[0] = make_float4(ar[r][0], ar[r][1], ar[r][2], ar[r][3]);
-            dst[1] = make_float4(ar[r][4], ar[r][5], ar[r][6], ar[r][7]);
+            if (ok) {       // a stage that did not arrive leaves the state alone
+                float4* dst = reinterpret_cast<float4*>(gref + (i0 + r) * DV + j0);
+                dst[0] = make_float4(ar[r][0], ar[r][1], ar[r][2], ar[r][3]);
+                dst[1] = make_float4(ar[r][4], ar[r][5], ar[r][6], ar[r][7]);
+            }
             mref[r] = mm;
         }
     }
@@ -720,7 +759,7 @@ __device__ __forceinline__ void step_tile(const StepParams& p, long long tile, c
                 pr[c] = v2.x;
                 pr[c + 1] = v2.y;
             }
-        colsum_finish<DK, DV>(pr, sh.red_r, sh.tot_r, warp, rbl, j0, true, wc, nullptr);
+        colsum_finish<DK, DV>(pr, sh.red_r, sh.tot_r, warp, rbl, j0, wc);
 #pragma unroll
         for (int c = 0; c < 8; c++) wc[c] = __fsub_rn(vv[c], wc[c]);       // e = v - r
     } else {
@@ -739,8 +778,7 @@ __device__ __forceinline__ void step_tile(const StepParams& p, long long tile, c
         for (int c = 0; c < 8; c++) po[c] = 0.0f;
 #pragma unroll
         for (int r = 0; r < 8; r++) {
-            // max |x| of the row = max(max x, -min x): three-input max / min
-            float mx = 0.0f, mn = 0.0f;
+            float mx = 0.0f;     // max |x| of the row (three-input max)
             const float ur = urow(r), qr = row_in(sq, r);
 #pragma unroll
             for (int c = 0; c < 8; c += 2) {
@@ -748,14 +786,13 @@ __device__ __forceinline__ void step_tile(const StepParams& p, long long tile, c
                 const float2 o2 = ffma2(x2, f2(qr, qr), f2(po[c], po[c + 1]));
                 po[c] = o2.x;
                 po[c + 1] = o2.y;
-                mx = fmaxf(fmaxf(mx, x2.x), x2.y);
-                mn = fminf(fminf(mn, x2.x), x2.y);
+                mx = fmaxf(fmaxf(mx, fabsf(x2.x)), fabsf(x2.y));
                 if constexpr (!BDR) {        // the decayed state is not needed again
                     a[r][c] = x2.x;
                     a[r][c + 1] = x2.y;
                 }
             }
-            m[r] = fmaxf(mx, -mn);
+            m[r] = mx;
         }
 #pragma unroll
         for (int off = G::CBW; off < 32; off <<= 1) {
@@ -763,36 +800,40 @@ __device__ __forceinline__ void step_tile(const StepParams& p, long long tile, c
             for (int c = 0; c < 8; c++) po[c] = __fadd_rn(po[c], __shfl_xor_sync(0xFFFFFFFFu, po[c], off));
         }
         if (rbl == 0) {
-            float4* r4 = reinterpret_cast<float4*>(sh.red_o + warp * DV + j0);
+            float4* r4 = reinterpret_cast<float4*>(xs.red_o + warp * DV + j0);
             r4[0] = make_float4(po[0], po[1], po[2], po[3]);
             r4[1] = make_float4(po[4], po[5], po[6], po[7]);
         }
         if (group != 0 && BITS != 32) {
-            float4* r4 = reinterpret_cast<float4*>(&sh.rmax[cb][i0]);
+            float4* r4 = reinterpret_cast<float4*>(&xs.rmax[cb][i0]);
             r4[0] = make_float4(m[0], m[1], m[2], m[3]);
             r4[1] = make_float4(m[4], m[5], m[6], m[7]);
             if (YOKED) {
-                float4* q4 = reinterpret_cast<float4*>(&sh.rmaxr[cb][i0]);
+                float4* q4 = reinterpret_cast<float4*>(&xs.rmaxr[cb][i0]);
                 q4[0] = make_float4(mref[0], mref[1], mref[2], mref[3]);
                 q4[1] = make_float4(mref[4], mref[5], mref[6], mref[7]);
             }
         }
         if (group == 0 && BITS != 32) {
+            // the maxima are non-negative and never NaN (fmaxf drops NaN), so
+            // their bit patterns order like the values: one integer warp max
             float t = m[0], tr = mref[0];
 #pragma unroll
             for (int r = 1; r < 8; r++) { t = fmaxf(t, m[r]); tr = fmaxf(tr, mref[r]); }
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                t = fmaxf(t, __shfl_xor_sync(0xFFFFFFFFu, t, off));
-                if (YOKED) tr = fmaxf(tr, __shfl_xor_sync(0xFFFFFFFFu, tr, off));
-            }
-            if (lane == 0) { sh.wred[0][warp] = t; sh.wred[1][warp] = tr; }
+            t = __uint_as_float(__reduce_max_sync(0xFFFFFFFFu, __float_as_uint(t)));
+            if (YOKED) tr = __uint_as_float(__reduce_max_sync(0xFFFFFFFFu, __float_as_uint(tr)));
+            if (lane == 0) { xs.wred[0][warp] = t; xs.wred[1][warp] = tr; }
         }
-        __syncthreads();
+        if constexpr (GDN) {
+            __syncthreads();     // the vote was taken at the top of the tile
+        } else {
+            if (!__syncthreads_and(ok)) return false;
+            at_barrier();
+        }
         if (threadIdx.x < DV) {
             float t[G::NWARPS];
 #pragma unroll
-            for (int w2 = 0; w2 < G::NWARPS; w2++) t[w2] = sh.red_o[w2 * DV + threadIdx.x];
+            for (int w2 = 0; w2 < G::NWARPS; w2++) t[w2] = xs.red_o[w2 * DV + threadIdx.x];
 #pragma unroll
             for (int n = G::NWARPS; n > 1; n >>= 1) {
 #pragma unroll
@@ -802,12 +843,12 @@ __device__ __forceinline__ void step_tile(const StepParams& p, long long tile, c
             if (BITS != 32 && !isfinite(t[0])) *badflag = 1;
         }
         if (group == 0 && BITS != 32) {
-            tmax = sh.wred[0][0];
-            tref = sh.wred[1][0];
+            tmax = xs.wred[0][0];
+            tref = xs.wred[1][0];
 #pragma unroll
             for (int w2 = 1; w2 < G::NWARPS; w2++) {
-                tmax = fmaxf(tmax, sh.wred[0][w2]);
-                tref = fmaxf(tref, sh.wred[1][w2]);
+                tmax = fmaxf(tmax, xs.wred[0][w2]);
+                tref = fmaxf(tref, xs.wred[1][w2]);
             }
         }
     }
@@ -830,27 +871,30 @@ __device__ __forceinline__ void step_tile(const StepParams& p, long long tile, c
             dst[0] = make_float4(x8[0], x8[1], x8[2], x8[3]);
             dst[1] = make_float4(x8[4], x8[5], x8[6], x8[7]);
         }
-        return;
+        return true;
     } else {
         // ---- 4. scales
         const float fq = float(QMAX);
+        // RN(1 / Qmax) for Qmax = 1, 7, 31, 127
+        constexpr float rq = QMAX == 7 ? 0x1.24924ap-3f : QMAX == 31 ? 0x1.08421p-5f
+                           : QMAX == 127 ? 0x1.020408p-7f : 1.0f;
         float inv[8];
         unsigned nsat = 0;
         auto new_scale = [&](float mm, float mr, float dp, bool& sat) -> float {
             sat = false;
-            if constexpr (YOKED) return to_stored(__fdiv_rn(mr, fq), sf32, sat);
+            if constexpr (YOKED) return to_stored(div_by_qmax(mr, fq, rq), sf32, sat);
             if (p.scale_mode == M_PERSISTENT)
-                return (mm > __fmul_rn(fq, dp)) ? to_stored(__fdiv_rn(mm, fq), sf32, sat) : dp;
-            return to_stored(__fdiv_rn(mm, fq), sf32, sat);
+                return (mm > __fmul_rn(fq, dp)) ? to_stored(div_by_qmax(mm, fq, rq), sf32, sat) : dp;
+            return to_stored(div_by_qmax(mm, fq, rq), sf32, sat);
         };
         bool bad = false;
         if (group) {
             switch (group / 8) {
-                case 1: group_scales<DK, DV, 1>(cb, lane, i0, sh, YOKED, inv, nsat, bad, new_scale, prev_scale, p, sbase, ng, gcol); break;
-                case 2: group_scales<DK, DV, 2>(cb, lane, i0, sh, YOKED, inv, nsat, bad, new_scale, prev_scale, p, sbase, ng, gcol); break;
-                case 4: group_scales<DK, DV, 4>(cb, lane, i0, sh, YOKED, inv, nsat, bad, new_scale, prev_scale, p, sbase, ng, gcol); break;
-                case 8: group_scales<DK, DV, 8>(cb, lane, i0, sh, YOKED, inv, nsat, bad, new_scale, prev_scale, p, sbase, ng, gcol); break;
-                default: group_scales<DK, DV, 16>(cb, lane, i0, sh, YOKED, inv, nsat, bad, new_scale, prev_scale, p, sbase, ng, gcol); break;
+                case 1: group_scales<DK, DV, 1>(cb, lane, i0, xs, YOKED, inv, nsat, bad, new_scale, prev_scale, p, sbase, ng, gcol); break;
+                case 2: group_scales<DK, DV, 2>(cb, lane, i0, xs, YOKED, inv, nsat, bad, new_scale, prev_scale, p, sbase, ng, gcol); break;
+                case 4: group_scales<DK, DV, 4>(cb, lane, i0, xs, YOKED, inv, nsat, bad, new_scale, prev_scale, p, sbase, ng, gcol); break;
+                case 8: group_scales<DK, DV, 8>(cb, lane, i0, xs, YOKED, inv, nsat, bad, new_scale, prev_scale, p, sbase, ng, gcol); break;
+                default: group_scales<DK, DV, 16>(cb, lane, i0, xs, YOKED, inv, nsat, bad, new_scale, prev_scale, p, sbase, ng, gcol); break;
             }
         } else {
             bool sat;
@@ -900,6 +944,7 @@ __device__ __forceinline__ void step_tile(const StepParams& p, long long tile, c
         // a tile-step is counted once if an output or a group maximum was not
         // finite (the flag is collected at the next tile's barrier)
         if (bad) *badflag = 1;
+        return true;
     }
 }
 
@@ -982,7 +1027,8 @@ template <int DK, int DV, int BITS, bool GDN, bool YOKED, bool BDR, bool BF>
 __global__ void __launch_bounds__(Geo<DK, DV>::NT, (Occupancy<DK, DV, YOKED>::MIN_BLOCKS))
 step_kernel(const StepParams p) {
     extern __shared__ __align__(128) uint8_t dsmem[];
-    __shared__ Shared<DK, DV> sh;
+    static_assert(SharedLayoutCheck<DK, DV, GDN, YOKED>::ok, "");
+    __shared__ Shared<DK, DV, GDN, YOKED> sh;
     __shared__ __align__(8) uint64_t bars[kMaxStages];
     __shared__ volatile int badf[2];
     const int S = p.nstages;
@@ -1009,10 +1055,55 @@ step_kernel(const StepParams p) {
         float n0, n1, nts;
         load_scalars(p, tile + gridDim.x, n0, n1, nts);    // next tile's scalars
         const bool ok = mbar_wait_bounded(&bars[s], parity, p.wait_polls);
-        // One barrier per tile: every thread has its stage (or has given up),
-        // and every thread has finished the previous tile, so its stage and the
-        // shared reduction buffers are free again.
-        if (!__syncthreads_and(ok)) {
+        // At this tile's first barrier every thread has finished the previous
+        // tile: its stage is refilled with the tile S strides ahead of it, and
+        // its non-finite flag is complete.  Without the delta rule that is the
+        // exchange barrier inside step_tile; Gated DeltaNet, whose column sums
+        // come first, takes a barrier here and refills one phase earlier.
+        auto at_barrier = [&]() {
+            if (threadIdx.x == 0 && it > 0) {
+                if (badf[(it - 1) & 1]) {
+                    badf[(it - 1) & 1] = 0;
+                    atomicAdd(p.counters, 1ull);
+                }
+                const long long nt = tile + (long long)(S - 1) * gridDim.x;
+                const int sp = (it - 1) % S;
+                if (nt < p.ntiles) issue_tile<DK, DV, YOKED>(p, nt, dsmem + sp * p.stage_bytes, &bars[sp]);
+            }
+        };
+        const uint8_t* st = dsmem + s * p.stage_bytes;
+        auto& xs = sh.x[it & 1];
+        volatile int* bf = &badf[it & 1];
+        uint8_t* ct;
+        int bits;
+        uint32_t cbytes;
+        tile_codes(p, tile, ct, bits, cbytes, DK, DV);
+        auto run_tile = [&](bool okv, auto& hook) -> bool {
+            if constexpr (BITS == 0) {
+                switch (bits) {
+                    case 2: return step_tile<DK, DV, 2, GDN, YOKED, BDR, BF>(p, tile, st, ct, g0, g1, pts, sh, xs, bf, okv, hook);
+                    case 4: return step_tile<DK, DV, 4, GDN, YOKED, BDR, BF>(p, tile, st, ct, g0, g1, pts, sh, xs, bf, okv, hook);
+                    case 6: return step_tile<DK, DV, 6, GDN, YOKED, BDR, BF>(p, tile, st, ct, g0, g1, pts, sh, xs, bf, okv, hook);
+                    default: return step_tile<DK, DV, 8, GDN, YOKED, BDR, BF>(p, tile, st, ct, g0, g1, pts, sh, xs, bf, okv, hook);
+                }
+            } else {
+                (void)bits;
+                return step_tile<DK, DV, BITS, GDN, YOKED, BDR, BF>(p, tile, st, ct, g0, g1, pts, sh, xs, bf, okv, hook);
+            }
+        };
+        bool done;
+        if constexpr (GDN) {
+            done = __syncthreads_and(ok);
+            if (done) {
+                at_barrier();
+                auto no_op = []() {};
+                run_tile(true, no_op);
+            }
+        } else {
+            done = run_tile(ok, at_barrier);
+        }
+        if (!done) {
+            // some thread gave up on this tile's stage (the vote is uniform)
             if (threadIdx.x == 0) {
                 atomicAdd(p.counters + 2, 1ull);
                 // drain this CTA's copies still in flight (tiles it .. it+S-1
@@ -1026,32 +1117,6 @@ step_kernel(const StepParams p) {
                 }
             }
             return;
-        }
-        if (threadIdx.x == 0 && it > 0 && badf[(it - 1) & 1]) {
-            badf[(it - 1) & 1] = 0;
-            atomicAdd(p.counters, 1ull);
-        }
-        if (threadIdx.x == 0 && it > 0) {
-            // refill the previous tile's stage with the tile S strides ahead of it
-            const long long nt = tile + (long long)(S - 1) * gridDim.x;
-            const int sp = (it - 1) % S;
-            if (nt < p.ntiles) issue_tile<DK, DV, YOKED>(p, nt, dsmem + sp * p.stage_bytes, &bars[sp]);
-        }
-        uint8_t* st = dsmem + s * p.stage_bytes;
-        uint8_t* ct;
-        int bits;
-        uint32_t cbytes;
-        tile_codes(p, tile, ct, bits, cbytes, DK, DV);
-        if constexpr (BITS == 0) {
-            switch (bits) {
-                case 2: step_tile<DK, DV, 2, GDN, YOKED, BDR, BF>(p, tile, st, ct, g0, g1, pts, sh, &badf[it & 1]); break;
-                case 4: step_tile<DK, DV, 4, GDN, YOKED, BDR, BF>(p, tile, st, ct, g0, g1, pts, sh, &badf[it & 1]); break;
-                case 6: step_tile<DK, DV, 6, GDN, YOKED, BDR, BF>(p, tile, st, ct, g0, g1, pts, sh, &badf[it & 1]); break;
-                default: step_tile<DK, DV, 8, GDN, YOKED, BDR, BF>(p, tile, st, ct, g0, g1, pts, sh, &badf[it & 1]); break;
-            }
-        } else {
-            (void)bits;
-            step_tile<DK, DV, BITS, GDN, YOKED, BDR, BF>(p, tile, st, ct, g0, g1, pts, sh, &badf[it & 1]);
         }
         g0 = n0;
         g1 = n1;
