@@ -153,6 +153,7 @@ int qstate_create(const qstate_layout* L, int bits, int group, qstate_scale_mode
     if (!L || !out) return QSTATE_EINVAL;
     *out = nullptr;
     if (L->batch < 0 || L->heads < 1 || L->layers < 1) return QSTATE_EINVAL;
+    if ((int64_t)L->layers * L->batch * L->heads > INT32_MAX) return QSTATE_EINVAL;
     if (L->d_k < 8 || L->d_v < 8 || L->d_k % 8 || L->d_v % 8) return QSTATE_EINVAL;
     if (L->kind < QSTATE_RETNET || L->kind > QSTATE_GDN) return QSTATE_EINVAL;
     if (L->qkv_dtype != QSTATE_F32 && L->qkv_dtype != QSTATE_BF16) return QSTATE_EINVAL;

@@ -192,34 +192,33 @@ __device__ __forceinline__ float2 fmul2(float2 a, float2 b) { return __fmul2_rn(
 __device__ __forceinline__ float2 fadd2(float2 a, float2 b) { return __fadd2_rn(a, b); }
 
 // ------------------------------------------------------------------ code decode
-// Exact float code values c[8] of one thread's 8 codes of a row.  A field
-// masked into place and XORed with 0x4B000000 plus its sign bit is the float
-// 2^23 + (field ^ signbit) * 2^pos; one fma scales by 2^-pos and removes the
-// bias exactly.
+// Exact float code values c[8] of one thread's 8 codes of a row.  A code with
+// its sign bit flipped is an unsigned field u = code + 2^(b-1); placed in the
+// low byte of the float 2^23 (byte permute) it gives 2^23 + u exactly, and one
+// add removes the bias.  Narrow fields that do not sit in bytes of their own
+// are masked into place and XORed with 0x4B000000 plus their sign bit instead,
+// giving 2^23 + u * 2^pos; one fma then scales by 2^-pos and removes the bias.
 template <int BITS>
 struct Decode;
 
 template <>
 struct Decode<4> {
+    // byte m holds codes 2m (low nibble) and 2m+1 (high nibble): the two
+    // nibble planes are split into bytes of their own
     static __device__ __forceinline__ void run(const uint8_t* row, int cb, float (&c)[8]) {
-        const uint32_t w = *reinterpret_cast<const uint32_t*>(row + cb * 4);
-        const uint32_t h = w >> 12;
-        const float f0 = __uint_as_float((w & 0xFu) ^ 0x4B000008u);
-        const float f1 = __uint_as_float((w & 0xF0u) ^ 0x4B000080u);
-        const float f2_ = __uint_as_float((w & 0xF00u) ^ 0x4B000800u);
-        const float f3 = __uint_as_float((w & 0xF000u) ^ 0x4B008000u);
-        const float f4 = __uint_as_float((w & 0xF0000u) ^ 0x4B080000u);
-        const float f5 = __uint_as_float((h & 0xF00u) ^ 0x4B000800u);
-        const float f6 = __uint_as_float((h & 0xF000u) ^ 0x4B008000u);
-        const float f7 = __uint_as_float((h & 0xF0000u) ^ 0x4B080000u);
-        // pos 0 / 4 :  scale 1 / 2^-4,   bias 2^23 + 8 / 2^19 + 8
-        float2 r01 = ffma2(f2(f0, f1), f2(1.0f, 0x1p-4f), f2(-8388616.0f, -524296.0f));
-        // pos 8 (codes 2 and 5), 12 (3 and 6), 16 (4 and 7)
-        float2 r25 = ffma2(f2(f2_, f5), f2(0x1p-8f, 0x1p-8f), f2(-32776.0f, -32776.0f));
-        float2 r36 = ffma2(f2(f3, f6), f2(0x1p-12f, 0x1p-12f), f2(-2056.0f, -2056.0f));
-        float2 r47 = ffma2(f2(f4, f7), f2(0x1p-16f, 0x1p-16f), f2(-136.0f, -136.0f));
-        c[0] = r01.x; c[1] = r01.y; c[2] = r25.x; c[5] = r25.y;
-        c[3] = r36.x; c[6] = r36.y; c[4] = r47.x; c[7] = r47.y;
+        const uint32_t w = *reinterpret_cast<const uint32_t*>(row + cb * 4) ^ 0x88888888u;
+        const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;
+        const float2 z = f2(-8388616.0f, -8388616.0f);   // -(2^23 + 8)
+        const float2 r01 = fadd2(f2(__uint_as_float(__byte_perm(lo, 0x4B000000u, 0x7540)),
+                                    __uint_as_float(__byte_perm(hi, 0x4B000000u, 0x7540))), z);
+        const float2 r23 = fadd2(f2(__uint_as_float(__byte_perm(lo, 0x4B000000u, 0x7541)),
+                                    __uint_as_float(__byte_perm(hi, 0x4B000000u, 0x7541))), z);
+        const float2 r45 = fadd2(f2(__uint_as_float(__byte_perm(lo, 0x4B000000u, 0x7542)),
+                                    __uint_as_float(__byte_perm(hi, 0x4B000000u, 0x7542))), z);
+        const float2 r67 = fadd2(f2(__uint_as_float(__byte_perm(lo, 0x4B000000u, 0x7543)),
+                                    __uint_as_float(__byte_perm(hi, 0x4B000000u, 0x7543))), z);
+        c[0] = r01.x; c[1] = r01.y; c[2] = r23.x; c[3] = r23.y;
+        c[4] = r45.x; c[5] = r45.y; c[6] = r67.x; c[7] = r67.y;
     }
 };
 
@@ -641,9 +640,11 @@ __device__ __forceinline__ bool step_tile(const StepParams& p, long long tile, c
     // k, v or the gates reaches the output o or a group maximum (0 * inf and
     // inf - inf are NaN), where it is counted.
 
-    const int ng = group ? DV / group : 1;
+    // group is a power of two (8 .. 128) dividing d_v
+    const int gsh = group ? __ffs(group) - 1 : 0;
+    const int ng = group ? DV >> gsh : 1;
     const long long sbase = tile * (long long)p.n_scales;
-    const int gcol = group ? j0 / group : 0;
+    const int gcol = group ? j0 >> gsh : 0;
     auto prev_scale = [&](int row) -> float {
         if (!group) return pts;
         const int idx = row * ng + gcol;
@@ -952,9 +953,11 @@ __device__ __forceinline__ bool step_tile(const StepParams& p, long long tile, c
 __device__ __forceinline__ void tile_codes(const StepParams& p, long long tile, uint8_t*& ptr,
                                            int& bits, uint32_t& bytes, int dk, int dv) {
     if (p.head_bits) {
-        const int h = int(tile % p.heads);
+        // tile counts fit 31 bits (checked at creation): 32-bit division
+        const uint32_t t32 = uint32_t(tile), hd = uint32_t(p.heads);
+        const uint32_t row = t32 / hd, h = t32 - row * hd;
         bits = p.head_bits[h];
-        ptr = p.codes + (tile / p.heads) * p.row_bytes + p.head_off[h];
+        ptr = p.codes + (long long)row * p.row_bytes + p.head_off[h];
     } else {
         bits = p.bits;
         ptr = p.codes + tile * p.tile_bytes;
@@ -1008,7 +1011,7 @@ __device__ __forceinline__ void load_scalars(const StepParams& p, long long tile
     if (p.kind == K_MAMBA2 || p.kind == K_GDN) g0 = ldg1(p.gates, tile * p.n_gate, p.gate_bf16 != 0);
     if (p.kind == K_GDN) g1 = ldg1(p.gates, tile * p.n_gate + 1, p.gate_bf16 != 0);
     if (p.group == 0) {
-        int bits = p.head_bits ? p.head_bits[tile % p.heads] : p.bits;
+        int bits = p.head_bits ? p.head_bits[uint32_t(tile) % uint32_t(p.heads)] : p.bits;
         if (bits != 32) pts = scale_at(p.scales, tile, p.scale_f32 != 0);
     }
 }
@@ -1049,9 +1052,9 @@ step_kernel(const StepParams p) {
     load_scalars(p, blockIdx.x, g0, g1, pts);
 
     int it = 0;
+    int s = 0;                 // stage of tile it = it % S
+    uint32_t parity = 0;       // its barrier phase = (it / S) & 1
     for (long long tile = blockIdx.x; tile < p.ntiles; tile += gridDim.x, it++) {
-        const int s = it % S;
-        const uint32_t parity = (it / S) & 1;
         float n0, n1, nts;
         load_scalars(p, tile + gridDim.x, n0, n1, nts);    // next tile's scalars
         const bool ok = mbar_wait_bounded(&bars[s], parity, p.wait_polls);
@@ -1067,7 +1070,7 @@ step_kernel(const StepParams p) {
                     atomicAdd(p.counters, 1ull);
                 }
                 const long long nt = tile + (long long)(S - 1) * gridDim.x;
-                const int sp = (it - 1) % S;
+                const int sp = s == 0 ? S - 1 : s - 1;     // stage of tile it - 1
                 if (nt < p.ntiles) issue_tile<DK, DV, YOKED>(p, nt, dsmem + sp * p.stage_bytes, &bars[sp]);
             }
         };
@@ -1121,6 +1124,10 @@ step_kernel(const StepParams p) {
         g0 = n0;
         g1 = n1;
         pts = nts;
+        if (++s == S) {
+            s = 0;
+            parity ^= 1u;
+        }
     }
     __syncthreads();
     if (threadIdx.x == 0 && it > 0 && badf[(it - 1) & 1]) atomicAdd(p.counters, 1ull);

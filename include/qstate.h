@@ -107,7 +107,8 @@ typedef struct qstate_layout {
     int32_t batch;            /* >= 0 (0: an empty object, steps are no-ops) */
     int32_t heads;            /* >= 1 */
     int32_t d_k, d_v;         /* each 64 or 128 */
-    int32_t layers;           /* independent layers held by the object, >= 1 */
+    int32_t layers;           /* independent layers held by the object, >= 1;
+                                 layers * batch * heads < 2^31 */
     int32_t kind;             /* qstate_kind */
     float gamma;              /* RetNet decay (ignored for the other kinds) */
     int32_t qkv_dtype;        /* QSTATE_F32 or QSTATE_BF16 */

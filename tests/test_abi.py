@@ -62,6 +62,7 @@ def _layout(q, **kw):
     (dict(qkv_dtype=2), dict(bits=4)),
     (dict(scale_dtype=1), dict(bits=4)),
     (dict(kind=0, gamma=float("inf")), dict(bits=4)),
+    (dict(batch=1 << 20, heads=1 << 8, layers=8), dict(bits=4)),   # 2^31 tiles
 ])
 def test_create_rejects_invalid(q, kw, args):
     L = _layout(q, **kw)
