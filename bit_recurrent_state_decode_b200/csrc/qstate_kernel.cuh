@@ -288,18 +288,15 @@ struct Pack;
 
 template <>
 struct Pack<4> {
-    // byte m = nibble of code 2m | nibble of code 2m+1 << 4, then the low bytes
-    // of the four pairs gathered into one word
+    // the low bytes of the even codes and of the odd codes are gathered into
+    // one word each; byte m = low nibble of code 2m | low nibble of code 2m+1 << 4
     static __device__ __forceinline__ void run(uint8_t* row, int cb, const float (&t)[8]) {
-        uint32_t b[4];
-#pragma unroll
-        for (int m = 0; m < 4; m++) {
-            const uint32_t lo = __float_as_uint(t[2 * m]), hi = __float_as_uint(t[2 * m + 1]) << 4;
-            b[m] = (lo & 0x0Fu) | (hi & ~0x0Fu);
-        }
-        const uint32_t w01 = __byte_perm(b[0], b[1], 0x0040);
-        const uint32_t w23 = __byte_perm(b[2], b[3], 0x0040);
-        *reinterpret_cast<uint32_t*>(row + cb * 4) = __byte_perm(w01, w23, 0x5410);
+        const uint32_t e01 = __byte_perm(__float_as_uint(t[0]), __float_as_uint(t[2]), 0x0040);
+        const uint32_t e23 = __byte_perm(__float_as_uint(t[4]), __float_as_uint(t[6]), 0x0040);
+        const uint32_t o01 = __byte_perm(__float_as_uint(t[1]), __float_as_uint(t[3]), 0x0040);
+        const uint32_t o23 = __byte_perm(__float_as_uint(t[5]), __float_as_uint(t[7]), 0x0040);
+        const uint32_t ev = __byte_perm(e01, e23, 0x5410), od = __byte_perm(o01, o23, 0x5410);
+        *reinterpret_cast<uint32_t*>(row + cb * 4) = (ev & 0x0F0F0F0Fu) | ((od << 4) & 0xF0F0F0F0u);
     }
 };
 
@@ -451,6 +448,13 @@ struct SharedLayoutCheck {
     static constexpr bool ok = true;
 };
 
+// 1.0f where a > b, else 0.0f (also for NaN), in one comparison
+__device__ __forceinline__ float set_gt(float a, float b) {
+    float r;
+    asm("set.gt.f32.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+    return r;
+}
+
 __device__ __forceinline__ float sgnf(float x) {
     return x > 0.0f ? 1.0f : (x < 0.0f ? -1.0f : 0.0f);
 }
@@ -536,8 +540,9 @@ __device__ __forceinline__ void round_pack_fast(const float (&a)[8][8], URow uro
                 const float2 s2 = ffma2(a2, f2(inv[r], inv[r]), cn);                // u - code
                 const float2 sg = fmul2(f2(sgr, sgr), f2(sgc[c], sgc[c + 1]));      // sign(d)
                 const float2 ss = fmul2(s2, sg);
-                const float2 add = f2(ss.x > eps_b ? sg.x : 0.0f, ss.y > eps_b ? sg.y : 0.0f);
-                t2 = fadd2(t2, add);
+                // one grid step toward the update where ss > eps (exact: t is an
+                // integer-valued float far below 2^24)
+                t2 = ffma2(f2(set_gt(ss.x, eps_b), set_gt(ss.y, eps_b)), sg, t2);
             }
             t8[c] = t2.x;
             t8[c + 1] = t2.y;
