@@ -154,7 +154,8 @@ def cpu_oracle_rate(wl, seconds=10.0, threads=None, max_steps=None, tiles=None):
     import oracle
     from bit_recurrent_state_decode_b200 import synth
     threads = threads or os.cpu_count() or 1
-    tiles = tiles or max(threads * 2, 8)
+    # enough tiles per step that the worker threads, not their dispatch, set the rate
+    tiles = tiles or max(threads * 64, 8)
     tiles = min(tiles, wl.tiles_per_layer)
     hb = wl.head_bits()
     sel = np.arange(tiles)
