@@ -38,6 +38,7 @@
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
+#include <type_traits>
 
 namespace qs {
 
@@ -608,7 +609,11 @@ __device__ __forceinline__ void group_scales(int cb, int lane, int i0, const X& 
 // write of the tile, when one of them gave up) and at_barrier() runs right
 // after it.  Gated DeltaNet tiles vote at a barrier of their own at the top
 // (the caller's), before their column sums.
-template <int DK, int DV, int BITS, bool GDN, bool YOKED, bool BDR, bool BF, class AtBarrier>
+// GM: how the scale groups are known at compile time (GM_ANY: group read at
+// run time; GM_TILE: one scale per tile; GM_ROWS: groups of >= 8 columns).
+enum { GM_ANY = 0, GM_TILE = 1, GM_ROWS = 2 };
+
+template <int DK, int DV, int BITS, bool GDN, bool YOKED, bool BDR, bool BF, int GM, class AtBarrier>
 __device__ __forceinline__ bool step_tile(const StepParams& p, long long tile, const uint8_t* st,
                                           uint8_t* ct, float g0, float g1, float pts,
                                           Shared<DK, DV, GDN, YOKED>& sh,
@@ -621,7 +626,8 @@ __device__ __forceinline__ bool step_tile(const StepParams& p, long long tile, c
     constexpr int QMAX = BITS == 32 ? 0 : (1 << (BITS - 1)) - 1;
     const bool sf32 = p.scale_f32 != 0;
     constexpr int isz = BF ? 2 : 4;
-    const int group = p.group;
+    const int group = GM == GM_TILE ? 0 : p.group;
+    if (GM == GM_ROWS) __builtin_assume(group >= 8);
 
     // step inputs (shared-memory stage); q and k are read row by row where
     // they are used, which keeps them out of the register file
@@ -1086,17 +1092,29 @@ step_kernel(const StepParams p) {
         int bits;
         uint32_t cbytes;
         tile_codes(p, tile, ct, bits, cbytes, DK, DV);
-        auto run_tile = [&](bool okv, auto& hook) -> bool {
+        auto run_tile_g = [&](auto gm, bool okv, auto& hook) -> bool {
+            constexpr int G = decltype(gm)::value;
             if constexpr (BITS == 0) {
                 switch (bits) {
-                    case 2: return step_tile<DK, DV, 2, GDN, YOKED, BDR, BF>(p, tile, st, ct, g0, g1, pts, sh, xs, bf, okv, hook);
-                    case 4: return step_tile<DK, DV, 4, GDN, YOKED, BDR, BF>(p, tile, st, ct, g0, g1, pts, sh, xs, bf, okv, hook);
-                    case 6: return step_tile<DK, DV, 6, GDN, YOKED, BDR, BF>(p, tile, st, ct, g0, g1, pts, sh, xs, bf, okv, hook);
-                    default: return step_tile<DK, DV, 8, GDN, YOKED, BDR, BF>(p, tile, st, ct, g0, g1, pts, sh, xs, bf, okv, hook);
+                    case 2: return step_tile<DK, DV, 2, GDN, YOKED, BDR, BF, G>(p, tile, st, ct, g0, g1, pts, sh, xs, bf, okv, hook);
+                    case 4: return step_tile<DK, DV, 4, GDN, YOKED, BDR, BF, G>(p, tile, st, ct, g0, g1, pts, sh, xs, bf, okv, hook);
+                    case 6: return step_tile<DK, DV, 6, GDN, YOKED, BDR, BF, G>(p, tile, st, ct, g0, g1, pts, sh, xs, bf, okv, hook);
+                    default: return step_tile<DK, DV, 8, GDN, YOKED, BDR, BF, G>(p, tile, st, ct, g0, g1, pts, sh, xs, bf, okv, hook);
                 }
             } else {
                 (void)bits;
-                return step_tile<DK, DV, BITS, GDN, YOKED, BDR, BF>(p, tile, st, ct, g0, g1, pts, sh, xs, bf, okv, hook);
+                return step_tile<DK, DV, BITS, GDN, YOKED, BDR, BF, G>(p, tile, st, ct, g0, g1, pts, sh, xs, bf, okv, hook);
+            }
+        };
+        // uniform-width objects without a reference state get a tile body for
+        // each kind of scale group (one branch per tile); the others read the
+        // group at run time
+        auto run_tile = [&](bool okv, auto& hook) -> bool {
+            if constexpr (BITS == 0 || YOKED) {
+                return run_tile_g(std::integral_constant<int, GM_ANY>{}, okv, hook);
+            } else {
+                if (p.group == 0) return run_tile_g(std::integral_constant<int, GM_TILE>{}, okv, hook);
+                return run_tile_g(std::integral_constant<int, GM_ROWS>{}, okv, hook);
             }
         };
         bool done;
