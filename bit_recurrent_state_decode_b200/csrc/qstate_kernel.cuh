@@ -383,6 +383,11 @@ __device__ __forceinline__ void colsum_finish(float (&p)[8], float* red, float* 
 }
 
 // ------------------------------------------------------------------ scales
+// a flag that is either a run-time bool or a compile-time constant
+__device__ __forceinline__ bool as_bool(bool b) { return b; }
+template <bool B>
+__device__ __forceinline__ bool as_bool(std::integral_constant<bool, B>) { return B; }
+
 // m / Qmax correctly rounded, for m >= 0 finite or +inf and rq = RN(1 / Qmax):
 // a product with the rounded reciprocal, then one correction by the exact
 // remainder (Markstein's scheme for division by a constant).  For every
@@ -561,16 +566,22 @@ __device__ __forceinline__ void round_pack_fast(const float (&a)[8][8], URow uro
 // block are in shared memory; lane lp of a group derives the scales of
 // rows lp*nv .. lp*nv + nv - 1 of its row block (nv = 8 / min(L, 8)), stores
 // them, and the reciprocals go back to the group's lanes with shuffles.
-template <int DK, int DV, int L, class X, class NewScale, class PrevScale>
+// SF32: the scales are binary32 (else binary16); sprev: the staged previous
+// scales of the tile.
+template <int DK, int DV, int L, bool SF32, class X, class NewScale>
 __device__ __forceinline__ void group_scales(int cb, int lane, int i0, const X& sh,
                                              bool yoked, float (&inv)[8], unsigned& nsat,
-                                             bool& bad, NewScale new_scale, PrevScale prev_scale,
+                                             bool& bad, NewScale new_scale, const uint8_t* sprev,
                                              const StepParams& p, long long sbase, int ng, int gcol) {
     constexpr int Lp = L < 8 ? L : 8, nv = 8 / Lp;
     const int lp = cb % L;
     const int cb0 = cb - lp;                 // first column block of the group
-    const bool sf32 = p.scale_f32 != 0;
     const int rbase = (lp % Lp) * nv;
+    auto prev_scale = [&](int row) -> float {
+        const int idx = row * ng + gcol;
+        if constexpr (SF32) return reinterpret_cast<const float*>(sprev)[idx];
+        else return __half2float(reinterpret_cast<const __half*>(sprev)[idx]);
+    };
     float invm[nv];
 #pragma unroll
     for (int k = 0; k < nv; k++) {
@@ -582,11 +593,11 @@ __device__ __forceinline__ void group_scales(int cb, int lane, int i0, const X& 
             if (yoked) mr = fmaxf(mr, sh.rmaxr[cb0 + b][row]);
         }
         bool sat;
-        const float d = new_scale(mm, mr, prev_scale(row), sat);
+        const float d = new_scale(mm, mr, prev_scale(row), sat, std::integral_constant<bool, SF32>{});
         invm[k] = d == 0.0f ? 0.0f : __frcp_rn(d);
         bad |= !isfinite(mm) || !isfinite(mr);
         if (lp < 8) {
-            store_scale(p.scales, sbase + (long long)row * ng + gcol, sf32, d);
+            store_scale(p.scales, sbase + (long long)row * ng + gcol, SF32, d);
             nsat += sat ? 1u : 0u;
         }
     }
@@ -656,12 +667,23 @@ __device__ __forceinline__ bool step_tile(const StepParams& p, long long tile, c
     const int ng = group ? DV >> gsh : 1;
     const long long sbase = tile * (long long)p.n_scales;
     const int gcol = group ? j0 >> gsh : 0;
-    auto prev_scale = [&](int row) -> float {
-        if (!group) return pts;
-        const int idx = row * ng + gcol;
-        return sf32 ? reinterpret_cast<const float*>(st + p.off_scales)[idx]
-                    : __half2float(reinterpret_cast<const __half*>(st + p.off_scales)[idx]);
-    };
+    // previous scales of this thread's 8 rows (its group), one dtype branch
+    float dprev[8];
+    if constexpr (BITS == 32) {
+#pragma unroll
+        for (int r = 0; r < 8; r++) dprev[r] = 0.0f;
+    } else if (group == 0) {
+#pragma unroll
+        for (int r = 0; r < 8; r++) dprev[r] = pts;
+    } else if (sf32) {
+        const float* sp = reinterpret_cast<const float*>(st + p.off_scales) + i0 * ng + gcol;
+#pragma unroll
+        for (int r = 0; r < 8; r++) dprev[r] = sp[r * ng];
+    } else {
+        const __half* sp = reinterpret_cast<const __half*>(st + p.off_scales) + i0 * ng + gcol;
+#pragma unroll
+        for (int r = 0; r < 8; r++) dprev[r] = __half2float(sp[r * ng]);
+    }
 
     // ---- yoked reference state: stepped first; only its group maxima stay
     float mref[8];
@@ -725,7 +747,6 @@ __device__ __forceinline__ bool step_tile(const StepParams& p, long long tile, c
 
     // ---- 1. decay: a = code * (alpha * scale)   (32-bit state: S * alpha)
     float a[8][8];
-    float dprev[8];
 #pragma unroll
     for (int r = 0; r < 8; r++) {
         float c8[8];
@@ -733,9 +754,7 @@ __device__ __forceinline__ bool step_tile(const StepParams& p, long long tile, c
         if constexpr (BITS == 32) {
             ld8(st + p.off_codes + ((i0 + r) * DV + j0) * 4, false, c8);
             eta = al[r];
-            dprev[r] = 0.0f;
         } else {
-            dprev[r] = prev_scale(i0 + r);
             eta = __fmul_rn(al[r], dprev[r]);
             const uint8_t* srow = st + p.off_codes;
             if constexpr (BITS == 4) Decode<4>::run(srow + (i0 + r) * (DV / 2), cb, c8);
@@ -892,25 +911,37 @@ __device__ __forceinline__ bool step_tile(const StepParams& p, long long tile, c
                            : QMAX == 127 ? 0x1.020408p-7f : 1.0f;
         float inv[8];
         unsigned nsat = 0;
-        auto new_scale = [&](float mm, float mr, float dp, bool& sat) -> float {
+        // sfc: the scale dtype, a compile-time constant (row groups) or not
+        auto new_scale = [&](float mm, float mr, float dp, bool& sat, auto sfc) -> float {
+            const bool F = as_bool(sfc);
             sat = false;
-            if constexpr (YOKED) return to_stored(div_by_qmax(mr, fq, rq), sf32, sat);
+            if constexpr (YOKED) return to_stored(div_by_qmax(mr, fq, rq), F, sat);
             if (p.scale_mode == M_PERSISTENT)
-                return (mm > __fmul_rn(fq, dp)) ? to_stored(div_by_qmax(mm, fq, rq), sf32, sat) : dp;
-            return to_stored(div_by_qmax(mm, fq, rq), sf32, sat);
+                return (mm > __fmul_rn(fq, dp)) ? to_stored(div_by_qmax(mm, fq, rq), F, sat) : dp;
+            return to_stored(div_by_qmax(mm, fq, rq), F, sat);
         };
         bool bad = false;
         if (group) {
+            // L = group / 8 lanes per group, and the scale dtype, fixed per call
+            auto gs = [&](auto lc, auto sfc) {
+                group_scales<DK, DV, decltype(lc)::value, decltype(sfc)::value>(
+                    cb, lane, i0, xs, YOKED, inv, nsat, bad, new_scale, st + p.off_scales, p, sbase,
+                    ng, gcol);
+            };
+            auto gs_l = [&](auto lc) {
+                if (sf32) gs(lc, std::true_type{});
+                else gs(lc, std::false_type{});
+            };
             switch (group / 8) {
-                case 1: group_scales<DK, DV, 1>(cb, lane, i0, xs, YOKED, inv, nsat, bad, new_scale, prev_scale, p, sbase, ng, gcol); break;
-                case 2: group_scales<DK, DV, 2>(cb, lane, i0, xs, YOKED, inv, nsat, bad, new_scale, prev_scale, p, sbase, ng, gcol); break;
-                case 4: group_scales<DK, DV, 4>(cb, lane, i0, xs, YOKED, inv, nsat, bad, new_scale, prev_scale, p, sbase, ng, gcol); break;
-                case 8: group_scales<DK, DV, 8>(cb, lane, i0, xs, YOKED, inv, nsat, bad, new_scale, prev_scale, p, sbase, ng, gcol); break;
-                default: group_scales<DK, DV, 16>(cb, lane, i0, xs, YOKED, inv, nsat, bad, new_scale, prev_scale, p, sbase, ng, gcol); break;
+                case 1: gs_l(std::integral_constant<int, 1>{}); break;
+                case 2: gs_l(std::integral_constant<int, 2>{}); break;
+                case 4: gs_l(std::integral_constant<int, 4>{}); break;
+                case 8: gs_l(std::integral_constant<int, 8>{}); break;
+                default: gs_l(std::integral_constant<int, 16>{}); break;
             }
         } else {
             bool sat;
-            const float d = new_scale(tmax, tref, pts, sat);
+            const float d = new_scale(tmax, tref, pts, sat, sf32);
             const float iv = d == 0.0f ? 0.0f : __frcp_rn(d);
 #pragma unroll
             for (int r = 0; r < 8; r++) inv[r] = iv;
