@@ -82,6 +82,12 @@ qs::StepParams params_of(const qstate* s) {
     p.qkv_bf16 = s->L.qkv_dtype == QSTATE_BF16;
     p.gate_bf16 = s->L.gate_dtype == QSTATE_BF16;
     p.scale_f32 = s->L.scale_dtype == QSTATE_F32;
+    // per-tile scalars: alpha (Mamba2, GDN), beta (GDN), the previous scale of
+    // a per-token quantized state (mixed widths are never 32)
+    p.scalars = 0;
+    if (s->L.kind == QSTATE_MAMBA2 || s->L.kind == QSTATE_GDN) p.scalars |= qs::SC_G0;
+    if (s->L.kind == QSTATE_GDN) p.scalars |= qs::SC_G1;
+    if (s->group == 0 && (!s->head_bits.empty() || s->bits != 32)) p.scalars |= qs::SC_PTS;
     p.gamma = s->L.gamma;
     p.eps_b = s->eps_b;
     p.nstages = s->stage.nstages;

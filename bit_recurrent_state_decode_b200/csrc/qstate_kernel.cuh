@@ -75,6 +75,7 @@ struct StepParams {
     int scale_mode;
     int n_gate;
     int qkv_bf16, gate_bf16, scale_f32;
+    int scalars;                    // SC_* flags: per-tile scalars the step reads
     float gamma, eps_b;
     // pipeline stage layout (byte offsets inside one stage; -1 = not staged)
     int nstages, stage_bytes;
@@ -84,6 +85,10 @@ struct StepParams {
     unsigned wait_polls;
     long long drop_from;
 };
+
+// per-tile scalar inputs read with plain loads: alpha (Mamba2, GDN), beta
+// (GDN), and the previous scale of a per-token quantized state
+enum { SC_G0 = 1, SC_G1 = 2, SC_PTS = 4 };
 
 template <int DK, int DV>
 struct Geo {
@@ -620,9 +625,11 @@ __device__ __forceinline__ void group_scales(int cb, int lane, int i0, const X& 
 // write of the tile, when one of them gave up) and at_barrier() runs right
 // after it.  Gated DeltaNet tiles vote at a barrier of their own at the top
 // (the caller's), before their column sums.
-// GM: how the scale groups are known at compile time (GM_ANY: group read at
-// run time; GM_TILE: one scale per tile; GM_ROWS: groups of >= 8 columns).
-enum { GM_ANY = 0, GM_TILE = 1, GM_ROWS = 2 };
+// GM: what the tile body knows at compile time.  Low two bits, the scale
+// groups (GM_ANY: group read at run time; GM_TILE: one scale per tile;
+// GM_ROWS: groups of >= 8 columns); GM_ALPHA: the form of the decay is known,
+// a per-row vector (GLA) with GM_VEC, else a scalar (RetNet, Mamba2, GDN).
+enum { GM_ANY = 0, GM_TILE = 1, GM_ROWS = 2, GM_ALPHA = 4, GM_VEC = 8 };
 
 template <int DK, int DV, int BITS, bool GDN, bool YOKED, bool BDR, bool BF, int GM, class AtBarrier>
 __device__ __forceinline__ bool step_tile(const StepParams& p, long long tile, const uint8_t* st,
@@ -637,8 +644,10 @@ __device__ __forceinline__ bool step_tile(const StepParams& p, long long tile, c
     constexpr int QMAX = BITS == 32 ? 0 : (1 << (BITS - 1)) - 1;
     const bool sf32 = p.scale_f32 != 0;
     constexpr int isz = BF ? 2 : 4;
-    const int group = GM == GM_TILE ? 0 : p.group;
-    if (GM == GM_ROWS) __builtin_assume(group >= 8);
+    constexpr int GMODE = GM & 3;
+    const int group = GMODE == GM_TILE ? 0 : p.group;
+    if (GMODE == GM_ROWS) __builtin_assume(group >= 8);
+    const bool vec_alpha = (GM & GM_ALPHA) ? (GM & GM_VEC) != 0 : p.kind == K_GLA;
 
     // step inputs (shared-memory stage); q and k are read row by row where
     // they are used, which keeps them out of the register file
@@ -650,7 +659,7 @@ __device__ __forceinline__ bool step_tile(const StepParams& p, long long tile, c
     };
     float vv[8], al[8];
     ld8(st + p.off_v + j0 * isz, BF, vv);
-    if (p.kind == K_GLA) {
+    if (vec_alpha) {
         ld8(st + p.off_ga + i0 * (p.gate_bf16 ? 2 : 4), p.gate_bf16 != 0, al);
     } else {
         const float s = p.kind == K_RETNET ? p.gamma : g0;
@@ -1037,10 +1046,10 @@ __device__ __forceinline__ void issue_tile(const StepParams& p, long long tile, 
         bulk_g2s(st + p.off_ref, p.ref + tile * (long long)DK * DV, DK * DV * 4, bar);
     // the tile's scalar inputs (gates, per-token scale) are read with plain
     // loads one tile ahead; warm L2 with them now
-    if (p.kind == K_MAMBA2 || p.kind == K_GDN)
+    if (p.scalars & SC_G0)
         asm volatile("prefetch.global.L2 [%0];" :: "l"(static_cast<const uint8_t*>(p.gates) +
                                                        tile * p.n_gate * gsz));
-    if (p.group == 0 && bits != 32)
+    if (p.scalars & SC_PTS)
         asm volatile("prefetch.global.L2 [%0];" :: "l"(static_cast<const uint8_t*>(p.scales) + tile * ssz));
 }
 
@@ -1050,12 +1059,10 @@ __device__ __forceinline__ void load_scalars(const StepParams& p, long long tile
     g0 = g1 = 0.0f;
     pts = 0.0f;
     if (tile >= p.ntiles) return;
-    if (p.kind == K_MAMBA2 || p.kind == K_GDN) g0 = ldg1(p.gates, tile * p.n_gate, p.gate_bf16 != 0);
-    if (p.kind == K_GDN) g1 = ldg1(p.gates, tile * p.n_gate + 1, p.gate_bf16 != 0);
-    if (p.group == 0) {
-        int bits = p.head_bits ? p.head_bits[uint32_t(tile) % uint32_t(p.heads)] : p.bits;
-        if (bits != 32) pts = scale_at(p.scales, tile, p.scale_f32 != 0);
-    }
+    const int f = p.scalars;
+    if (f & SC_G0) g0 = ldg1(p.gates, tile * p.n_gate, p.gate_bf16 != 0);
+    if (f & SC_G1) g1 = ldg1(p.gates, tile * p.n_gate + 1, p.gate_bf16 != 0);
+    if (f & SC_PTS) pts = scale_at(p.scales, tile, p.scale_f32 != 0);
 }
 
 // ------------------------------------------------------------------ kernel
@@ -1143,9 +1150,17 @@ step_kernel(const StepParams p) {
         auto run_tile = [&](bool okv, auto& hook) -> bool {
             if constexpr (BITS == 0 || YOKED) {
                 return run_tile_g(std::integral_constant<int, GM_ANY>{}, okv, hook);
-            } else {
+            } else if constexpr (GDN) {
                 if (p.group == 0) return run_tile_g(std::integral_constant<int, GM_TILE>{}, okv, hook);
                 return run_tile_g(std::integral_constant<int, GM_ROWS>{}, okv, hook);
+            } else {
+                constexpr int S_ = GM_ALPHA, V_ = GM_ALPHA | GM_VEC;
+                if (p.kind == K_GLA) {
+                    if (p.group == 0) return run_tile_g(std::integral_constant<int, GM_TILE | V_>{}, okv, hook);
+                    return run_tile_g(std::integral_constant<int, GM_ROWS | V_>{}, okv, hook);
+                }
+                if (p.group == 0) return run_tile_g(std::integral_constant<int, GM_TILE | S_>{}, okv, hook);
+                return run_tile_g(std::integral_constant<int, GM_ROWS | S_>{}, okv, hook);
             }
         };
         bool done;
