@@ -653,9 +653,17 @@ __device__ __forceinline__ bool step_tile(const StepParams& p, long long tile, c
     // they are used, which keeps them out of the register file
     const uint8_t* sk = st + p.off_k + i0 * isz;
     const uint8_t* sq = st + p.off_q + i0 * isz;
+    // (16-byte loads of 8 bf16 or 4 fp32 rows; the unrolled uses of one
+    // vector share its load)
     auto row_in = [](const uint8_t* base, int r) -> float {
-        if constexpr (BF) return __uint_as_float(uint32_t(reinterpret_cast<const uint16_t*>(base)[r]) << 16);
-        else return reinterpret_cast<const float*>(base)[r];
+        if constexpr (BF) {
+            const uint4 u = reinterpret_cast<const uint4*>(base)[0];
+            const uint32_t w = (r >> 1) == 0 ? u.x : (r >> 1) == 1 ? u.y : (r >> 1) == 2 ? u.z : u.w;
+            return __uint_as_float((r & 1) ? (w & 0xFFFF0000u) : (w << 16));
+        } else {
+            const float4 f = reinterpret_cast<const float4*>(base)[r >> 2];
+            return (r & 3) == 0 ? f.x : (r & 3) == 1 ? f.y : (r & 3) == 2 ? f.z : f.w;
+        }
     };
     float vv[8], al[8];
     ld8(st + p.off_v + j0 * isz, BF, vv);
@@ -870,16 +878,18 @@ __device__ __forceinline__ bool step_tile(const StepParams& p, long long tile, c
             if (!__syncthreads_and(ok)) return false;
             at_barrier();
         }
-        if (threadIdx.x < DV) {
+        // the last DV threads sum the outputs (warp 0 refills the pipeline)
+        if (threadIdx.x >= G::NT - DV) {
+            const int j = threadIdx.x - (G::NT - DV);
             float t[G::NWARPS];
 #pragma unroll
-            for (int w2 = 0; w2 < G::NWARPS; w2++) t[w2] = xs.red_o[w2 * DV + threadIdx.x];
+            for (int w2 = 0; w2 < G::NWARPS; w2++) t[w2] = xs.red_o[w2 * DV + j];
 #pragma unroll
             for (int n = G::NWARPS; n > 1; n >>= 1) {
 #pragma unroll
                 for (int u = 0; u < n / 2; u++) t[u] = __fadd_rn(t[2 * u], t[2 * u + 1]);
             }
-            p.out[tile * DV + threadIdx.x] = t[0];
+            p.out[tile * DV + j] = t[0];
             if (BITS != 32 && !isfinite(t[0])) *badflag = 1;
         }
         if (group == 0 && BITS != 32) {
@@ -955,7 +965,7 @@ __device__ __forceinline__ bool step_tile(const StepParams& p, long long tile, c
 #pragma unroll
             for (int r = 0; r < 8; r++) inv[r] = iv;
             bad |= !isfinite(tmax) || !isfinite(tref);
-            if (threadIdx.x == 0) {
+            if (threadIdx.x == G::NT - 1) {
                 store_scale(p.scales, sbase, sf32, d);
                 nsat += sat ? 1u : 0u;
             }
