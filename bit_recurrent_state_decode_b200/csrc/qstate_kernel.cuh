@@ -369,16 +369,17 @@ __device__ __forceinline__ void colsum_finish(float (&p)[8], float* red, float* 
         r4[1] = make_float4(p[4], p[5], p[6], p[7]);
     }
     __syncthreads();
-    if (threadIdx.x < DV) {
+    if (threadIdx.x >= G::NT - DV) {       // the last warps (warp 0 refills)
+        const int j = threadIdx.x - (G::NT - DV);
         float t[G::NWARPS];
 #pragma unroll
-        for (int w2 = 0; w2 < G::NWARPS; w2++) t[w2] = red[w2 * DV + threadIdx.x];
+        for (int w2 = 0; w2 < G::NWARPS; w2++) t[w2] = red[w2 * DV + j];
 #pragma unroll
         for (int n = G::NWARPS; n > 1; n >>= 1) {
 #pragma unroll
             for (int u = 0; u < n / 2; u++) t[u] = __fadd_rn(t[2 * u], t[2 * u + 1]);
         }
-        tot[threadIdx.x] = t[0];
+        tot[j] = t[0];
     }
     __syncthreads();
     const float4 a = reinterpret_cast<const float4*>(tot + j0)[0];
