@@ -430,7 +430,10 @@ __device__ __forceinline__ float bdr1(float t, float s, float d, float eps) {
 template <int DK, int DV, bool YOKED>
 struct __align__(16) Xchg {
     using G = Geo<DK, DV>;
-    float red_o[G::NWARPS * DV];
+    // output partials: one per row block when a warp holds 4 or more row
+    // blocks (d_v = 64), else one per warp (row blocks joined by a shuffle)
+    static constexpr int NPART = G::RBW >= 4 ? G::NWARPS * G::RBW : G::NWARPS;
+    float red_o[NPART * DV];
     float wred[2][G::NWARPS];
     // per-row maxima of each 8-column block, column-block major; rows padded
     // by 4 so the lanes of a warp (different column blocks) hit different banks
@@ -843,15 +846,22 @@ __device__ __forceinline__ bool step_tile(const StepParams& p, long long tile, c
             }
             m[r] = mx;
         }
-#pragma unroll
-        for (int off = G::CBW; off < 32; off <<= 1) {
-#pragma unroll
-            for (int c = 0; c < 8; c++) po[c] = __fadd_rn(po[c], __shfl_xor_sync(0xFFFFFFFFu, po[c], off));
-        }
-        if (rbl == 0) {
-            float4* r4 = reinterpret_cast<float4*>(xs.red_o + warp * DV + j0);
+        if constexpr (G::RBW >= 4) {
+            // every row block's partials go to shared memory as they are
+            float4* r4 = reinterpret_cast<float4*>(xs.red_o + (warp * G::RBW + rbl) * DV + j0);
             r4[0] = make_float4(po[0], po[1], po[2], po[3]);
             r4[1] = make_float4(po[4], po[5], po[6], po[7]);
+        } else {
+#pragma unroll
+            for (int off = G::CBW; off < 32; off <<= 1) {
+#pragma unroll
+                for (int c = 0; c < 8; c++) po[c] = __fadd_rn(po[c], __shfl_xor_sync(0xFFFFFFFFu, po[c], off));
+            }
+            if (rbl == 0) {
+                float4* r4 = reinterpret_cast<float4*>(xs.red_o + warp * DV + j0);
+                r4[0] = make_float4(po[0], po[1], po[2], po[3]);
+                r4[1] = make_float4(po[4], po[5], po[6], po[7]);
+            }
         }
         if (group != 0 && BITS != 32) {
             float4* r4 = reinterpret_cast<float4*>(&xs.rmax[cb][i0]);
@@ -881,12 +891,15 @@ __device__ __forceinline__ bool step_tile(const StepParams& p, long long tile, c
         }
         // the last DV threads sum the outputs (warp 0 refills the pipeline)
         if (threadIdx.x >= G::NT - DV) {
+            // adjacent pairs, then pairs of pairs, .. over the partials in row
+            // order: the canonical block tree
+            constexpr int NP = Xchg<DK, DV, YOKED>::NPART;
             const int j = threadIdx.x - (G::NT - DV);
-            float t[G::NWARPS];
+            float t[NP];
 #pragma unroll
-            for (int w2 = 0; w2 < G::NWARPS; w2++) t[w2] = xs.red_o[w2 * DV + j];
+            for (int w2 = 0; w2 < NP; w2++) t[w2] = xs.red_o[w2 * DV + j];
 #pragma unroll
-            for (int n = G::NWARPS; n > 1; n >>= 1) {
+            for (int n = NP; n > 1; n >>= 1) {
 #pragma unroll
                 for (int u = 0; u < n / 2; u++) t[u] = __fadd_rn(t[2 * u], t[2 * u + 1]);
             }
