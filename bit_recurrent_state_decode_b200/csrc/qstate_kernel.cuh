@@ -12,21 +12,25 @@
 // stage, completing on an mbarrier; the CTA computes the tile from shared
 // memory and writes the new codes, scales and output straight to global
 // memory.  Every wait on an mbarrier is bounded: on expiry the kernel counts a
-// pipeline timeout, drains its own copies (again bounded) and returns.
+// pipeline timeout, drains its own copies (again bounded) and returns.  A tile
+// has one CTA barrier, the exchange of output partials and maxima (Gated
+// DeltaNet adds one at the top and two for its column sums); the stage of the
+// previous tile is refilled right after it.
 //
 // Each thread owns an 8 x 8 block of the tile: 8 consecutive rows (one row
 // block of the canonical reduction) and 8 consecutive columns.  A warp covers
 // all d_v columns of 32/(d_v/8) row blocks, so
 //   - the column sums r_j, o_j are an in-thread fma chain over the block (the
-//     canonical block sum), an xor butterfly across the warp's row blocks
-//     (adjacent blocks first) and a pairwise tree across warps in shared
-//     memory;
-//   - the group maxima along d_v are an in-thread max plus a reduce-scatter
-//     across the lanes sharing the group, so each lane derives the scale of
-//     one (row, group) and broadcasts its reciprocal with shuffles.
+//     canonical block sum), then a pairwise tree over the row blocks in row
+//     order: an xor butterfly across the warp's row blocks and shared memory
+//     across warps (d_v = 128), or shared memory for all of it (d_v = 64);
+//   - the group maxima along d_v are an in-thread max; the per-row maxima of
+//     every 8-column block go through shared memory with the output partials,
+//     and each lane of a group derives the scales of 8/L of its rows and
+//     broadcasts their reciprocals with shuffles.
 // Element arithmetic is branch-free and uses the packed fp32x2 instructions
 // of sm_100 (each lane of a pair rounds exactly as the scalar instruction).
-// Codes are decoded with exponent-bias tricks (a masked field ORed into the
+// Codes are decoded with exponent-bias tricks (a field placed in the
 // significand of 2^23 is an exact float, no int->float conversion) and
 // rounded with one fma against 1.5 * 2^23 (the exact product x * inv rounded
 // half to even).  No tensor cores: per tile the step is a rank-1 update and

@@ -154,6 +154,24 @@ def test_bits_and_groups(bits, group, kind):
     assert all(s["flips"] == 0 for s in stats)
 
 
+@pytest.mark.parametrize("kind", [synth.RETNET, synth.MAMBA2, synth.GLA, synth.GDN])
+@pytest.mark.parametrize("group", [0, 32])
+@pytest.mark.parametrize("sdt", [synth.F16, synth.F32])
+@pytest.mark.parametrize("rm", [synth.RTN, synth.BDR])
+def test_tile_bodies(kind, group, sdt, rm):
+    """Every compiled tile body of a uniform-width object: one scale per tile or
+    row groups, scalar or per-row decay, binary16 or binary32 scales, RTN or
+    BDR, over both warp geometries."""
+    base = {synth.RETNET: C1, synth.MAMBA2: C2, synth.GLA: C3, synth.GDN: C4}[kind]
+    dk, dv = (128, 64) if (kind + group // 32) % 2 == 0 else (64, 128)
+    wl = base.scaled(batch=2, heads=3, layers=1, d_k=dk, d_v=dv, bits=8 if group == 0 else 4,
+                     group=group, scale_dtype=sdt, round_mode=rm,
+                     scale_modes=(synth.DYNAMIC, synth.PERSISTENT), head_bits_multiset=(),
+                     q_sigma=base.q_sigma or 0.1, k_sigma=base.k_sigma or 0.1)
+    stats, status, _ = run_pair(wl, steps=8, check_every=4)
+    assert all(s["flips"] == 0 for s in stats)
+
+
 @pytest.mark.parametrize("eps", [0.0, 0.3])
 def test_bdr_eps(eps):
     wl = C4.scaled(batch=2, heads=4, layers=1, eps_b=eps)
