@@ -147,8 +147,9 @@ def default_steps(step_seconds_estimate):
     return max(50, int(3.0 / max(step_seconds_estimate, 1e-7)))
 
 
-def cpu_oracle_rate(wl, seconds=10.0, threads=None, max_steps=None, tiles=None):
-    """State-updates/s of the CPU oracle on a bounded sample of the workload."""
+def cpu_oracle_rate(wl, seconds=10.0, threads=None, max_steps=None, tiles=None, warmup=0):
+    """State-updates/s of the CPU oracle on a bounded sample of the workload;
+    the first `warmup` steps run untimed."""
     import numpy as np
 
     import oracle
@@ -168,9 +169,19 @@ def cpu_oracle_rate(wl, seconds=10.0, threads=None, max_steps=None, tiles=None):
         states.append(oracle.State(cfg, tile_bits))
     steps = 0
     busy = 0.0
+    for w in range(warmup):
+        x = synth.gen_step(wl, w, tiles=sel)
+        q, k, v, g = x.as_f32(wl)
+        alpha = beta = None
+        if wl.kind in (synth.MAMBA2, synth.GLA):
+            alpha = g
+        elif wl.kind == synth.GDN:
+            alpha, beta = g[:, :1], g[:, 1]
+        for st in states:
+            st.step(q, k, v, alpha, beta, threads=threads)
     t_end = time.perf_counter() + seconds
     while time.perf_counter() < t_end and (max_steps is None or steps < max_steps):
-        x = synth.gen_step(wl, steps, tiles=sel)
+        x = synth.gen_step(wl, warmup + steps, tiles=sel)
         q, k, v, g = x.as_f32(wl)
         alpha = beta = None
         if wl.kind in (synth.MAMBA2, synth.GLA):
@@ -419,7 +430,7 @@ def run_reference(args):
     probe = cpu_oracle_rate(wl, seconds=1.0, threads=threads, max_steps=2)
     per_tile = 1.0 / probe["value"]
     tiles = max(1, min(wl.tiles_per_layer, int(100.0 / max(K + W, 1) / per_tile)))
-    r = cpu_oracle_rate(wl, seconds=1e9, threads=threads, max_steps=K + W, tiles=tiles)
+    r = cpu_oracle_rate(wl, seconds=1e9, threads=threads, max_steps=K, tiles=tiles, warmup=W)
     return {
         "impl": "reference", "metric": "quantized state-updates/s", "value": r["value"],
         "unit": "state-updates/s", "n_gpus": 0, "steps": K, "warmup": W,
