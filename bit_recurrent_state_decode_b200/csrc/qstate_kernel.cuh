@@ -1072,16 +1072,10 @@ __device__ __forceinline__ void issue_tile(const StepParams& p, long long tile, 
         bulk_g2s(st + p.off_ga, static_cast<const uint8_t*>(p.gates) + tile * DK * gsz, DK * gsz, bar);
     if (YOKED)
         bulk_g2s(st + p.off_ref, p.ref + tile * (long long)DK * DV, DK * DV * 4, bar);
-    // the tile's scalar inputs (gates, per-token scale) are read with plain
-    // loads one tile ahead; warm L2 with them now
-    if (p.scalars & SC_G0)
-        asm volatile("prefetch.global.L2 [%0];" :: "l"(static_cast<const uint8_t*>(p.gates) +
-                                                       tile * p.n_gate * gsz));
-    if (p.scalars & SC_PTS)
-        asm volatile("prefetch.global.L2 [%0];" :: "l"(static_cast<const uint8_t*>(p.scales) + tile * ssz));
 }
 
-// Scalar per-tile inputs that are too small for a bulk copy.
+// Scalar per-tile inputs that are too small for a bulk copy, loaded one tile
+// ahead of their use.
 __device__ __forceinline__ void load_scalars(const StepParams& p, long long tile, float& g0,
                                              float& g1, float& pts) {
     g0 = g1 = 0.0f;
