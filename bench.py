@@ -274,12 +274,13 @@ def run_ours(args, rank, world, local_rank):
     e1.record(stream)
     torch.cuda.synchronize()
     est = e0.elapsed_time(e1) / 10 / 1e3
-    K = args.steps or default_steps(est)
-    W = args.warmup
-
     dist = world > 1
     if dist:
         import torch.distributed as tdist
+        # every rank sizes its loops from the same estimate (same K, same e2e steps)
+        est = max_over_ranks(est, dev)
+    K = args.steps or default_steps(est)
+    W = args.warmup
 
     for i in range(W):
         step(i)
