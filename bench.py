@@ -465,7 +465,7 @@ def main():
         tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                  device_id=torch.device("cuda", local_rank))
     res = run_ours(args, rank, world, local_rank)
-    if rank == 0 and not args.no_cpu:
+    if rank == 0 and world == 1 and not args.no_cpu:     # the CPU baseline at N = 1 only
         from bit_recurrent_state_decode_b200 import synth
         r = cpu_oracle_rate(synth.WORKLOADS[args.workload], seconds=10.0)
         res["cpu_baseline"] = {"value": r["value"], "unit": "state-updates/s",
