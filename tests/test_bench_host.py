@@ -1,0 +1,69 @@
+"""Host-side logic of bench.py (no GPU): the L2-cold replica count, the step
+count, and the lookup of the committed ncu traffic figure by source hash."""
+from __future__ import annotations
+
+import hashlib
+import os
+
+import bench
+from bit_recurrent_state_decode_b200 import synth
+
+
+def test_replicas_exceed_four_l2():
+    l2 = 126_000_000
+    for name, wl in synth.WORKLOADS.items():
+        per_layer = 20_000_000
+        r = bench.pick_replicas(wl, l2, per_layer)
+        if wl.layers > 1:
+            assert r == 1, name            # already many layers: stepped as stated
+        else:
+            assert r * per_layer >= 4 * l2 and (r - 1) * per_layer < 4 * l2, name
+
+
+def test_default_steps():
+    assert bench.default_steps(1.0) == 50          # never fewer than 50
+    assert 29_990 <= bench.default_steps(1e-4) <= 30_000   # about 3 s of timed work
+    assert bench.default_steps(0.0) > 0
+
+
+def _fake_root(tmp_path, profile_hash, value="123456"):
+    csrc = tmp_path / "bit_recurrent_state_decode_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (csrc / "a.cuh").write_bytes(b"kernel source A")
+    (csrc / "b.cu").write_bytes(b"kernel source B")
+    (csrc / "notes.txt").write_bytes(b"not hashed")
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh", ".h")):
+            h.update((csrc / f).read_bytes())
+    digest = h.hexdigest()[:16]
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    (prof / "step_kernel_w.md").write_text(
+        f"# summary\n\n- source_sha256_16: `{profile_hash or digest}`\n"
+        f"- dram_bytes_per_launch_full_size: {value}\n")
+    return digest
+
+
+def test_traffic_read_when_sources_match(tmp_path, monkeypatch):
+    _fake_root(tmp_path, None)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.read_traffic("w") == 123456.0
+    assert bench.read_traffic("missing") is None
+
+
+def test_traffic_null_once_the_kernel_changes(tmp_path, monkeypatch):
+    _fake_root(tmp_path, "0000000000000000")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.read_traffic("w") is None
+
+
+def test_committed_profiles_name_their_kernel_and_command():
+    prof = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "profiles")
+    files = [f for f in os.listdir(prof) if f.endswith(".md")]
+    assert files
+    for f in files:
+        text = open(os.path.join(prof, f)).read()
+        assert f.startswith("step_kernel_")
+        assert "source_sha256_16:" in text and "dram_bytes_per_launch_full_size:" in text
+        assert "ncu " in text and "--clock-control none" in text and "python bench.py" in text
