@@ -96,6 +96,9 @@ def lib():
         _lib.or_step.restype = ctypes.c_int
         _lib.or_step.argtypes = [ctypes.POINTER(_Cfg), ctypes.c_int64, P, P, P, P, P,
                                  P, P, P, P, P, P, ctypes.POINTER(Counts)]
+        _lib.or_step_trace.restype = ctypes.c_int
+        _lib.or_step_trace.argtypes = [ctypes.POINTER(_Cfg), ctypes.c_int64, P, P, P, P, P,
+                                       P, P, P, P, P, P, ctypes.POINTER(Counts), P, P, P]
         _lib.or_n_scales.restype = ctypes.c_int
         _lib.or_n_scales.argtypes = [ctypes.POINTER(_Cfg)]
         _lib.or_dequant.argtypes = [ctypes.POINTER(_Cfg), ctypes.c_int, P, P, P]
@@ -254,6 +257,33 @@ class State:
             for name, _ in Counts._fields_:
                 setattr(self.counts, name, getattr(self.counts, name) + getattr(c, name))
         return out
+
+    def step_trace(self, q, k, v, alpha=None, beta=None):
+        """One step of every tile (as ``step``), also returning the decayed
+        state a, the updated state before rounding x (both [T, d_k, d_v] f32)
+        and each element's rounding class ([T, d_k, d_v] int8: NONE / LOST /
+        MOVED / REVERSED)."""
+        cfg = self.cfg
+        T = self.ntiles
+        q, k, v = _f32(q).reshape(T, -1), _f32(k).reshape(T, -1), _f32(v).reshape(T, -1)
+        if alpha is not None:
+            alpha = _f32(alpha).reshape(T, -1)
+        if beta is not None:
+            beta = _f32(beta).reshape(T)
+        out = np.zeros((T, cfg.d_v), np.float32)
+        a = np.zeros((T, cfg.d_k, cfg.d_v), np.float32)
+        x = np.zeros_like(a)
+        cls = np.zeros((T, cfg.d_k, cfg.d_v), np.int8)
+        cnt = Counts()
+        rc = lib().or_step_trace(ctypes.byref(cfg.c), T, _ptr(self.tile_bits), _ptr(self.codes),
+                                 _ptr(self.S), _ptr(self.scales), _ptr(self.ref), _ptr(q),
+                                 _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(out),
+                                 ctypes.byref(cnt), _ptr(a), _ptr(x), _ptr(cls))
+        if rc != 0:
+            raise ValueError("oracle rejected the configuration")
+        for name, _ in Counts._fields_:
+            setattr(self.counts, name, getattr(self.counts, name) + getattr(cnt, name))
+        return out, a, x, cls
 
     def dequant(self) -> np.ndarray:
         T = self.ntiles

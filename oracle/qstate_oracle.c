@@ -279,7 +279,7 @@ static int finite_all(const float* p, int n)
 static void tile_step(const or_cfg* c, int bits, int8_t* codes, float* S, float* scales,
                       float* ref, const float* q, const float* k, const float* v,
                       const float* alpha, float beta, float* out, or_counts* cnt,
-                      float* a, float* x, float* aref, float* xref)
+                      float* a, float* x, float* aref, float* xref, int8_t* cls)
 {
     const int dk = c->d_k, dv = c->d_v;
     const int yoked = (c->scale_mode == OR_YOKED) && bits != 32;
@@ -378,11 +378,14 @@ static void tile_step(const or_cfg* c, int bits, int8_t* codes, float* S, float*
         for (int i = i0; i < i1; i++)
             for (int j = j0; j < j1; j++) {
                 size_t e = (size_t)i * dv + j;
-                if (cnt && c->taxonomy) {
-                    int cls = or_classify(a[e], x[e], inv, qmax);
-                    if (cls == OR_LOST) cnt->lost++;
-                    else if (cls == OR_MOVED) cnt->moved++;
-                    else if (cls == OR_REVERSED) cnt->reversed++;
+                if ((cnt && c->taxonomy) || cls) {
+                    int k3 = or_classify(a[e], x[e], inv, qmax);
+                    if (cls) cls[e] = (int8_t)k3;
+                    if (cnt && c->taxonomy) {
+                        if (k3 == OR_LOST) cnt->lost++;
+                        else if (k3 == OR_MOVED) cnt->moved++;
+                        else if (k3 == OR_REVERSED) cnt->reversed++;
+                    }
                 }
                 codes[e] = (int8_t)or_round(c, a[e], x[e], inv, qmax, cnt);
             }
@@ -395,6 +398,16 @@ int or_step(const or_cfg* c, int64_t ntiles, const int* tile_bits,
             int8_t* codes, float* S, float* scales, float* ref,
             const float* q, const float* k, const float* v,
             const float* alpha, const float* beta, float* out, or_counts* cnt)
+{
+    return or_step_trace(c, ntiles, tile_bits, codes, S, scales, ref, q, k, v, alpha, beta,
+                         out, cnt, NULL, NULL, NULL);
+}
+
+int or_step_trace(const or_cfg* c, int64_t ntiles, const int* tile_bits,
+                  int8_t* codes, float* S, float* scales, float* ref,
+                  const float* q, const float* k, const float* v,
+                  const float* alpha, const float* beta, float* out, or_counts* cnt,
+                  float* a_out, float* x_out, int8_t* cls_out)
 {
     if (!valid_cfg(c)) return -1;
     const int dk = c->d_k, dv = c->d_v;
@@ -414,7 +427,9 @@ int or_step(const or_cfg* c, int64_t ntiles, const int* tile_bits,
                   scales ? scales + t * nsc : NULL, ref ? ref + t * n : NULL,
                   q + t * dk, k + t * dk, v + t * dv,
                   alpha ? alpha + t * na : NULL, beta ? beta[t] : 0.0f,
-                  out + t * dv, cnt, buf, buf + n, buf + 2 * n, buf + 3 * n);
+                  out + t * dv, cnt,
+                  a_out ? a_out + t * n : buf, x_out ? x_out + t * n : buf + n,
+                  buf + 2 * n, buf + 3 * n, cls_out ? cls_out + t * n : NULL);
     }
     free(buf);
     return 0;

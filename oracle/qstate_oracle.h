@@ -97,6 +97,16 @@ int or_step(const or_cfg* c, int64_t ntiles, const int* tile_bits,
             const float* q, const float* k, const float* v,
             const float* alpha, const float* beta, float* out, or_counts* cnt);
 
+/* or_step, also returning per tile the decayed state a [ntiles][d_k][d_v],
+ * the updated state before rounding x (same layout) and, for quantized
+ * tiles, each element's rounding class (OR_NONE / OR_LOST / OR_MOVED /
+ * OR_REVERSED, or_classify); any of the three may be NULL. */
+int or_step_trace(const or_cfg* c, int64_t ntiles, const int* tile_bits,
+                  int8_t* codes, float* S, float* scales, float* ref,
+                  const float* q, const float* k, const float* v,
+                  const float* alpha, const float* beta, float* out, or_counts* cnt,
+                  float* a_out, float* x_out, int8_t* cls_out);
+
 int or_n_scales(const or_cfg* c);
 
 /* Dequantized state of one tile: S_hat = code * scale. */
