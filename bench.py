@@ -35,8 +35,13 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-DEFAULT_WORKLOAD = "mamba2_b64_h32_dk128_dv64_int8tok"
+DEFAULT_WORKLOAD = "gdn_l24_b256_h32_d128_int4g64_bdr"
+# workloads at batch >= 64 (the bandwidth goal applies to these) and the
+# long-horizon mixed-width one (reported only)
+ALL_WORKLOADS = ("gdn_l24_b256_h32_d128_int4g64_bdr", "mamba2_b64_h32_dk128_dv64_int8tok",
+                 "gla_b128_h16_d128_int4g32_persistent", "gdn_b32_h16_d128_mixed_3modes")
 FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0
 
 
 def parse():
@@ -44,7 +49,8 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
+                    help="a workload name, or 'all' for one line per workload in ALL_WORKLOADS")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--replicas", type=int, default=0,
                     help="independent layer replicas (0: enough to exceed 4x L2)")
@@ -234,7 +240,7 @@ def run_ours(args, rank, world, local_rank):
     bytes_per_step = sum(o.bytes_per_step() for o in objs)
 
     # ring of resident inputs (distinct layer seeds per rank)
-    ring_n = 16 if T * (wl0.d_k * 2 + wl0.d_v) * 4 * 16 < 8e9 else 4
+    ring_n = 16 if T <= 65536 else 8
     bf = wl0.qkv_dtype == synth.BF16
     gbf = wl0.gate_dtype == synth.BF16
 
@@ -354,7 +360,11 @@ def run_ours(args, rank, world, local_rank):
 
     peak, peak_kind = measured_peaks()
     achieved = dom_bytes / (launch_ms / 1e3) / 1e9
-    traffic = read_traffic(args.workload)
+    footprint = per_layer * layers            # state + step operands of one step
+    cold = footprint > 4 * props.L2_cache_size
+    # DRAM traffic per launch from the committed ncu summary, scaled to this
+    # launch by tiles (traffic grows in proportion once the launch is L2-cold)
+    traffic = read_traffic(wl0.name, T) if cold else None
     result = {
         "metric": "quantized state-updates/s",
         "value": world * T * K / (ms_total / 1e3),
@@ -373,8 +383,10 @@ def run_ours(args, rank, world, local_rank):
             "heads": wl0.heads, "d_k": wl0.d_k, "d_v": wl0.d_v, "layers": layers,
             "layer_replicas": replicas, "tiles_per_gpu": T,
             "objects": len(objs), "scale_modes": list(wl0.scale_modes),
-            "l2": f"cold: state + inputs of {layers} layers ({(per_layer * layers) / 1e6:.0f} MB) "
-                  f"> 4x L2 ({props.L2_cache_size / 1e6:.0f} MB) per step",
+            "l2": (f"cold: state + inputs of {layers} layers ({footprint / 1e6:.0f} MB) "
+                   f"> 4x L2 ({props.L2_cache_size / 1e6:.0f} MB) per step" if cold else
+                   f"warm: state + inputs of {layers} layers ({footprint / 1e6:.0f} MB) "
+                   f"<= 4x L2 ({props.L2_cache_size / 1e6:.0f} MB); L2-resident between steps"),
             "parallelism": f"dp{world} (tile shards, no collective)",
         },
         "tokens_per_s": world * wl0.batch * K / (ms_total / 1e3),
@@ -382,6 +394,7 @@ def run_ours(args, rank, world, local_rank):
         "bytes_per_step": bytes_per_step,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_source": peak_kind,
+                     "frac_of_nominal_8TBps": achieved / NOMINAL_HBM_GBS,
                      "traffic": traffic, "kernel": "qs::step_kernel",
                      "bytes_per_launch": dom_bytes, "launch_ms": launch_ms},
         "gpu_launches": K * len(objs),
@@ -392,9 +405,10 @@ def run_ours(args, rank, world, local_rank):
     return result
 
 
-def read_traffic(workload):
+def read_traffic(workload, tiles=None):
     """DRAM bytes per launch from the committed ncu summary of this workload,
-    if its recorded kernel-source hash matches the current sources."""
+    if its recorded kernel-source hash matches the current sources; scaled
+    from the summary's full-size launch to `tiles` tiles when given."""
     import hashlib
     src = os.path.join(ROOT, "bit_recurrent_state_decode_b200", "csrc")
     h = hashlib.sha256()
@@ -415,15 +429,17 @@ def read_traffic(workload):
     if vals.get("source_sha256_16") != digest:
         return None
     try:
-        return float(vals["dram_bytes_per_launch_full_size"])
+        full = float(vals["dram_bytes_per_launch_full_size"])
+        full_tiles = float(vals["tiles_per_launch_full_size"])
     except (KeyError, ValueError):
         return None
+    return full if tiles is None else full * tiles / full_tiles
 
 
 # ------------------------------------------------------------------ reference arm
 def run_reference(args):
     from bit_recurrent_state_decode_b200 import synth
-    wl = synth.WORKLOADS[args.workload]
+    wl = synth.WORKLOADS[DEFAULT_WORKLOAD if args.workload == "all" else args.workload]
     K = args.steps or 50
     W = args.warmup
     threads = os.cpu_count() or 1
@@ -464,20 +480,23 @@ def main():
         torch.cuda.set_device(local_rank)
         tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                  device_id=torch.device("cuda", local_rank))
-    res = run_ours(args, rank, world, local_rank)
-    if rank == 0 and world == 1 and not args.no_cpu:     # the CPU baseline at N = 1 only
-        from bit_recurrent_state_decode_b200 import synth
-        r = cpu_oracle_rate(synth.WORKLOADS[args.workload], seconds=10.0)
-        res["cpu_baseline"] = {"value": r["value"], "unit": "state-updates/s",
-                               "cores": r["threads"], "kind": "oracle",
-                               "sample": f"{r['tiles']} tiles x {r['steps']} steps of "
-                                         f"{args.workload} ({r['seconds']:.1f} s)"}
+    names = ALL_WORKLOADS if args.workload == "all" else (args.workload,)
+    for name in names:
+        args.workload = name
+        res = run_ours(args, rank, world, local_rank)
+        if rank == 0 and world == 1 and not args.no_cpu:     # the CPU baseline at N = 1 only
+            from bit_recurrent_state_decode_b200 import synth
+            r = cpu_oracle_rate(synth.WORKLOADS[name], seconds=10.0)
+            res["cpu_baseline"] = {"value": r["value"], "unit": "state-updates/s",
+                                   "cores": r["threads"], "kind": "oracle",
+                                   "sample": f"{r['tiles']} tiles x {r['steps']} steps of "
+                                             f"{name} ({r['seconds']:.1f} s)"}
+        if rank == 0:
+            print(json.dumps(res), flush=True)
     if world > 1:
         import torch.distributed as tdist
         tdist.barrier()
         tdist.destroy_process_group()
-    if rank == 0:
-        print(json.dumps(res), flush=True)
 
 
 if __name__ == "__main__":

@@ -6,6 +6,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 #include <new>
 #include <vector>
 
@@ -23,6 +24,16 @@ void launch_dequant(int dk, int dv, const StepParams& p, float* S, cudaStream_t 
     else if (dk == 64) launch_dequant_64_128(p, S, st);
     else if (dv == 64) launch_dequant_128_64(p, S, st);
     else launch_dequant_128_128(p, S, st);
+}
+
+bool raise_dyn_smem_limit(const void* kernel, int bytes) {
+    static std::mutex mu;
+    std::lock_guard<std::mutex> lock(mu);
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess) return false;
+    if (fa.maxDynamicSharedSizeBytes >= bytes) return true;
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) ==
+           cudaSuccess;
 }
 }  // namespace qs
 

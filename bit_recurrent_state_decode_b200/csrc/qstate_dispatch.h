@@ -41,4 +41,10 @@ inline int bits_index(int bits) {
 
 void launch_dequant(int dk, int dv, const StepParams& p, float* S, cudaStream_t st);
 
+// Raise the kernel's dynamic shared-memory limit to at least `bytes` (never
+// lower it: objects of different layouts launch the same kernel with
+// different stage sizes).  Serialised by a process-wide lock; false if a
+// CUDA call failed.
+bool raise_dyn_smem_limit(const void* kernel, int bytes);
+
 }  // namespace qs

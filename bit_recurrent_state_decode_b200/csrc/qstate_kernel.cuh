@@ -628,11 +628,12 @@ __device__ __forceinline__ void group_scales(int cb, int lane, int i0, const X& 
 // st: the tile's shared-memory stage; ct: its codes in global memory.
 // g0, g1: scalar gates (alpha, beta) and pts: per-token previous scale,
 // prefetched by the caller.  ok: this thread's stage arrived.  Without the delta
-// rule the tile has one CTA barrier, the exchange of output partials and
-// maxima; it votes on ok (false is returned by every thread, before any global
-// write of the tile, when one of them gave up) and at_barrier() runs right
-// after it.  Gated DeltaNet tiles vote at a barrier of their own at the top
-// (the caller's), before their column sums.
+// rule or a reference state the tile has one CTA barrier, the exchange of
+// output partials and maxima; it votes on ok (false is returned by every
+// thread, before any global write of the tile, when one of them gave up) and
+// at_barrier() runs right after it.  Gated DeltaNet and yoked tiles vote at a
+// barrier of their own at the top (the caller's), before their column sums or
+// their reference-state writes.
 // GM: what the tile body knows at compile time.  Low two bits, the scale
 // groups (GM_ANY: group read at run time; GM_TILE: one scale per tile;
 // GM_ROWS: groups of >= 8 columns); GM_ALPHA: the form of the decay is known,
@@ -761,7 +762,7 @@ __device__ __forceinline__ bool step_tile(const StepParams& p, long long tile, c
                 ar[r][c + 1] = v2.y;
                 mm = fmaxf(mm, fmaxf(fabsf(v2.x), fabsf(v2.y)));
             }
-            if (ok) {       // a stage that did not arrive leaves the state alone
+            {               // the stage vote was taken at the top of the tile
                 float4* dst = reinterpret_cast<float4*>(gref + (i0 + r) * DV + j0);
                 dst[0] = make_float4(ar[r][0], ar[r][1], ar[r][2], ar[r][3]);
                 dst[1] = make_float4(ar[r][4], ar[r][5], ar[r][6], ar[r][7]);
@@ -887,7 +888,7 @@ __device__ __forceinline__ bool step_tile(const StepParams& p, long long tile, c
             if (YOKED) tr = __uint_as_float(__reduce_max_sync(0xFFFFFFFFu, __float_as_uint(tr)));
             if (lane == 0) { xs.wred[0][warp] = t; xs.wred[1][warp] = tr; }
         }
-        if constexpr (GDN) {
+        if constexpr (GDN || YOKED) {
             __syncthreads();     // the vote was taken at the top of the tile
         } else {
             if (!__syncthreads_and(ok)) return false;
@@ -1131,9 +1132,10 @@ step_kernel(const StepParams p) {
         const bool ok = mbar_wait_bounded(&bars[s], parity, p.wait_polls);
         // At this tile's first barrier every thread has finished the previous
         // tile: its stage is refilled with the tile S strides ahead of it, and
-        // its non-finite flag is complete.  Without the delta rule that is the
-        // exchange barrier inside step_tile; Gated DeltaNet, whose column sums
-        // come first, takes a barrier here and refills one phase earlier.
+        // its non-finite flag is complete.  Without the delta rule or a
+        // reference state that is the exchange barrier inside step_tile; Gated
+        // DeltaNet (column sums first) and yoked tiles (reference rows written
+        // before the exchange) take a barrier here and refill one phase earlier.
         auto at_barrier = [&]() {
             if (threadIdx.x == 0 && it > 0) {
                 if (badf[(it - 1) & 1]) {
@@ -1186,7 +1188,7 @@ step_kernel(const StepParams p) {
             }
         };
         bool done;
-        if constexpr (GDN) {
+        if constexpr (GDN || YOKED) {
             done = __syncthreads_and(ok);
             if (done) {
                 at_barrier();

@@ -131,6 +131,7 @@ class QState:
             self._hb = (ctypes.c_uint8 * heads)(*[int(b) for b in head_bits])
             L.head_bits = ctypes.cast(self._hb, ctypes.POINTER(ctypes.c_uint8))
         h = ctypes.c_void_p()
+        self.device = torch.cuda.current_device() if torch.cuda.is_available() else 0
         _check("qstate_create", lib().qstate_create(ctypes.byref(L), int(bits), int(group),
                                                     int(scale_mode), int(round_mode),
                                                     float(eps_b), ctypes.byref(h)))
@@ -176,6 +177,52 @@ class QState:
     def bytes_per_step(self) -> int:
         return int(lib().qstate_bytes_per_step(self._h))
 
+    # ------------------------------------------------------------ argument checks
+    def _operand_specs(self):
+        """(name, bytes, dtype) of q, k, v, gates, out for one step."""
+        z = self.sizes
+        return (("q", z["q_bytes"], self.qkv_torch_dtype), ("k", z["q_bytes"], self.qkv_torch_dtype),
+                ("v", z["v_bytes"], self.qkv_torch_dtype),
+                ("gates", z["gate_bytes"], self.gate_torch_dtype),
+                ("out", z["out_bytes"], torch.float32))
+
+    def _check_operands(self, fn, tensors, host):
+        """Reject, before the C call, operands the kernels would read or write
+        out of bounds: wrong device, dtype, layout or size.  The C layer sees
+        only pointers and cannot tell."""
+        for (name, nbytes, dtype), t in zip(self._operand_specs(), tensors):
+            if nbytes == 0 and t is None:
+                continue
+            if t is None:
+                raise ValueError(f"{fn}: {name} is required for this layer kind")
+            if isinstance(t, torch.Tensor):
+                if host and t.is_cuda:
+                    raise ValueError(f"{fn}: {name} must be a host tensor")
+                if not host:
+                    if not t.is_cuda:
+                        raise ValueError(f"{fn}: {name} must be a CUDA tensor")
+                    if t.device.index != self.device:
+                        raise ValueError(f"{fn}: {name} is on cuda:{t.device.index}, "
+                                         f"the object on cuda:{self.device}")
+                # bf16 operands may also come as raw 16-bit patterns
+                ok_dtypes = {dtype} | ({torch.int16, torch.uint16} if dtype == torch.bfloat16
+                                       else set())
+                if t.dtype not in ok_dtypes:
+                    raise ValueError(f"{fn}: {name} has dtype {t.dtype}, expected {dtype}")
+                if not t.is_contiguous():
+                    raise ValueError(f"{fn}: {name} must be contiguous")
+                have = t.numel() * t.element_size()
+            else:
+                import numpy as np
+                a = np.asarray(t)
+                if not a.flags["C_CONTIGUOUS"]:
+                    raise ValueError(f"{fn}: {name} must be contiguous")
+                if a.dtype.itemsize != torch.tensor([], dtype=dtype).element_size():
+                    raise ValueError(f"{fn}: {name} has item size {a.dtype.itemsize}")
+                have = a.nbytes
+            if have < nbytes:
+                raise ValueError(f"{fn}: {name} holds {have} bytes, the step needs {nbytes}")
+
     # ------------------------------------------------------------ calls
     def reset(self, stream=None):
         _check("qstate_reset", lib().qstate_reset(self._h, _stream(stream)))
@@ -183,11 +230,15 @@ class QState:
     def step(self, q, k, v, gates, out, stream=None):
         """One decode step; q, k, v, gates, out are CUDA tensors in the
         layouts of include/qstate.h (gates None for RetNet)."""
+        self._check_operands("step", (q, k, v, gates, out), host=False)
         _check("qstate_step", lib().qstate_step(self._h, _ptr(q), _ptr(k), _ptr(v), _ptr(gates),
                                                 _ptr(out), _stream(stream)))
 
     def step_host(self, q, k, v, gates, out, stream=None):
-        """The same step from host buffers (pinned CPU tensors or numpy arrays)."""
+        """The same step from host buffers (pinned CPU tensors or numpy arrays).
+        Calls on one object must be issued on one stream: they share the
+        object's device staging buffers."""
+        self._check_operands("step_host", (q, k, v, gates, out), host=True)
         _check("qstate_step_host", lib().qstate_step_host(self._h, _ptr(q), _ptr(k), _ptr(v),
                                                           _ptr(gates), _ptr(out), _stream(stream)))
 

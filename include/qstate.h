@@ -139,6 +139,13 @@ typedef struct qstate_sizes {
 } qstate_sizes;
 
 /* Create a zero state (codes, scales and reference all zero).
+ * The layer kinds are the rows of Table 1 of "Preserving Updates in Low-Bit
+ * Recurrent State Quantization"; the scale modes `sm` are the three of the
+ * Abstract of "When Dynamic Scaling Fails"; group-wise INT4 at 4.50 bits
+ * (group 32, binary16 scales) is Table 2 of the first page; per-token scales
+ * (group 0) and per-head widths (L->head_bits) are the Abstract of "Low-Bit
+ * Recurrent States in Hybrid Language Models"; `rm` and `eps_b` are BDR and
+ * its threshold eps_B (Abstract, Figure 4 and Table 6 of the first page).
  * bits: 2, 4, 6, 8, or 32 (quantization disabled, fp32 state); ignored when
  *   L->head_bits is given.
  * group: columns per scale group along d_v, a multiple of 8 dividing d_v, or
@@ -153,7 +160,11 @@ int qstate_destroy(qstate* s);
 /* Zero the state again (asynchronous on stream). */
 int qstate_reset(qstate* s, qstate_stream stream);
 
-/* One decode step of every tile (one kernel launch), asynchronous on stream.
+/* One decode step of every tile (one kernel launch), asynchronous on stream:
+ * S_t = A_t S_{t-1} + B_t with the decay and update of the object's layer
+ * kind (Table 1 of "Preserving Updates in Low-Bit Recurrent State
+ * Quantization"), o_t = S_t^T q_t, then the scale, rounding and repacking of
+ * the state in the order given at the top of this file.
  * q, k, v, gates, out: caller-owned DEVICE buffers in the layouts above
  * (gates may be NULL for RetNet).  Returns after the launch. */
 int qstate_step(qstate* s, const void* q, const void* k, const void* v, const void* gates,
@@ -162,16 +173,23 @@ int qstate_step(qstate* s, const void* q, const void* k, const void* v, const vo
 /* The same step from HOST buffers: copies q, k, v, gates host->device into
  * library-owned staging buffers, launches the step and copies out
  * device->host, all asynchronous on stream (synchronise the stream before
- * reading out).  Pinned host memory makes the copies asynchronous. */
+ * reading out).  Pinned host memory makes the copies asynchronous.  The
+ * staging buffers are allocated by the first call and shared by every later
+ * call on the object: issue all qstate_step_host calls of one object on one
+ * stream (calls on different streams would overwrite each other's
+ * operands). */
 int qstate_step_host(qstate* s, const void* q, const void* k, const void* v,
                      const void* gates, float* out, qstate_stream stream);
 
-/* Dequantized state S_hat = code * scale, float32 [tiles][d_k][d_v] (device). */
+/* Dequantized state S_hat = code * scale, float32 [tiles][d_k][d_v] (device):
+ * the state a quantized recurrence carries ("Preserving Updates in Low-Bit
+ * Recurrent State Quantization", Abstract). */
 int qstate_dequant(const qstate* s, float* S_out, qstate_stream stream);
 
 /* Copy the raw state out to / in from caller device buffers of
  * qstate_sizes() bytes (codes, scales, ref; ref may be NULL if not yoked).
- * Used for checkpoints and teacher-forced parity. */
+ * Used for checkpoints and teacher-forced parity (no counterpart on the
+ * pages; the layouts are the ones above). */
 int qstate_export(const qstate* s, void* codes, void* scales, float* ref,
                   qstate_stream stream);
 int qstate_import(qstate* s, const void* codes, const void* scales, const float* ref,
@@ -181,11 +199,13 @@ int qstate_get_sizes(const qstate* s, qstate_sizes* out);
 
 /* Algorithmic bytes one step must move: packed state read + write, scales
  * read + write, q, k, v and gates read, out written, and in yoked mode the
- * float32 reference state read + write.  Returns -1 on a NULL object. */
+ * float32 reference state read + write (the memory traffic that makes FP32
+ * states costly at large batch, Abstract of "Preserving Updates in Low-Bit
+ * Recurrent State Quantization").  Returns -1 on a NULL object. */
 int64_t qstate_bytes_per_step(const qstate* s);
 
 /* Read the sticky counters: copies them device->host on stream and
- * synchronises that stream. */
+ * synchronises that stream (no counterpart on the pages). */
 int qstate_status(qstate* s, qstate_counters* out, qstate_stream stream);
 
 /* Fault injection for tests of the bounded waits (no counterpart on the

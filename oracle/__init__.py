@@ -105,6 +105,18 @@ def lib():
     return _lib
 
 
+_pools = {}
+
+
+def _pool(threads: int):
+    """A thread pool kept for the life of the process (the C step releases
+    the GIL, so the threads run the scalar code in parallel)."""
+    import concurrent.futures
+    if threads not in _pools:
+        _pools[threads] = concurrent.futures.ThreadPoolExecutor(threads)
+    return _pools[threads]
+
+
 def _ptr(a):
     return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
 
@@ -222,6 +234,11 @@ class State:
         """One step of every tile; ``threads`` > 1 splits the tiles over host
         threads (the tiles are independent; each thread runs the same scalar
         code on its own slice)."""
+        return step_many([(self, (q, k, v, alpha, beta))], threads)[0]
+
+    def _jobs(self, q, k, v, alpha, beta, pieces):
+        """The step of this state's tiles cut into `pieces` independent jobs;
+        returns (jobs, out)."""
         cfg = self.cfg
         T = self.ntiles
         q, k, v = _f32(q).reshape(T, -1), _f32(k).reshape(T, -1), _f32(v).reshape(T, -1)
@@ -245,18 +262,13 @@ class State:
                 raise ValueError("oracle rejected the configuration")
             return cnt
 
-        threads = max(1, min(int(threads), T))
-        if threads == 1:
-            parts = [run(0, T)]
-        else:
-            import concurrent.futures
-            bounds = np.linspace(0, T, threads + 1).astype(int)
-            with concurrent.futures.ThreadPoolExecutor(threads) as ex:
-                parts = list(ex.map(lambda i: run(bounds[i], bounds[i + 1]), range(threads)))
-        for c in parts:
-            for name, _ in Counts._fields_:
-                setattr(self.counts, name, getattr(self.counts, name) + getattr(c, name))
-        return out
+        pieces = max(1, min(int(pieces), T))
+        bounds = np.linspace(0, T, pieces + 1).astype(int)
+        return [(run, int(bounds[i]), int(bounds[i + 1])) for i in range(pieces)], out
+
+    def _add_counts(self, c):
+        for name, _ in Counts._fields_:
+            setattr(self.counts, name, getattr(self.counts, name) + getattr(c, name))
 
     def step_trace(self, q, k, v, alpha=None, beta=None):
         """One step of every tile (as ``step``), also returning the decayed
@@ -298,6 +310,27 @@ class State:
 
     def packed(self, t: int) -> np.ndarray:
         return pack(int(self.tile_bits[t]), self.codes[t])
+
+
+def step_many(work, threads: int = 1):
+    """One step of several independent oracle states at once: ``work`` is a
+    list of (state, (q, k, v, alpha, beta)).  The tiles of all states are
+    cut into jobs that ``threads`` host threads run together; returns the
+    outputs in order."""
+    pieces = max(1, int(threads))
+    jobs, outs = [], []
+    for st, args in work:
+        j, out = st._jobs(*args, pieces=pieces)
+        jobs.append((st, j))
+        outs.append(out)
+    flat = [(st, job) for st, js in jobs for job in js]
+    if len(flat) == 1 or threads <= 1:
+        results = [run(lo, hi) for _, (run, lo, hi) in flat]
+    else:
+        results = list(_pool(pieces).map(lambda sj: sj[1][0](sj[1][1], sj[1][2]), flat))
+    for (st, _), c in zip(flat, results):
+        st._add_counts(c)
+    return outs
 
 
 if __name__ == "__main__":  # pragma: no cover

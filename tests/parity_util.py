@@ -145,12 +145,48 @@ def compare(view: GpuView, out_gpu: np.ndarray, st: oracle.State, out_orc: np.nd
     return stats
 
 
+def _gen_chunk(wl, steps, layer_ids, orig_tiles):
+    """Inputs of several consecutive steps at once (a leading step axis), the
+    layers' tiles concatenated in object order."""
+    parts = [synth.gen_step(wl, np.asarray(steps), layer=l, tiles=orig_tiles) for l in layer_ids]
+
+    def cat(name):
+        arrs = [getattr(p, name) for p in parts]
+        return None if arrs[0] is None else np.concatenate(arrs, axis=1)
+    return synth.StepInputs(cat("q"), cat("k"), cat("v"), cat("gates"))
+
+
+def _chunk_to_device(a, bf16):
+    """[steps, T, n] host array -> list of per-step CUDA views, each starting
+    on a 16-byte boundary (the step's operand alignment)."""
+    if a is None:
+        return None
+    S, T, n = a.shape
+    esize = 2 if bf16 else 4
+    Tp = T
+    while (Tp * n * esize) % 16:
+        Tp += 1
+    dt = torch.bfloat16 if bf16 else torch.float32
+    host = np.zeros((S, Tp, n), np.uint16 if bf16 else np.float32)
+    host[:, :T] = a
+    t = torch.from_numpy(host.view(np.int16) if bf16 else host)
+    d = (t.view(torch.bfloat16) if bf16 else t).to("cuda")
+    assert d.dtype == dt
+    return [d[i, :T] for i in range(S)]
+
+
 def run_pair(wl: synth.Workload, modes=None, batch_sel=None, layers=1, steps=8, start_step=0,
-             check_every=1, teacher_forced=False):
+             check_every=1, teacher_forced=False, layer_ids=None, threads=1, chunk=64,
+             final_dequant=False):
     """Step the GPU and the oracle side by side on batch rows ``batch_sel`` of
-    ``layers`` layers; compare every ``check_every`` steps.  Returns stats."""
+    ``layers`` layers (seeded as layers ``layer_ids``, default 0 .. layers-1);
+    compare every ``check_every`` steps and after the last.  Inputs are drawn
+    ``chunk`` steps at a time; ``threads`` host threads step the oracle.
+    Returns (stats, status, oracle counters)."""
     modes = modes or wl.scale_modes
     batch_sel = np.arange(wl.batch) if batch_sel is None else np.asarray(batch_sel)
+    layer_ids = list(range(layers)) if layer_ids is None else list(layer_ids)
+    layers = len(layer_ids)
     H = wl.heads
     B = len(batch_sel)
     orig_tiles = (batch_sel[:, None] * H + np.arange(H)[None, :]).reshape(-1)
@@ -159,23 +195,37 @@ def run_pair(wl: synth.Workload, modes=None, batch_sel=None, layers=1, steps=8, 
     orc = {m: oracle_state(wl, m, tile_heads) for m in modes}
     T = B * H * layers
     all_stats = []
-    for step in range(start_step, start_step + steps):
-        x = concat_inputs([synth.gen_step(wl, step, layer=l, tiles=orig_tiles)
-                           for l in range(layers)])
-        qd, kd, vd, gd = gpu_inputs(wl, x)
-        oq, ok_, ov, oa, ob = oracle_inputs(wl, x)
-        for m in modes:
-            if teacher_forced:
-                import_oracle_state(gpu[m], orc[m])
-            out = torch.empty((T, wl.d_v), dtype=torch.float32, device="cuda")
-            gpu[m].step(qd, kd, vd, gd, out)
-            o_orc = orc[m].step(oq, ok_, ov, oa, ob)
-            if (step - start_step + 1) % check_every == 0 or step == start_step + steps - 1:
-                view = GpuView(gpu[m])
-                s = compare(view, out.cpu().numpy(), orc[m], o_orc, range(T), range(T))
-                s.update(step=step, mode=m)
-                all_stats.append(s)
+    out = {m: torch.empty((T, wl.d_v), dtype=torch.float32, device="cuda") for m in modes}
+    end = start_step + steps
+    for c0 in range(start_step, end, chunk):
+        c1 = min(end, c0 + chunk)
+        xs = _gen_chunk(wl, range(c0, c1), layer_ids, orig_tiles)
+        dq, dk, dv, dg = (_chunk_to_device(a, bf) for a, bf in
+                          zip((xs.q, xs.k, xs.v, xs.gates),
+                              (wl.qkv_dtype == synth.BF16,) * 3 + (wl.gate_dtype == synth.BF16,)))
+        for i, step in enumerate(range(c0, c1)):
+            x = synth.StepInputs(xs.q[i], xs.k[i], xs.v[i], None if xs.gates is None else xs.gates[i])
+            oq, ok_, ov, oa, ob = oracle_inputs(wl, x)
+            for m in modes:
+                if teacher_forced:
+                    import_oracle_state(gpu[m], orc[m])
+                gpu[m].step(dq[i], dk[i], dv[i], None if dg is None else dg[i], out[m])
+            o_all = oracle.step_many([(orc[m], (oq, ok_, ov, oa, ob)) for m in modes], threads)
+            for m, o_orc in zip(modes, o_all):
+                if (step - start_step + 1) % check_every == 0 or step == end - 1:
+                    view = GpuView(gpu[m])
+                    s = compare(view, out[m].cpu().numpy(), orc[m], o_orc, range(T), range(T))
+                    s.update(step=step, mode=m)
+                    all_stats.append(s)
     status = {m: gpu[m].status() for m in modes}
+    if final_dequant:
+        # the dequantized state after the last step, tile by tile (c15 metric)
+        for m in modes:
+            deq = gpu[m].dequant().cpu().numpy()
+            ref = orc[m].dequant()
+            worst = max(rel_err(deq[t], ref[t]) for t in range(T))
+            assert worst <= REL_TOL, (m, worst)
+            all_stats.append(dict(mode=m, dequant_rel=worst))
     for m in modes:
         gpu[m].close()
         assert status[m]["pipeline_timeouts"] == 0, status

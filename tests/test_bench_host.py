@@ -41,7 +41,8 @@ def _fake_root(tmp_path, profile_hash, value="123456"):
     prof.mkdir()
     (prof / "step_kernel_w.md").write_text(
         f"# summary\n\n- source_sha256_16: `{profile_hash or digest}`\n"
-        f"- dram_bytes_per_launch_full_size: {value}\n")
+        f"- dram_bytes_per_launch_full_size: {value}\n"
+        f"- tiles_per_launch_full_size: 1000\n")
     return digest
 
 
@@ -50,6 +51,16 @@ def test_traffic_read_when_sources_match(tmp_path, monkeypatch):
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     assert bench.read_traffic("w") == 123456.0
     assert bench.read_traffic("missing") is None
+
+
+def test_traffic_scaled_to_the_launch_by_tiles(tmp_path, monkeypatch):
+    """A launch of another size (other --layers / --replicas) gets the
+    committed full-size traffic scaled by its tile count, not the full-size
+    figure itself."""
+    _fake_root(tmp_path, None)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.read_traffic("w", 1000) == 123456.0
+    assert bench.read_traffic("w", 250) == 123456.0 / 4
 
 
 def test_traffic_null_once_the_kernel_changes(tmp_path, monkeypatch):
