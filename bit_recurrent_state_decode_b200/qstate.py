@@ -24,7 +24,7 @@ F32, BF16, F16 = 0, 1, 2
 
 # every symbol include/qstate.h declares
 EXPORTS = ("qstate_create", "qstate_destroy", "qstate_reset", "qstate_step", "qstate_step_host",
-           "qstate_dequant", "qstate_export", "qstate_import", "qstate_get_sizes",
+           "qstate_step_host_static", "qstate_dequant", "qstate_export", "qstate_import", "qstate_get_sizes",
            "qstate_bytes_per_step", "qstate_status", "qstate_debug_set", "qstate_error_string")
 
 
@@ -71,6 +71,7 @@ def lib():
         L.qstate_reset.argtypes = [P, S]
         L.qstate_step.argtypes = [P, P, P, P, P, P, S]
         L.qstate_step_host.argtypes = [P, P, P, P, P, P, S]
+        L.qstate_step_host_static.argtypes = [P, P, P, P, P, P, S]
         L.qstate_dequant.argtypes = [P, P, S]
         L.qstate_export.argtypes = [P, P, P, P, S]
         L.qstate_import.argtypes = [P, P, P, P, S]
@@ -241,6 +242,16 @@ class QState:
         self._check_operands("step_host", (q, k, v, gates, out), host=True)
         _check("qstate_step_host", lib().qstate_step_host(self._h, _ptr(q), _ptr(k), _ptr(v),
                                                           _ptr(gates), _ptr(out), _stream(stream)))
+
+    def step_host_static(self, q, k, v, gates, out, stream=None):
+        """The host-buffer step that allocates no device memory: the operands
+        are staged in the library's fixed device array (see
+        qstate_step_host_static in include/qstate.h for its size limit and
+        sharing rules)."""
+        self._check_operands("step_host_static", (q, k, v, gates, out), host=True)
+        _check("qstate_step_host_static",
+               lib().qstate_step_host_static(self._h, _ptr(q), _ptr(k), _ptr(v), _ptr(gates),
+                                             _ptr(out), _stream(stream)))
 
     def dequant(self, out=None, stream=None) -> torch.Tensor:
         if out is None:

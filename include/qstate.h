@@ -181,6 +181,35 @@ int qstate_step(qstate* s, const void* q, const void* k, const void* v, const vo
 int qstate_step_host(qstate* s, const void* q, const void* k, const void* v,
                      const void* gates, float* out, qstate_stream stream);
 
+/* Size of the device array that qstate_step_host_static stages operands in. */
+#define QSTATE_STATIC_STAGING_BYTES (16u << 20)
+
+/* qstate_step_host for callers that must not allocate device memory.  No
+ * counterpart on the pages: it exists for the callers of this library that
+ * cannot call cudaMalloc, such as a serving process whose device memory is
+ * all handed out by its own pool allocator, or a decode loop that must not
+ * stall (cudaMalloc may synchronise the device).  qstate_step_host allocates
+ * its staging buffers on its first call; this call allocates nothing: it
+ * copies q, k, v and gates into one fixed device array of
+ * QSTATE_STATIC_STAGING_BYTES bytes that the library image holds on every GPU
+ * that loads it until the process exits, launches the step on that copy and
+ * copies out back, all asynchronous on stream.  The object itself is still
+ * created (and its state allocated) by qstate_create.
+ *  - Size limit: q, k, v, gates and out of the object (qstate_get_sizes),
+ *    each rounded up to 256 bytes, must fit in QSTATE_STATIC_STAGING_BYTES;
+ *    larger objects get QSTATE_EINVAL and nothing is copied.
+ *  - The first call on a device looks up the array's device address (once
+ *    per device, under a lock); make that first call before capturing any
+ *    stream on that device.
+ *  - Every call on a device shares the one array and it keeps the last call's
+ *    contents; nothing in it needs clearing, since each call copies in every
+ *    operand the step reads and the step writes every element of out.  Calls
+ *    that overlap on the GPU (other streams, other objects) race on the
+ *    array: issue them on one stream, or order them with events.
+ *  - Pinned host memory makes the copies asynchronous. */
+int qstate_step_host_static(qstate* s, const void* q, const void* k, const void* v,
+                            const void* gates, float* out, qstate_stream stream);
+
 /* Dequantized state S_hat = code * scale, float32 [tiles][d_k][d_v] (device):
  * the state a quantized recurrence carries ("Preserving Updates in Low-Bit
  * Recurrent State Quantization", Abstract). */

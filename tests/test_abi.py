@@ -24,7 +24,7 @@ def _declared():
 
 def test_exports_every_declared_symbol(q):
     declared = _declared()
-    assert len(declared) == 13
+    assert len(declared) == 14
     assert sorted(q.EXPORTS) == declared
     lib = q.lib()
     for name in declared:
@@ -93,6 +93,7 @@ def test_null_object_calls(q):
     assert lib.qstate_create(None, 4, 64, 0, 0, 0.0, None) == q.EINVAL
     assert lib.qstate_step(None, None, None, None, None, None, None) == q.EINVAL
     assert lib.qstate_step_host(None, None, None, None, None, None, None) == q.EINVAL
+    assert lib.qstate_step_host_static(None, None, None, None, None, None, None) == q.EINVAL
     assert lib.qstate_dequant(None, None, None) == q.EINVAL
     assert lib.qstate_export(None, None, None, None, None) == q.EINVAL
     assert lib.qstate_import(None, None, None, None, None) == q.EINVAL
