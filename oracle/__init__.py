@@ -52,7 +52,7 @@ class _Cfg(ctypes.Structure):
                 ("group", ctypes.c_int), ("scale_mode", ctypes.c_int),
                 ("round_mode", ctypes.c_int), ("scale_f32", ctypes.c_int),
                 ("gamma", ctypes.c_float), ("eps_b", ctypes.c_float),
-                ("taxonomy", ctypes.c_int)]
+                ("taxonomy", ctypes.c_int), ("rotate", ctypes.c_int)]
 
 
 class Counts(ctypes.Structure):
@@ -102,6 +102,7 @@ def lib():
         _lib.or_n_scales.restype = ctypes.c_int
         _lib.or_n_scales.argtypes = [ctypes.POINTER(_Cfg)]
         _lib.or_dequant.argtypes = [ctypes.POINTER(_Cfg), ctypes.c_int, P, P, P]
+        _lib.or_fwht.argtypes = [ctypes.c_int, P]
     return _lib
 
 
@@ -178,6 +179,13 @@ def canon_dot(a: np.ndarray, b: np.ndarray) -> float:
     return float(lib().or_canon_dot(len(a), _ptr(a), 1, _ptr(b)))
 
 
+def fwht(x: np.ndarray) -> np.ndarray:
+    """H x for the Sylvester Hadamard matrix H (butterfly order of the C code)."""
+    y = _f32(x).copy()
+    lib().or_fwht(len(y), _ptr(y))
+    return y
+
+
 def round_rtn(x: float, inv: float, qmax: int) -> int:
     return int(lib().or_round_rtn(float(x), float(inv), int(qmax)))
 
@@ -190,9 +198,9 @@ class Config:
     """Per-tile configuration of the oracle (mirrors the step's parameters)."""
 
     def __init__(self, d_k, d_v, kind, group, scale_mode=DYNAMIC, round_mode=RTN,
-                 scale_f32=False, gamma=1.0 - 2.0 ** -5, eps_b=0.0, taxonomy=False):
+                 scale_f32=False, gamma=1.0 - 2.0 ** -5, eps_b=0.0, taxonomy=False, rotate=0):
         self.c = _Cfg(d_k, d_v, kind, group, scale_mode, round_mode, int(bool(scale_f32)),
-                      gamma, eps_b, int(bool(taxonomy)))
+                      gamma, eps_b, int(bool(taxonomy)), int(rotate))
 
     def __getattr__(self, name):
         return getattr(self.__dict__["c"], name)

@@ -174,6 +174,34 @@ float or_canon_dot(int n, const float* a, int stride, const float* b)
 }
 
 /* ------------------------------------------------------------------------
+ * Hadamard rotation ("INT4+Had applies a Hadamard rotation before INT4
+ * quantization", Table 2 of "Preserving Updates ...").
+ * Reading: the rotation acts on the value axis of the state (the axis the
+ * scale groups run along), S_rot = S H with H the Sylvester Hadamard matrix of
+ * order d_v (entries +-1, symmetric, H H = d_v I).  Every decay A_t acts on the
+ * key axis and every update is k w^T, so the rotated state follows the same
+ * recurrence with the update k (H w)^T:
+ *   rank-1:  S_rot,t = A_t S_rot,t-1 + k (H v)^T
+ *   GDN:     r_rot = (A_t S_rot,t-1)^T k = H r, e_rot = H v - r_rot = H e
+ * and the output is o = S^T q = H (S_rot^T q) / d_v.  The state is quantized
+ * in the rotated form; unrotated H (no 1/sqrt(d_v)) keeps every entry exact
+ * and the final 1/d_v is a power of two.
+ * H x is evaluated by the butterfly: for h = 1, 2, 4, ..., n/2 and every i
+ * with (i & h) == 0, (x_i, x_{i+h}) <- (x_i + x_{i+h}, x_i - x_{i+h}), one
+ * binary32 rounding per operation, in this order.
+ * ---------------------------------------------------------------------- */
+void or_fwht(int n, float* x)
+{
+    for (int h = 1; h < n; h *= 2)
+        for (int i = 0; i < n; i++)
+            if ((i & h) == 0) {
+                float a = x[i], b = x[i + h];
+                x[i] = a + b;
+                x[i + h] = a - b;
+            }
+}
+
+/* ------------------------------------------------------------------------
  * Rounding.
  * Reading: symmetric codes in [-Qmax, Qmax], Qmax = 2^(b-1) - 1; the scaled
  * value is the exact product x * inv (exact in double: two 24-bit
@@ -264,6 +292,8 @@ static int valid_cfg(const or_cfg* c)
     if (c->kind < OR_RETNET || c->kind > OR_GDN) return 0;
     if (c->scale_mode < OR_DYNAMIC || c->scale_mode > OR_YOKED) return 0;
     if (c->round_mode < OR_RTN || c->round_mode > OR_BDR) return 0;
+    if (c->rotate < 0 || c->rotate > 1) return 0;
+    if (c->rotate && (c->d_v > 512 || (c->d_v & (c->d_v - 1)))) return 0;
     return 1;
 }
 
@@ -283,6 +313,12 @@ static void tile_step(const or_cfg* c, int bits, int8_t* codes, float* S, float*
 {
     const int dk = c->d_k, dv = c->d_v;
     const int yoked = (c->scale_mode == OR_YOKED) && bits != 32;
+    float vrot[512];
+    if (c->rotate) {                    /* the update's value vector, rotated */
+        memcpy(vrot, v, sizeof(float) * (size_t)dv);
+        or_fwht(dv, vrot);
+        v = vrot;
+    }
     const int qmax = bits == 32 ? 0 : (1 << (bits - 1)) - 1;
     const int gs = c->group ? c->group : dv;             /* group width in columns */
     const int ng = dv / gs;                                /* groups per row */
@@ -333,6 +369,10 @@ static void tile_step(const or_cfg* c, int bits, int8_t* codes, float* S, float*
     /* 3. output o_t = S_t^T q_t from the updated, not yet rounded state.
      * Reading: the output is taken before the scale and rounding steps. */
     for (int j = 0; j < dv; j++) out[j] = or_canon_dot(dk, x + j, dv, q);
+    if (c->rotate) {                    /* o = H (S_rot^T q) / d_v */
+        or_fwht(dv, out);
+        for (int j = 0; j < dv; j++) out[j] = out[j] * (1.0f / (float)dv);
+    }
     int bad_out = !finite_all(out, dv);
 
     if (bits == 32) {                     /* quantization disabled */

@@ -54,6 +54,8 @@ typedef struct {
     float gamma;      /* RetNet decay */
     float eps_b;      /* BDR threshold, in grid steps of the new scale */
     int taxonomy;     /* nonzero: count lost / moved / reversed elements */
+    int rotate;       /* 1: the state is kept rotated by a Hadamard matrix along d_v
+                         (INT4+Had of Table 2 of "Preserving Updates ..."); 0: none */
 } or_cfg;
 
 typedef struct {
@@ -72,6 +74,10 @@ uint16_t or_f32_to_bf16(float x);     /* round-to-nearest-even */
 int64_t or_tile_bytes(int bits, int d_k, int d_v);
 void or_pack(int bits, int d_k, int d_v, const int8_t* codes, uint8_t* out);
 void or_unpack(int bits, int d_k, int d_v, const uint8_t* in, int8_t* codes);
+
+/* ---- Walsh-Hadamard transform, in place: x <- H x, H the n x n Sylvester
+ * Hadamard matrix (entries +-1, H H = n I), n a power of two ------------- */
+void or_fwht(int n, float* x);
 
 /* ---- canonical reduction: sum_i a[i*stride] * b[i], i < n ------------- */
 float or_canon_dot(int n, const float* a, int stride, const float* b);
