@@ -103,7 +103,18 @@ def lib():
         _lib.or_n_scales.argtypes = [ctypes.POINTER(_Cfg)]
         _lib.or_dequant.argtypes = [ctypes.POINTER(_Cfg), ctypes.c_int, P, P, P]
         _lib.or_fwht.argtypes = [ctypes.c_int, P]
+        _lib.or_lrb_step.restype = ctypes.c_int
+        _lib.or_lrb_step.argtypes = [ctypes.POINTER(_Cfg), ctypes.POINTER(LrbCfg), ctypes.c_int64,
+                                     P, P, P, P, P, P, P, P, P, P, P, P, P, P, P,
+                                     ctypes.POINTER(Counts), P]
+        _lib.or_rank_k.argtypes = [ctypes.c_int, ctypes.c_int, P, ctypes.c_int, P, P, P]
+        _lib.or_lrb_bits.restype = ctypes.c_double
+        _lib.or_lrb_bits.argtypes = [ctypes.c_int] * 5 + [ctypes.c_double]
     return _lib
+
+
+class LrbCfg(ctypes.Structure):
+    _fields_ = [("k", ctypes.c_int), ("m", ctypes.c_int), ("eps_l", ctypes.c_float)]
 
 
 _pools = {}
@@ -318,6 +329,80 @@ class State:
 
     def packed(self, t: int) -> np.ndarray:
         return pack(int(self.tile_bits[t]), self.codes[t])
+
+
+def rank_k(R: np.ndarray, k: int):
+    """Top-k singular values and vectors (s[k], U[k][rows], V[k][cols]) of R."""
+    R = np.ascontiguousarray(R, np.float64)
+    rows, cols = R.shape
+    s = np.zeros(k)
+    U = np.zeros((k, rows))
+    V = np.zeros((k, cols))
+    lib().or_rank_k(rows, cols, _ptr(R), k, _ptr(s), _ptr(U), _ptr(V))
+    return s, U, V
+
+
+def lrb_bits(bits: int, group: int, d_k: int, d_v: int, cols_used: float,
+             scale_bits: int = 16) -> float:
+    """Storage per state element with `cols_used` bypass columns."""
+    return float(lib().or_lrb_bits(bits, group, scale_bits, d_k, d_v, float(cols_used)))
+
+
+class LrbState(State):
+    """A quantized state with a Low-Rank Bypass (readings L1-L6 of the C
+    code): codes and scales as State, plus per tile u [k+m][d_k] and
+    w [k+m][d_v] (binary16 patterns), g [k+m] and the slot counts."""
+
+    def __init__(self, cfg: Config, tile_bits, k: int, m: int, eps_l: float):
+        super().__init__(cfg, tile_bits)
+        self.lcfg = LrbCfg(k, m, eps_l)
+        T = self.ntiles
+        K = k + m
+        self.u = np.zeros((T, K, cfg.d_k), np.uint16)
+        self.w = np.zeros((T, K, cfg.d_v), np.uint16)
+        self.g = np.zeros((T, K), np.float32)
+        self.nres = np.zeros(T, np.int32)
+        self.nnew = np.zeros(T, np.int32)
+        self.D = np.ones(T, np.float32)     # decay since the last merge
+        self.merged = np.zeros(T, np.int32)
+        self.peak_cols = 0                  # most columns held at once (before a merge)
+
+    def step(self, q, k, v, alpha=None, beta=None, threads: int = 1):
+        cfg = self.cfg
+        T = self.ntiles
+        q, k, v = _f32(q).reshape(T, -1), _f32(k).reshape(T, -1), _f32(v).reshape(T, -1)
+        if alpha is not None:
+            alpha = _f32(alpha).reshape(T, -1)[:, :1].copy()
+        if beta is not None:
+            beta = _f32(beta).reshape(T)
+        out = np.zeros((T, cfg.d_v), np.float32)
+        self.peak_cols = max(self.peak_cols, int(np.max(self.nres + self.nnew)) + 1)
+        cnt = Counts()
+        rc = lib().or_lrb_step(ctypes.byref(cfg.c), ctypes.byref(self.lcfg), T,
+                               _ptr(self.tile_bits), _ptr(self.codes), _ptr(self.scales),
+                               _ptr(self.u), _ptr(self.w), _ptr(self.g), _ptr(self.nres),
+                               _ptr(self.nnew), _ptr(self.D), _ptr(q), _ptr(k), _ptr(v),
+                               _ptr(alpha),
+                               _ptr(beta), _ptr(out), ctypes.byref(cnt), _ptr(self.merged))
+        if rc != 0:
+            raise ValueError("oracle rejected the LRB configuration")
+        self._add_counts(cnt)
+        return out
+
+    def cols_used(self) -> np.ndarray:
+        """Bypass columns held per tile after the last step."""
+        return self.nres + self.nnew
+
+    def state(self, t: int) -> np.ndarray:
+        """The tile's state D * S_hat + P (fp64)."""
+        return float(self.D[t]) * self.dequant()[t].astype(np.float64) + self.bypass(t)
+
+    def bypass(self, t: int) -> np.ndarray:
+        """The bypass matrix P = sum_l g_l u_l w_l^T of tile t (fp64)."""
+        n = int(self.nres[t] + self.nnew[t])
+        u = self.u[t, :n].view(np.float16).astype(np.float64)
+        w = self.w[t, :n].view(np.float16).astype(np.float64)
+        return np.einsum("l,li,lj->ij", self.g[t, :n].astype(np.float64), u, w)
 
 
 def step_many(work, threads: int = 1):

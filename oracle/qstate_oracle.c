@@ -487,3 +487,308 @@ void or_dequant(const or_cfg* c, int bits, const int8_t* codes, const float* sca
             S_out[(size_t)i * dv + j] = (float)codes[(size_t)i * dv + j] * delta;
         }
 }
+
+/* ========================================================================
+ * Low-Rank Bypass (LRB), "Preserving Updates in Low-Bit Recurrent State
+ * Quantization": the Abstract (small updates are accumulated in a compact
+ * low-rank buffer whose sufficiently large elements are periodically merged
+ * into the state), Figure 3 (updates go to the bypass and are written into
+ * the quantized state every m steps), Table 6 (k, m, eps_L per model, and
+ * the average / peak storage per state element) and Tables 8-9 (the rank k
+ * and the number k + m of bypass columns).
+ *
+ * Readings (the pages give the structure and the storage, not the rule):
+ *  L1 The bypass of a tile holds up to k + m column pairs (u_l in R^{d_k},
+ *     w_l in R^{d_v}) in binary16 with one binary32 coefficient g_l each; it
+ *     stands for P = sum_l g_l u_l w_l^T, and the tile's state is the
+ *     dequantized codes plus P.  Storage per column: (d_k + d_v) 16-bit
+ *     values plus the 32-bit coefficient (this reproduces the bits of
+ *     Tables 6, 8 and 9; see or_lrb_bits).
+ *  L2 Slots 0 .. n_res-1 hold the rank-k residual, slots n_res .. n-1 the
+ *     fresh updates in arrival order.
+ *  L3 Between merges the codes and scales are not touched: the decay since
+ *     the last merge accumulates in one binary32 factor D per tile,
+ *     D <- alpha * D (scalar decays: RetNet gamma, Mamba2 and GDN alpha_t),
+ *     so the decayed quantized part is a_ij = code_ij * (D * scale_ij), the
+ *     plain step's decay with D for alpha; rounding happens only at a merge
+ *     (a re-rounding every step would lose the decay of every code below
+ *     1 / (2 (1 - alpha)) under a persistent scale).  The per-row decay of
+ *     GLA would need a factor per row (one binary32 per row: the extra 1/16
+ *     bit of GLA in Table 6 at d_v = 512) and is not read here.  Every
+ *     column's coefficient decays with its own product since insertion,
+ *     g_l <- alpha * g_l, a new column starting at g = 1.
+ *  L4 The step's update enters the bypass as a new column: rank-1 kinds
+ *     (binary16(k), binary16(v), 1); GDN (binary16(beta k), binary16(e), 1)
+ *     with e = v - r and r = (A_t S_{t-1})^T k over the whole state:
+ *     r_j = csum_i(a_ij k_i), then for each column l in slot order
+ *     r_j <- fma(g_l * csum_i(u_li k_i), w_lj, r_j).
+ *  L5 The output is o_t = (a + P_t)^T q_t in the same form: the canonical
+ *     sum over the decayed quantized part, then the columns in slot order.
+ *  L6 When the m-th fresh column arrives the bypass is merged: the dense
+ *     P_ij = sum_l fma(g_l * u_li, w_lj, .) (slots in order, from +0) is
+ *     formed; an element is merged when |P_ij| >= eps_L * (D * scale_ij), eps_L
+ *     grid steps of the decayed grid it lives on; the state is requantized
+ *     from x = a + P on merged elements and x = a elsewhere (the scale rule
+ *     and the rounding rule of the plain step, BDR with d = x - a) and D is
+ *     reset to 1; the unmerged part R (P with the merged elements zeroed) is
+ *     replaced by its best rank-k approximation (truncated SVD, Eckart-Young)
+ *     stored as u_l = binary16(sqrt(s_l) U_l), w_l = binary16(sqrt(s_l) V_l),
+ *     g_l = 1; the fresh slots are emptied.  With k = 0, m = 1 and eps_L = 0
+ *     this is the plain quantized step (a + u w rounds once, as fma(k, v, a),
+ *     when k and v are exact in binary16).
+ * ====================================================================== */
+
+/* binary16 round trip of a binary32 value (the stored bypass precision) */
+static float f16r(float x) { return or_f16_to_f32(or_f32_to_f16(x)); }
+
+/* Top-k singular triplets of R (rows x cols, row-major, fp64) by cyclic
+ * Jacobi on the Gram matrix R^T R (cols x cols): eigenvalues s^2 and
+ * eigenvectors V; U_l = R V_l / s_l.  Writes s[k], U[k][rows], V[k][cols]
+ * (zeros past the rank). */
+void or_rank_k(int rows, int cols, const double* R, int k, double* s, double* U, double* V)
+{
+    double* A = (double*)calloc((size_t)cols * cols, sizeof(double));
+    double* E = (double*)calloc((size_t)cols * cols, sizeof(double));
+    for (int a = 0; a < cols; a++) {
+        E[(size_t)a * cols + a] = 1.0;
+        for (int b = 0; b < cols; b++) {
+            double t = 0.0;
+            for (int i = 0; i < rows; i++) t += R[(size_t)i * cols + a] * R[(size_t)i * cols + b];
+            A[(size_t)a * cols + b] = t;
+        }
+    }
+    for (int sweep = 0; sweep < 60; sweep++) {
+        double off = 0.0, diag = 0.0;
+        for (int a = 0; a < cols; a++) {
+            diag += A[(size_t)a * cols + a] * A[(size_t)a * cols + a];
+            for (int b = a + 1; b < cols; b++) off += A[(size_t)a * cols + b] * A[(size_t)a * cols + b];
+        }
+        if (off <= 1e-30 * (diag + 1e-300)) break;
+        for (int p = 0; p < cols; p++)
+            for (int q = p + 1; q < cols; q++) {
+                double apq = A[(size_t)p * cols + q];
+                if (apq == 0.0) continue;
+                double app = A[(size_t)p * cols + p], aqq = A[(size_t)q * cols + q];
+                double theta = (aqq - app) / (2.0 * apq);
+                double t = (theta >= 0 ? 1.0 : -1.0) / (fabs(theta) + sqrt(theta * theta + 1.0));
+                double cs = 1.0 / sqrt(t * t + 1.0), sn = t * cs;
+                for (int r = 0; r < cols; r++) {          /* A <- J^T A J */
+                    double arp = A[(size_t)r * cols + p], arq = A[(size_t)r * cols + q];
+                    A[(size_t)r * cols + p] = cs * arp - sn * arq;
+                    A[(size_t)r * cols + q] = sn * arp + cs * arq;
+                }
+                for (int r = 0; r < cols; r++) {
+                    double apr = A[(size_t)p * cols + r], aqr = A[(size_t)q * cols + r];
+                    A[(size_t)p * cols + r] = cs * apr - sn * aqr;
+                    A[(size_t)q * cols + r] = sn * apr + cs * aqr;
+                }
+                for (int r = 0; r < cols; r++) {          /* E <- E J */
+                    double erp = E[(size_t)r * cols + p], erq = E[(size_t)r * cols + q];
+                    E[(size_t)r * cols + p] = cs * erp - sn * erq;
+                    E[(size_t)r * cols + q] = sn * erp + cs * erq;
+                }
+            }
+    }
+    /* pick the k largest eigenvalues */
+    char* used = (char*)calloc((size_t)cols, 1);
+    for (int l = 0; l < k; l++) {
+        int best = -1;
+        for (int a = 0; a < cols; a++)
+            if (!used[a] && (best < 0 || A[(size_t)a * cols + a] > A[(size_t)best * cols + best])) best = a;
+        double lam = best >= 0 ? A[(size_t)best * cols + best] : 0.0;
+        double sig = lam > 0.0 ? sqrt(lam) : 0.0;
+        s[l] = sig;
+        for (int b = 0; b < cols; b++) V[(size_t)l * cols + b] = (best >= 0 && sig > 0.0) ? E[(size_t)b * cols + best] : 0.0;
+        for (int i = 0; i < rows; i++) {
+            double t = 0.0;
+            if (sig > 0.0)
+                for (int b = 0; b < cols; b++) t += R[(size_t)i * cols + b] * V[(size_t)l * cols + b];
+            U[(size_t)l * rows + i] = sig > 0.0 ? t / sig : 0.0;
+        }
+        if (best >= 0) used[best] = 1;
+    }
+    free(used);
+    free(A);
+    free(E);
+}
+
+/* Storage per state element of a tile with `cols_used` bypass columns. */
+double or_lrb_bits(int bits, int group, int scale_bits, int d_k, int d_v, double cols_used)
+{
+    double base = (double)bits + (group ? (double)scale_bits / group : (double)scale_bits / ((double)d_k * d_v));
+    return base + cols_used * 16.0 * (d_k + d_v + 2) / ((double)d_k * d_v);
+}
+
+static int valid_lrb(const or_cfg* c, const or_lrb_cfg* L)
+{
+    if (!valid_cfg(c) || !L) return 0;
+    if (c->kind == OR_GLA || c->scale_mode == OR_YOKED || c->rotate) return 0;
+    if (L->k < 0 || L->m < 1 || L->k + L->m > OR_LRB_MAX_COLS) return 0;
+    if (!(L->eps_l >= 0.0f)) return 0;
+    return 1;
+}
+
+/* One LRB step of one tile (bits 2..8).  u, w: [k+m][d_k], [k+m][d_v]
+ * binary16 bit patterns; g: [k+m]; nres, nnew: slot counts. */
+static void lrb_tile_step(const or_cfg* c, const or_lrb_cfg* L, int bits, int8_t* codes,
+                          float* scales, uint16_t* u, uint16_t* w, float* g, int* nres, int* nnew,
+                          float* D,
+                          const float* q, const float* k, const float* v, const float* alpha,
+                          float beta, float* out, or_counts* cnt, int* merged_out)
+{
+    const int dk = c->d_k, dv = c->d_v;
+    const int qmax = (1 << (bits - 1)) - 1;
+    const int gs = c->group ? c->group : dv, ng = dv / gs;
+    const size_t n_el = (size_t)dk * dv;
+    float* a = (float*)malloc(sizeof(float) * n_el);
+    float* x = (float*)malloc(sizeof(float) * n_el);
+    float* P = (float*)malloc(sizeof(float) * n_el);
+    float uf[OR_LRB_MAX_COLS][512], wf[OR_LRB_MAX_COLS][512];
+    const float al = c->kind == OR_RETNET ? c->gamma : alpha[0];
+
+    /* L3: the decay accumulates in D; the decayed quantized part as the plain
+     * step's decay with D for alpha; the columns' own decays */
+    *D = al * *D;
+    for (int i = 0; i < dk; i++)
+        for (int j = 0; j < dv; j++) {
+            size_t e = (size_t)i * dv + j;
+            float delta = c->group ? scales[i * ng + j / gs] : scales[0];
+            a[e] = (float)codes[e] * (*D * delta);
+        }
+    int n = *nres + *nnew;
+    for (int l = 0; l < n; l++) g[l] = al * g[l];
+
+    /* L4: the update as a new column */
+    for (int l = 0; l < n; l++) {
+        for (int i = 0; i < dk; i++) uf[l][i] = or_f16_to_f32(u[(size_t)l * dk + i]);
+        for (int j = 0; j < dv; j++) wf[l][j] = or_f16_to_f32(w[(size_t)l * dv + j]);
+    }
+    float wnew[512], unew[512];
+    if (c->kind == OR_GDN) {
+        float r[512];
+        for (int j = 0; j < dv; j++) r[j] = or_canon_dot(dk, a + j, dv, k);
+        for (int l = 0; l < n; l++) {
+            float cl = g[l] * or_canon_dot(dk, uf[l], 1, k);
+            for (int j = 0; j < dv; j++) r[j] = fmaf(cl, wf[l][j], r[j]);
+        }
+        for (int j = 0; j < dv; j++) wnew[j] = f16r(v[j] - r[j]);
+        for (int i = 0; i < dk; i++) unew[i] = f16r(beta * k[i]);
+    } else {
+        for (int j = 0; j < dv; j++) wnew[j] = f16r(v[j]);
+        for (int i = 0; i < dk; i++) unew[i] = f16r(k[i]);
+    }
+    for (int i = 0; i < dk; i++) { u[(size_t)n * dk + i] = or_f32_to_f16(unew[i]); uf[n][i] = unew[i]; }
+    for (int j = 0; j < dv; j++) { w[(size_t)n * dv + j] = or_f32_to_f16(wnew[j]); wf[n][j] = wnew[j]; }
+    g[n] = 1.0f;
+    n++;
+    (*nnew)++;
+
+    /* L5: output */
+    for (int j = 0; j < dv; j++) out[j] = or_canon_dot(dk, a + j, dv, q);
+    for (int l = 0; l < n; l++) {
+        float cl = g[l] * or_canon_dot(dk, uf[l], 1, q);
+        for (int j = 0; j < dv; j++) out[j] = fmaf(cl, wf[l][j], out[j]);
+    }
+
+    /* L6: merge every m fresh columns; otherwise requantize the decayed state */
+    const int merge = *nnew == L->m;
+    int n_merged = 0;
+    memcpy(x, a, sizeof(float) * n_el);
+    if (merge) {
+        for (size_t e = 0; e < n_el; e++) P[e] = 0.0f;
+        for (int l = 0; l < n; l++)
+            for (int i = 0; i < dk; i++) {
+                float gu = g[l] * uf[l][i];
+                for (int j = 0; j < dv; j++)
+                    P[(size_t)i * dv + j] = fmaf(gu, wf[l][j], P[(size_t)i * dv + j]);
+            }
+        for (int i = 0; i < dk; i++)
+            for (int j = 0; j < dv; j++) {
+                size_t e = (size_t)i * dv + j;
+                float dprev = c->group ? scales[i * ng + j / gs] : scales[0];
+                if (fabsf(P[e]) >= L->eps_l * (*D * dprev)) {
+                    x[e] = a[e] + P[e];
+                    P[e] = 0.0f;                     /* merged: leaves the residual */
+                    n_merged++;
+                }
+            }
+    }
+    if (!merge) {                  /* L3: nothing is rounded between merges */
+        if (merged_out) *merged_out = 0;
+        free(a);
+        free(x);
+        free(P);
+        return;
+    }
+    /* scale and rounding (the plain step's rules, on x, with a for BDR) */
+    const int ngroups = or_n_scales(c);
+    const float fq = (float)qmax;
+    for (int gi = 0; gi < ngroups; gi++) {
+        int i0 = c->group ? gi / ng : 0, i1 = c->group ? i0 + 1 : dk;
+        int j0 = c->group ? (gi % ng) * gs : 0, j1 = c->group ? j0 + gs : dv;
+        float m = 0.0f;
+        for (int i = i0; i < i1; i++)
+            for (int j = j0; j < j1; j++) m = fmaxf(m, fabsf(x[(size_t)i * dv + j]));
+        float delta;
+        if (c->scale_mode == OR_DYNAMIC) {
+            delta = to_stored_scale(c, m / fq, cnt);
+        } else {
+            float dp = scales[gi];
+            delta = (m > fq * dp) ? to_stored_scale(c, m / fq, cnt) : dp;
+        }
+        scales[gi] = delta;
+        float inv = delta == 0.0f ? 0.0f : 1.0f / delta;
+        for (int i = i0; i < i1; i++)
+            for (int j = j0; j < j1; j++) {
+                size_t e = (size_t)i * dv + j;
+                codes[e] = (int8_t)or_round(c, a[e], x[e], inv, qmax, cnt);
+            }
+    }
+    if (merge) {
+        /* the unmerged residual as its best rank-k approximation */
+        const int kk = L->k;
+        if (kk > 0) {
+            double* R = (double*)malloc(sizeof(double) * n_el);
+            double* U = (double*)malloc(sizeof(double) * (size_t)kk * dk);
+            double* V = (double*)malloc(sizeof(double) * (size_t)kk * dv);
+            double s[OR_LRB_MAX_COLS];
+            for (size_t e = 0; e < n_el; e++) R[e] = P[e];
+            or_rank_k(dk, dv, R, kk, s, U, V);
+            for (int l = 0; l < kk; l++) {
+                double rs = sqrt(s[l]);
+                for (int i = 0; i < dk; i++)
+                    u[(size_t)l * dk + i] = or_f32_to_f16((float)(rs * U[(size_t)l * dk + i]));
+                for (int j = 0; j < dv; j++)
+                    w[(size_t)l * dv + j] = or_f32_to_f16((float)(rs * V[(size_t)l * dv + j]));
+                g[l] = 1.0f;
+            }
+            free(R);
+            free(U);
+            free(V);
+        }
+        *nres = kk;
+        *nnew = 0;
+        *D = 1.0f;
+    }
+    if (merged_out) *merged_out = n_merged;
+    free(a);
+    free(x);
+    free(P);
+}
+
+int or_lrb_step(const or_cfg* c, const or_lrb_cfg* L, int64_t ntiles, const int* tile_bits,
+                int8_t* codes, float* scales, uint16_t* u, uint16_t* w, float* g, int* nres,
+                int* nnew, float* D, const float* q, const float* k, const float* v,
+                const float* alpha, const float* beta, float* out, or_counts* cnt, int* merged)
+{
+    if (!valid_lrb(c, L)) return -1;
+    const int dk = c->d_k, dv = c->d_v, K = L->k + L->m, nsc = or_n_scales(c);
+    for (int64_t t = 0; t < ntiles; t++)
+        if (tile_bits[t] < 2 || tile_bits[t] > 8 || tile_bits[t] % 2) return -1;
+    for (int64_t t = 0; t < ntiles; t++)
+        lrb_tile_step(c, L, tile_bits[t], codes + t * dk * dv, scales + t * nsc,
+                      u + t * K * dk, w + t * K * dv, g + t * K, nres + t, nnew + t, D + t,
+                      q + t * dk, k + t * dk, v + t * dv, alpha ? alpha + t : NULL,
+                      beta ? beta[t] : 0.0f, out + t * dv, cnt, merged ? merged + t : NULL);
+    return 0;
+}

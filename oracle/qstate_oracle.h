@@ -119,6 +119,33 @@ int or_n_scales(const or_cfg* c);
 void or_dequant(const or_cfg* c, int bits, const int8_t* codes, const float* scales,
                 float* S_out);
 
+/* ---- Low-Rank Bypass (LRB): readings L1-L6 in qstate_oracle.c ---------- */
+#define OR_LRB_MAX_COLS 32
+
+typedef struct {
+    int k;            /* rank of the residual kept across merges */
+    int m;            /* fresh columns (steps) between merges */
+    float eps_l;      /* merge threshold, in grid steps of the element's scale */
+} or_lrb_cfg;
+
+/* One LRB step over ntiles tiles (quantized widths 2..8 only; RetNet,
+ * Mamba2, GDN; dynamic or persistent scales).  Bypass per tile: u
+ * [k+m][d_k] and w [k+m][d_v] binary16 bit patterns, g [k+m] binary32,
+ * nres / nnew the residual and fresh slot counts, D [ntiles] the decay since
+ * the last merge (1 at the start).  merged (may be NULL):
+ * per tile, the number of elements merged by this step.  -1 if invalid. */
+int or_lrb_step(const or_cfg* c, const or_lrb_cfg* L, int64_t ntiles, const int* tile_bits,
+                int8_t* codes, float* scales, uint16_t* u, uint16_t* w, float* g, int* nres,
+                int* nnew, float* D, const float* q, const float* k, const float* v,
+                const float* alpha, const float* beta, float* out, or_counts* cnt, int* merged);
+
+/* Top-k singular triplets of a rows x cols fp64 matrix (Jacobi on R^T R). */
+void or_rank_k(int rows, int cols, const double* R, int k, double* s, double* U, double* V);
+
+/* Storage per state element: bits + scale bits per element + cols_used
+ * bypass columns of (d_k + d_v) 16-bit values and a 32-bit coefficient. */
+double or_lrb_bits(int bits, int group, int scale_bits, int d_k, int d_v, double cols_used);
+
 #ifdef __cplusplus
 }
 #endif
