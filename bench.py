@@ -216,7 +216,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     props = torch.cuda.get_device_properties(dev)
-    wl0 = synth.WORKLOADS[args.workload]
+    wl0 = synth.workload(args.workload)
     hb = wl0.head_bits()
 
     def make(mode, layers):
@@ -439,7 +439,7 @@ def read_traffic(workload, tiles=None):
 # ------------------------------------------------------------------ reference arm
 def run_reference(args):
     from bit_recurrent_state_decode_b200 import synth
-    wl = synth.WORKLOADS[DEFAULT_WORKLOAD if args.workload == "all" else args.workload]
+    wl = synth.workload(DEFAULT_WORKLOAD if args.workload == "all" else args.workload)
     K = args.steps or 50
     W = args.warmup
     threads = os.cpu_count() or 1
@@ -486,7 +486,7 @@ def main():
         res = run_ours(args, rank, world, local_rank)
         if rank == 0 and world == 1 and not args.no_cpu:     # the CPU baseline at N = 1 only
             from bit_recurrent_state_decode_b200 import synth
-            r = cpu_oracle_rate(synth.WORKLOADS[name], seconds=10.0)
+            r = cpu_oracle_rate(synth.workload(name), seconds=10.0)
             res["cpu_baseline"] = {"value": r["value"], "unit": "state-updates/s",
                                    "cores": r["threads"], "kind": "oracle",
                                    "sample": f"{r['tiles']} tiles x {r['steps']} steps of "

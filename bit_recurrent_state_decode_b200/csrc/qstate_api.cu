@@ -54,9 +54,17 @@ struct qstate {
     unsigned char* d_head_bits = nullptr;
     const qs::StepEntry* entry = nullptr;
     int grid = 1;
+    // the general kernel, when `entry` is a specialised one (the taxonomy
+    // counts run in the general kernel only)
+    const qs::StepEntry* entry_general = nullptr;
+    int grid_general = 1;
+    bool taxonomy = false;
     int dyn_smem = 0;                 // bytes of pipeline stages per CTA
     unsigned wait_polls = qs::kWaitPolls;
     long long drop_from = -1;
+    // set by qstate_import: the next step takes the general tile bodies (an
+    // imported state may hold the code -2^(bits-1), which no step produces)
+    bool import_pending = false;
     qs::StepParams stage{};           // stage layout fields only
     // staging buffers of qstate_step_host (allocated by its first call)
     void* st_q = nullptr;
@@ -112,6 +120,9 @@ qs::StepParams params_of(const qstate* s) {
     p.off_ref = s->stage.off_ref;
     p.wait_polls = s->wait_polls;
     p.drop_from = s->drop_from;
+    p.fast = s->import_pending ? 0 : 1;
+    p.taxonomy = s->taxonomy ? 1 : 0;
+    p.rotate = s->L.rotation;
     return p;
 }
 
@@ -139,7 +150,8 @@ int zero_state(qstate* s, cudaStream_t st) {
         return QSTATE_ECUDA;
     if (s->ref_bytes && cudaMemsetAsync(s->d_ref, 0, s->ref_bytes, st) != cudaSuccess)
         return QSTATE_ECUDA;
-    if (cudaMemsetAsync(s->d_counters, 0, 3 * sizeof(unsigned long long), st) != cudaSuccess)
+    if (cudaMemsetAsync(s->d_counters, 0, qs::kNumCounters * sizeof(unsigned long long), st) !=
+        cudaSuccess)
         return QSTATE_ECUDA;
     return QSTATE_OK;
 }
@@ -177,6 +189,7 @@ int qstate_create(const qstate_layout* L, int bits, int group, qstate_scale_mode
     if (L->gate_dtype != QSTATE_F32 && L->gate_dtype != QSTATE_BF16) return QSTATE_EINVAL;
     if (L->scale_dtype != QSTATE_F16 && L->scale_dtype != QSTATE_F32) return QSTATE_EINVAL;
     if (L->kind == QSTATE_RETNET && !std::isfinite(L->gamma)) return QSTATE_EINVAL;
+    if (L->rotation != 0 && L->rotation != 1) return QSTATE_EINVAL;
     if (sm < QSTATE_DYNAMIC || sm > QSTATE_YOKED) return QSTATE_EINVAL;
     if (rm < QSTATE_RTN || rm > QSTATE_BDR) return QSTATE_EINVAL;
     if (!(eps_b >= 0.0f) || !std::isfinite(eps_b)) return QSTATE_EINVAL;
@@ -235,7 +248,7 @@ int qstate_create(const qstate_layout* L, int bits, int group, qstate_scale_mode
     bool ok = alloc((void**)&s->d_codes, s->code_bytes) &&
               alloc(&s->d_scales, s->scale_bytes) &&
               alloc((void**)&s->d_ref, s->ref_bytes) &&
-              alloc((void**)&s->d_counters, 3 * sizeof(unsigned long long));
+              alloc((void**)&s->d_counters, qs::kNumCounters * sizeof(unsigned long long));
     if (ok && !hb.empty()) {
         ok = alloc((void**)&s->d_head_off, head_off.size() * sizeof(long long)) &&
              alloc((void**)&s->d_head_bits, hb.size()) &&
@@ -259,6 +272,20 @@ int qstate_create(const qstate_layout* L, int bits, int group, qstate_scale_mode
     const int bidx = qs::bits_index(hb.empty() ? bits : 0);
     const int yk = sm == QSTATE_YOKED, bd = rm == QSTATE_BDR, bf = L->qkv_dtype == QSTATE_BF16;
     s->entry = &tab[((yk * 2 + bd) * 2 + bf) * 6 + bidx];
+    // the kernel with the extra features: taxonomy counts (switched on later)
+    // and the rotated layout (fixed at creation)
+    s->entry_general = &tab[48 + ((yk * 2 + bd) * 2 + bf) * 6 + bidx];
+    if (L->rotation) s->entry = s->entry_general;
+    // rank-1 updates with round-to-nearest, one width of 4 or 8 bits, no
+    // reference state, scale groups of 32 or 64 columns and d_v = 128: the
+    // row-batched kernel (16 rows per thread, group maxima inside a warp)
+    if (L->kind != QSTATE_GDN && rm == QSTATE_RTN && sm != QSTATE_YOKED && hb.empty() &&
+        (bits == 4 || bits == 8) && dv == 128 && (group == 32 || group == 64) &&
+        L->rotation == 0) {
+        const int ridx = ((((dk == 128) * 2 + (bits == 8)) * 2 + (group == 64)) * 2 +
+                          (L->kind == QSTATE_GLA)) * 2 + bf;
+        s->entry = &qs::rows_table()[ridx];
+    }
     if (!s->entry->launch) {
         free_all(s);
         delete s;
@@ -294,23 +321,34 @@ int qstate_create(const qstate_layout* L, int bits, int group, qstate_scale_mode
     }
     int sms = 0;
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, s->device);
-    int per_sm = s->entry->blocks_per_sm(s->dyn_smem);
-    while (per_sm < 1 && s->stage.nstages > 2) {      // fewer stages if they do not fit
+    // resident CTAs per SM of both kernels with this stage size
+    auto occupancy = [&](int& fast_sm, int& general_sm) {
+        fast_sm = s->entry->blocks_per_sm(s->dyn_smem);
+        general_sm = s->entry_general == s->entry ? fast_sm
+                                                  : s->entry_general->blocks_per_sm(s->dyn_smem);
+    };
+    int per_sm, per_sm_general;
+    occupancy(per_sm, per_sm_general);
+    while ((per_sm < 1 || per_sm_general < 1) && s->stage.nstages > 2) {   // fewer stages
         cudaGetLastError();
         s->stage.nstages--;
         s->dyn_smem = s->stage.nstages * s->stage.stage_bytes;
-        per_sm = s->entry->blocks_per_sm(s->dyn_smem);
+        occupancy(per_sm, per_sm_general);
     }
-    if (per_sm < 1) {
+    if (per_sm < 1 || per_sm_general < 1) {
         cudaGetLastError();
         free_all(s);
         delete s;
         return QSTATE_EUNSUPPORTED;
     }
-    long long g = (long long)sms * per_sm;
-    if (g < 1) g = 1;
-    if (s->tiles < g) g = s->tiles > 0 ? s->tiles : 1;
-    s->grid = (int)g;
+    auto grid_of = [&](int resident) {
+        long long g = (long long)sms * resident;
+        if (g < 1) g = 1;
+        if (s->tiles < g) g = s->tiles > 0 ? s->tiles : 1;
+        return (int)g;
+    };
+    s->grid = grid_of(per_sm);
+    s->grid_general = grid_of(per_sm_general);
 
     int rc = zero_state(s, nullptr);
     if (rc == QSTATE_OK && cudaDeviceSynchronize() != cudaSuccess) rc = QSTATE_ECUDA;
@@ -351,8 +389,13 @@ int qstate_step(qstate* s, const void* q, const void* k, const void* v, const vo
     p.v = v;
     p.gates = gates;
     p.out = out;
-    s->entry->launch(p, s->grid, s->dyn_smem, (cudaStream_t)stream);
-    return cudaGetLastError() == cudaSuccess ? QSTATE_OK : QSTATE_ECUDA;
+    if (s->taxonomy)
+        s->entry_general->launch(p, s->grid_general, s->dyn_smem, (cudaStream_t)stream);
+    else
+        s->entry->launch(p, s->grid, s->dyn_smem, (cudaStream_t)stream);
+    if (cudaGetLastError() != cudaSuccess) return QSTATE_ECUDA;
+    s->import_pending = false;     // every code is within +-Qmax after a step
+    return QSTATE_OK;
 }
 
 int qstate_get_sizes(const qstate* s, qstate_sizes* o) {
@@ -445,6 +488,7 @@ int qstate_import(qstate* s, const void* codes, const void* scales, const float*
     if (s->ref_bytes &&
         cudaMemcpyAsync(s->d_ref, ref, s->ref_bytes, cudaMemcpyDefault, st) != cudaSuccess)
         return QSTATE_ECUDA;
+    s->import_pending = true;
     return QSTATE_OK;
 }
 
@@ -465,7 +509,7 @@ int qstate_debug_set(qstate* s, int64_t drop_from_tile, uint32_t wait_polls) {
 
 int qstate_status(qstate* s, qstate_counters* o, qstate_stream stream) {
     if (!s || !o) return QSTATE_EINVAL;
-    unsigned long long h[3] = {0, 0, 0};
+    unsigned long long h[qs::kNumCounters] = {};
     cudaStream_t st = (cudaStream_t)stream;
     if (cudaMemcpyAsync(h, s->d_counters, sizeof(h), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
         cudaStreamSynchronize(st) != cudaSuccess)
@@ -473,6 +517,17 @@ int qstate_status(qstate* s, qstate_counters* o, qstate_stream stream) {
     o->nonfinite = h[0];
     o->saturated = h[1];
     o->pipeline_timeouts = h[2];
+    o->exact_path_warps = h[3];
+    o->lost = h[4];
+    o->moved = h[5];
+    o->reversed = h[6];
+    o->bdr_applied = h[7];
+    return QSTATE_OK;
+}
+
+int qstate_set_taxonomy(qstate* s, int on) {
+    if (!s || (on != 0 && on != 1)) return QSTATE_EINVAL;
+    s->taxonomy = on != 0;
     return QSTATE_OK;
 }
 

@@ -15,8 +15,10 @@ struct StepEntry {
     int threads;
 };
 
-// One table per (d_k, d_v, GDN?) with 48 entries, indexed by
-// ((yoked * 2 + bdr) * 2 + bf16) * 6 + bits_index (see gen_instances.py).
+// One table per (d_k, d_v, GDN?) with 96 entries, indexed by
+// (((extra * 2 + yoked) * 2 + bdr) * 2 + bf16) * 6 + bits_index (see
+// gen_instances.py); extra = 1: the kernels that also hold the taxonomy
+// counts and the Hadamard-rotated layout.
 const StepEntry* step_table_64_64_0();
 const StepEntry* step_table_64_64_1();
 const StepEntry* step_table_64_128_0();
@@ -25,6 +27,12 @@ const StepEntry* step_table_128_64_0();
 const StepEntry* step_table_128_64_1();
 const StepEntry* step_table_128_128_0();
 const StepEntry* step_table_128_128_1();
+
+// The row-batched kernel for rank-1 updates with round-to-nearest, one code
+// width of 4 or 8 bits, scale groups of 32 or 64 columns and d_v = 128:
+// 32 entries indexed by
+// ((((d_k == 128) * 2 + (bits == 8)) * 2 + (group == 64)) * 2 + gla) * 2 + bf16.
+const StepEntry* rows_table();
 
 // 0 = per-head widths, then 2, 4, 6, 8, 32 bits; -1 if invalid
 inline int bits_index(int bits) {

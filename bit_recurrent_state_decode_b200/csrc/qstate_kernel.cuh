@@ -65,7 +65,9 @@ struct StepParams {
     const void* gates;
     float* out;
     unsigned long long* counters;   // [0] non-finite tile-steps, [1] saturated scales,
-                                    // [2] pipeline wait timeouts
+                                    // [2] pipeline wait timeouts, [3] warp-tiles that took
+                                    // the element-wise rounding path, [4..6] lost / moved /
+                                    // reversed elements, [7] BDR steps applied (taxonomy)
     const long long* head_off;      // per-head byte offset in a (layer, batch) row, or null
     const unsigned char* head_bits; // per-head bit width, or null (uniform)
     long long row_bytes;            // code bytes of one (layer, batch) row (mixed bits)
@@ -88,7 +90,18 @@ struct StepParams {
     // never copied (their waits run out), -1 = off
     unsigned wait_polls;
     long long drop_from;
+    // 1: the tile bodies that assume every stored code is within +-Qmax may
+    // run (0 for the first step after an import, which may hold -2^(b-1))
+    int fast;
+    // 1: classify every element of every tile-step (lost / moved / reversed)
+    // into counters[4..7]; 0: nothing is computed
+    int taxonomy;
+    // 1: the state is kept rotated by the Hadamard matrix along d_v (the step
+    // takes H v for v and emits H o_rot / d_v); 0: none
+    int rotate;
 };
+
+constexpr int kNumCounters = 8;
 
 // per-tile scalar inputs read with plain loads: alpha (Mamba2, GDN), beta
 // (GDN), and the previous scale of a per-token quantized state
@@ -445,7 +458,7 @@ struct __align__(16) Xchg {
     float rmaxr[YOKED ? DV / 8 : 1][DK + 4];   // of the yoked reference state
 };
 
-template <int DK, int DV, bool GDN, bool YOKED>
+template <int DK, int DV, bool GDN, bool YOKED, bool EXTRA = false>
 struct __align__(16) Shared {
     using G = Geo<DK, DV>;
     // Gated DeltaNet column sums r = a^T k, used before the exchange barrier
@@ -454,16 +467,21 @@ struct __align__(16) Shared {
     float red_r[GDN ? G::NWARPS * DV : 4];
     float tot_r[GDN ? DV : 4];
     Xchg<DK, DV, YOKED> x[2];
+    // Hadamard-rotated states (kernels with the extra features only): H v of
+    // the tile, and the output transform's exchange across warps (two
+    // buffers, one per stage parity)
+    float vrot[EXTRA ? DV : 4];
+    float orot[2][EXTRA ? DV : 4];
 };
 // the partials are written and read as float4: every array starts on 16 bytes
-template <int DK, int DV, bool GDN, bool YOKED>
+template <int DK, int DV, bool GDN, bool YOKED, bool EXTRA>
 struct SharedLayoutCheck {
     using X = Xchg<DK, DV, YOKED>;
-    using S = Shared<DK, DV, GDN, YOKED>;
+    using S = Shared<DK, DV, GDN, YOKED, EXTRA>;
     static_assert(offsetof(X, red_o) % 16 == 0 && offsetof(X, rmax) % 16 == 0 &&
                   offsetof(X, rmaxr) % 16 == 0 && sizeof(X) % 16 == 0, "exchange layout");
     static_assert(offsetof(S, red_r) % 16 == 0 && offsetof(S, tot_r) % 16 == 0 &&
-                  offsetof(S, x) % 16 == 0, "shared layout");
+                  offsetof(S, x) % 16 == 0 && offsetof(S, vrot) % 16 == 0, "shared layout");
     static constexpr bool ok = true;
 };
 
@@ -624,6 +642,132 @@ __device__ __forceinline__ void group_scales(int cb, int lane, int i0, const X& 
     }
 }
 
+// ------------------------------------------------------------------ Hadamard rotation
+// H x for the Sylvester Hadamard matrix of order n (entries +-1), by the
+// butterfly of the specification: for h = 1, 2, 4, .. and every i with
+// (i & h) == 0, (x_i, x_{i+h}) <- (x_i + x_{i+h}, x_i - x_{i+h}), one
+// rounding per operation.  The pairs of one stage are independent, so any
+// schedule that finishes each stage before the next gives the same bits.
+
+// H v of a staged v (d_v values, f32 or bf16) into vrot, by warp 0: lane l
+// holds elements E*l .. E*l + E - 1 (E = d_v / 32); stages below E run in the
+// lane, the others pair lane l with lane l ^ (h / E).
+template <int DV, bool BF>
+__device__ __forceinline__ void rotate_v(const uint8_t* sv, float* vrot) {
+    constexpr int E = DV / 32;
+    if (threadIdx.x >= 32) return;
+    const int lane = threadIdx.x;
+    float x[E];
+#pragma unroll
+    for (int e = 0; e < E; e++) {
+        const int i = E * lane + e;
+        x[e] = BF ? __uint_as_float(uint32_t(reinterpret_cast<const uint16_t*>(sv)[i]) << 16)
+                  : reinterpret_cast<const float*>(sv)[i];
+    }
+#pragma unroll
+    for (int h = 1; h < E; h *= 2) {
+#pragma unroll
+        for (int e = 0; e < E; e++)
+            if ((e & h) == 0) {
+                const float a = x[e], b = x[e + h];
+                x[e] = __fadd_rn(a, b);
+                x[e + h] = __fsub_rn(a, b);
+            }
+    }
+#pragma unroll
+    for (int h = E; h < DV; h *= 2) {
+        const int o = h / E;
+        const bool upper = (lane & o) != 0;
+#pragma unroll
+        for (int e = 0; e < E; e++) {
+            const float other = __shfl_xor_sync(0xFFFFFFFFu, x[e], o);
+            x[e] = upper ? __fsub_rn(other, x[e]) : __fadd_rn(x[e], other);
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < E; e++) vrot[E * lane + e] = x[e];
+}
+
+// H o / d_v across the DV threads that hold one output each (o of column j,
+// j = the thread's index among them; they are whole warps): stages below 32
+// with shuffles, the others through shared memory behind a named barrier
+// (id 1) that only these DV threads join.
+template <int DV>
+__device__ __forceinline__ float rotate_out(float o, int j, float (*orot)[DV]) {
+    const int lane = j & 31;
+#pragma unroll
+    for (int h = 1; h < 32 && h < DV; h *= 2) {
+        const float other = __shfl_xor_sync(0xFFFFFFFFu, o, h);
+        o = (lane & h) ? __fsub_rn(other, o) : __fadd_rn(o, other);
+    }
+    int buf = 0;
+#pragma unroll
+    for (int h = 32; h < DV; h *= 2) {
+        orot[buf][j] = o;
+        asm volatile("bar.sync 1, %0;" :: "r"(DV) : "memory");
+        const float other = orot[buf][j ^ h];
+        o = (j & h) ? __fsub_rn(other, o) : __fadd_rn(o, other);
+        buf ^= 1;
+    }
+    return __fmul_rn(o, 1.0f / float(DV));
+}
+
+// ------------------------------------------------------------------ taxonomy
+// The rounding taxonomy of Figure 4 of "Preserving Updates in Low-Bit
+// Recurrent State Quantization" on a thread's 8 x 8 block, counted into
+// counters[4..7] (lost, moved, reversed, BDR steps applied).  The decayed
+// value a and the updated value x are formed again from the staged codes with
+// the step's own operations and order, so the classes are those of the exact
+// values the step rounded: with u = a * inv and w = x * inv (exact products),
+// c = clamp(RTN(w)) and d = x - a != 0, the element is reversed when c lies
+// strictly beyond u on the side away from the update (the sign of the single
+// rounding of u - c is exact), else lost when c = clamp(RTN(u)), else moved.
+// A BDR step is applied when d > 0 and u - c > eps_B, or d < 0 and
+// u - c < -eps_B.  Diagnostic only: it runs when counters are asked for.
+template <int DK, int DV, int BITS, bool BDR, class URow>
+__device__ __forceinline__ void taxonomy_count(const StepParams& p, const uint8_t* st, int i0, int cb,
+                                            const float (&eta)[8], URow urow,
+                                            const float (&wc)[8], const float (&inv)[8]) {
+    constexpr float fq = float((1 << (BITS - 1)) - 1);
+    unsigned nl = 0, nm = 0, nr = 0, nb = 0;
+#pragma unroll 1
+    for (int r = 0; r < 8; r++) {
+        float c8[8];
+        const uint8_t* srow = st + p.off_codes;
+        if constexpr (BITS == 4) Decode<4>::run(srow + (i0 + r) * (DV / 2), cb, c8);
+        else if constexpr (BITS == 8) Decode<8>::run(srow + (i0 + r) * DV, cb, c8);
+        else if constexpr (BITS == 2) Decode<2>::run(srow + (i0 + r) * (DV / 4), cb, c8);
+        else Decode6<DK, DV>::run(srow, i0 + r, cb, c8);
+        const float ur = urow(r);
+#pragma unroll
+        for (int c = 0; c < 8; c++) {
+            const float a = __fmul_rn(c8[c], eta[r]);
+            const float x = __fmaf_rn(ur, wc[c], a);
+            const float d = __fsub_rn(x, a);
+            if (d != 0.0f) {
+                const float t = fminf(fmaxf(__fmaf_rn(x, inv[r], kMagic), kMagic - fq), kMagic + fq);
+                const float tu = fminf(fmaxf(__fmaf_rn(a, inv[r], kMagic), kMagic - fq), kMagic + fq);
+                const float s = __fmaf_rn(a, inv[r], -__fsub_rn(t, kMagic));    // u - c
+                const bool rev = (s > 0.0f && d > 0.0f) || (s < 0.0f && d < 0.0f);
+                nr += rev ? 1u : 0u;
+                nl += (!rev && t == tu) ? 1u : 0u;
+                nm += (!rev && t != tu) ? 1u : 0u;
+                if (BDR) nb += ((d > 0.0f && s > p.eps_b) || (d < 0.0f && s < -p.eps_b)) ? 1u : 0u;
+            }
+        }
+    }
+    nl = __reduce_add_sync(0xFFFFFFFFu, nl);
+    nm = __reduce_add_sync(0xFFFFFFFFu, nm);
+    nr = __reduce_add_sync(0xFFFFFFFFu, nr);
+    nb = __reduce_add_sync(0xFFFFFFFFu, nb);
+    if ((threadIdx.x & 31) == 0) {
+        if (nl) atomicAdd(p.counters + 4, (unsigned long long)nl);
+        if (nm) atomicAdd(p.counters + 5, (unsigned long long)nm);
+        if (nr) atomicAdd(p.counters + 6, (unsigned long long)nr);
+        if (nb) atomicAdd(p.counters + 7, (unsigned long long)nb);
+    }
+}
+
 // ------------------------------------------------------------------ one tile
 // st: the tile's shared-memory stage; ct: its codes in global memory.
 // g0, g1: scalar gates (alpha, beta) and pts: per-token previous scale,
@@ -640,10 +784,11 @@ __device__ __forceinline__ void group_scales(int cb, int lane, int i0, const X& 
 // a per-row vector (GLA) with GM_VEC, else a scalar (RetNet, Mamba2, GDN).
 enum { GM_ANY = 0, GM_TILE = 1, GM_ROWS = 2, GM_ALPHA = 4, GM_VEC = 8 };
 
-template <int DK, int DV, int BITS, bool GDN, bool YOKED, bool BDR, bool BF, int GM, class AtBarrier>
+template <int DK, int DV, int BITS, bool GDN, bool YOKED, bool BDR, bool BF, bool EXTRA, int GM,
+          class AtBarrier>
 __device__ __forceinline__ bool step_tile(const StepParams& p, long long tile, const uint8_t* st,
                                           uint8_t* ct, float g0, float g1, float pts,
-                                          Shared<DK, DV, GDN, YOKED>& sh,
+                                          Shared<DK, DV, GDN, YOKED, EXTRA>& sh,
                                           Xchg<DK, DV, YOKED>& xs, volatile int* badflag,
                                           bool ok, AtBarrier at_barrier) {
     using G = Geo<DK, DV>;
@@ -675,7 +820,17 @@ __device__ __forceinline__ bool step_tile(const StepParams& p, long long tile, c
         }
     };
     float vv[8], al[8];
-    ld8(st + p.off_v + j0 * isz, BF, vv);
+    bool rotated = false;
+    if constexpr (EXTRA) {
+        if (p.rotate) {
+            // the update's value vector of a rotated state is H v
+            rotate_v<DV, BF>(st + p.off_v, sh.vrot);
+            __syncthreads();
+            ld8(reinterpret_cast<const uint8_t*>(sh.vrot + j0), false, vv);
+            rotated = true;
+        }
+    }
+    if (!rotated) ld8(st + p.off_v + j0 * isz, BF, vv);
     if (vec_alpha) {
         ld8(st + p.off_ga + i0 * (p.gate_bf16 ? 2 : 4), p.gate_bf16 != 0, al);
     } else {
@@ -908,8 +1063,12 @@ __device__ __forceinline__ bool step_tile(const StepParams& p, long long tile, c
 #pragma unroll
                 for (int u = 0; u < n / 2; u++) t[u] = __fadd_rn(t[2 * u], t[2 * u + 1]);
             }
-            p.out[tile * DV + j] = t[0];
-            if (BITS != 32 && !isfinite(t[0])) *badflag = 1;
+            float o = t[0];
+            if constexpr (EXTRA) {
+                if (p.rotate) o = rotate_out<DV>(o, j, sh.orot);
+            }
+            p.out[tile * DV + j] = o;
+            if (BITS != 32 && !isfinite(o)) *badflag = 1;
         }
         if (group == 0 && BITS != 32) {
             tmax = xs.wred[0][0];
@@ -1015,13 +1174,29 @@ __device__ __forceinline__ bool step_tile(const StepParams& p, long long tile, c
                 const float eta = __fmul_rn(al[r], dprev[r]);
                 const float floor_ = fmaxf(__fmul_rn(eta, float(1 << (BITS - 1)) * 0x1p-21f), 0x1p-120f);
                 slow |= !(__fmaf_rn(fabsf(urow(r)), wmin, -floor_) > 0.0f);
-                if (__any_sync(0xFFFFFFFFu, __fmaf_rn(m[r], inv[r], -fq) > 0.0f)) clampmask |= 1u << r;
+                // A BDR step leaves the code range only from a code at +-Qmax
+                // toward u with |u| > Qmax, and then |w| > Qmax as well (w lies
+                // beyond u).  With every stored code within +-Qmax (not the step
+                // after an import), |u| <= Qmax |eta| inv (1 + 2^-23), so rows
+                // with |eta| inv <= 1 - 2^-22 (a persistent scale with a decay
+                // below 1) never need the clamp.
+                const bool may_leave = __fmaf_rn(m[r], inv[r], -fq) > 0.0f &&
+                    (!p.fast || !(__fmaf_rn(fabsf(eta), inv[r], -(1.0f - 0x1p-22f)) <= 0.0f));
+                if (__any_sync(0xFFFFFFFFu, may_leave)) clampmask |= 1u << r;
             }
         }
-        if (__any_sync(0xFFFFFFFFu, slow))
+        if (__any_sync(0xFFFFFFFFu, slow)) {
+            if (lane == 0) atomicAdd(p.counters + 3, 1ull);
             round_pack_exact<DK, DV, BITS, BDR>(a, urow, wc, inv, p.eps_b, ct, i0, cb);
-        else
+        } else {
             round_pack_fast<DK, DV, BITS, BDR>(a, urow, wc, inv, p.eps_b, clampmask, ct, i0, cb);
+        }
+        if (EXTRA && p.taxonomy) {
+            float eta[8];
+#pragma unroll
+            for (int r = 0; r < 8; r++) eta[r] = __fmul_rn(al[r], dprev[r]);
+            taxonomy_count<DK, DV, BITS, BDR>(p, st, i0, cb, eta, urow, wc, inv);
+        }
         // a tile-step is counted once if an output or a group maximum was not
         // finite (the flag is collected at the next tile's barrier)
         if (bad) *badflag = 1;
@@ -1098,12 +1273,15 @@ struct Occupancy {
 
 // BITS: the uniform code width of the object (2, 4, 6, 8, 32), or 0 when the
 // width varies per head (dispatched per tile).  BF: q, k, v are bf16.
-template <int DK, int DV, int BITS, bool GDN, bool YOKED, bool BDR, bool BF>
+// EXTRA: the kernel also holds the rounding-taxonomy counts and the
+// Hadamard-rotated layout (both switched per launch); the kernels without
+// them are the ones stepped in the ordinary case.
+template <int DK, int DV, int BITS, bool GDN, bool YOKED, bool BDR, bool BF, bool EXTRA>
 __global__ void __launch_bounds__(Geo<DK, DV>::NT, (Occupancy<DK, DV, YOKED>::MIN_BLOCKS))
 step_kernel(const StepParams p) {
     extern __shared__ __align__(128) uint8_t dsmem[];
-    static_assert(SharedLayoutCheck<DK, DV, GDN, YOKED>::ok, "");
-    __shared__ Shared<DK, DV, GDN, YOKED> sh;
+    static_assert(SharedLayoutCheck<DK, DV, GDN, YOKED, EXTRA>::ok, "");
+    __shared__ Shared<DK, DV, GDN, YOKED, EXTRA> sh;
     __shared__ __align__(8) uint64_t bars[kMaxStages];
     __shared__ volatile int badf[2];
     const int S = p.nstages;
@@ -1158,21 +1336,21 @@ step_kernel(const StepParams p) {
             constexpr int G = decltype(gm)::value;
             if constexpr (BITS == 0) {
                 switch (bits) {
-                    case 2: return step_tile<DK, DV, 2, GDN, YOKED, BDR, BF, G>(p, tile, st, ct, g0, g1, pts, sh, xs, bf, okv, hook);
-                    case 4: return step_tile<DK, DV, 4, GDN, YOKED, BDR, BF, G>(p, tile, st, ct, g0, g1, pts, sh, xs, bf, okv, hook);
-                    case 6: return step_tile<DK, DV, 6, GDN, YOKED, BDR, BF, G>(p, tile, st, ct, g0, g1, pts, sh, xs, bf, okv, hook);
-                    default: return step_tile<DK, DV, 8, GDN, YOKED, BDR, BF, G>(p, tile, st, ct, g0, g1, pts, sh, xs, bf, okv, hook);
+                    case 2: return step_tile<DK, DV, 2, GDN, YOKED, BDR, BF, EXTRA, G>(p, tile, st, ct, g0, g1, pts, sh, xs, bf, okv, hook);
+                    case 4: return step_tile<DK, DV, 4, GDN, YOKED, BDR, BF, EXTRA, G>(p, tile, st, ct, g0, g1, pts, sh, xs, bf, okv, hook);
+                    case 6: return step_tile<DK, DV, 6, GDN, YOKED, BDR, BF, EXTRA, G>(p, tile, st, ct, g0, g1, pts, sh, xs, bf, okv, hook);
+                    default: return step_tile<DK, DV, 8, GDN, YOKED, BDR, BF, EXTRA, G>(p, tile, st, ct, g0, g1, pts, sh, xs, bf, okv, hook);
                 }
             } else {
                 (void)bits;
-                return step_tile<DK, DV, BITS, GDN, YOKED, BDR, BF, G>(p, tile, st, ct, g0, g1, pts, sh, xs, bf, okv, hook);
+                return step_tile<DK, DV, BITS, GDN, YOKED, BDR, BF, EXTRA, G>(p, tile, st, ct, g0, g1, pts, sh, xs, bf, okv, hook);
             }
         };
         // uniform-width objects without a reference state get a tile body for
         // each kind of scale group (one branch per tile); the others read the
         // group at run time
         auto run_tile = [&](bool okv, auto& hook) -> bool {
-            if constexpr (BITS == 0 || YOKED) {
+            if constexpr (BITS == 0 || YOKED || EXTRA) {
                 return run_tile_g(std::integral_constant<int, GM_ANY>{}, okv, hook);
             } else if constexpr (GDN) {
                 if (p.group == 0) return run_tile_g(std::integral_constant<int, GM_TILE>{}, okv, hook);

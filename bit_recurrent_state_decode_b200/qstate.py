@@ -25,7 +25,8 @@ F32, BF16, F16 = 0, 1, 2
 # every symbol include/qstate.h declares
 EXPORTS = ("qstate_create", "qstate_destroy", "qstate_reset", "qstate_step", "qstate_step_host",
            "qstate_step_host_static", "qstate_dequant", "qstate_export", "qstate_import", "qstate_get_sizes",
-           "qstate_bytes_per_step", "qstate_status", "qstate_debug_set", "qstate_error_string")
+           "qstate_bytes_per_step", "qstate_status", "qstate_set_taxonomy", "qstate_debug_set",
+           "qstate_error_string")
 
 
 class QStateError(RuntimeError):
@@ -39,12 +40,13 @@ class Layout(ctypes.Structure):
                 ("d_v", ctypes.c_int32), ("layers", ctypes.c_int32), ("kind", ctypes.c_int32),
                 ("gamma", ctypes.c_float), ("qkv_dtype", ctypes.c_int32),
                 ("gate_dtype", ctypes.c_int32), ("scale_dtype", ctypes.c_int32),
-                ("head_bits", ctypes.POINTER(ctypes.c_uint8))]
+                ("head_bits", ctypes.POINTER(ctypes.c_uint8)), ("rotation", ctypes.c_int32)]
 
 
 class Counters(ctypes.Structure):
-    _fields_ = [("nonfinite", ctypes.c_uint64), ("saturated", ctypes.c_uint64),
-                ("pipeline_timeouts", ctypes.c_uint64)]
+    _fields_ = [(n, ctypes.c_uint64) for n in ("nonfinite", "saturated", "pipeline_timeouts",
+                                               "exact_path_warps", "lost", "moved", "reversed",
+                                               "bdr_applied")]
 
 
 class Sizes(ctypes.Structure):
@@ -80,6 +82,7 @@ def lib():
         L.qstate_bytes_per_step.restype = ctypes.c_int64
         L.qstate_status.argtypes = [P, ctypes.POINTER(Counters), S]
         L.qstate_debug_set.argtypes = [P, ctypes.c_int64, ctypes.c_uint32]
+        L.qstate_set_taxonomy.argtypes = [P, I]
         L.qstate_error_string.argtypes = [I]
         L.qstate_error_string.restype = ctypes.c_char_p
         for name in EXPORTS:
@@ -123,11 +126,11 @@ class QState:
 
     def __init__(self, batch, heads, d_k, d_v, kind, bits=4, group=64, scale_mode=DYNAMIC,
                  round_mode=RTN, eps_b=0.0, layers=1, gamma=1.0 - 2.0 ** -5, qkv_dtype=F32,
-                 gate_dtype=F32, scale_dtype=F16, head_bits=None):
+                 gate_dtype=F32, scale_dtype=F16, head_bits=None, rotation=0):
         self._h = None
         self._hb = None
         L = Layout(batch, heads, d_k, d_v, layers, kind, gamma, qkv_dtype, gate_dtype,
-                   scale_dtype, None)
+                   scale_dtype, None, int(rotation))
         if head_bits is not None:
             self._hb = (ctypes.c_uint8 * heads)(*[int(b) for b in head_bits])
             L.head_bits = ctypes.cast(self._hb, ctypes.POINTER(ctypes.c_uint8))
@@ -142,6 +145,7 @@ class QState:
         self.scale_mode, self.round_mode, self.eps_b = scale_mode, round_mode, eps_b
         self.qkv_dtype, self.gate_dtype, self.scale_dtype = qkv_dtype, gate_dtype, scale_dtype
         self.head_bits = None if head_bits is None else [int(b) for b in head_bits]
+        self.rotation = int(rotation)
         z = Sizes()
         _check("qstate_get_sizes", lib().qstate_get_sizes(self._h, ctypes.byref(z)))
         self.sizes = {n: int(getattr(z, n)) for n, _ in Sizes._fields_}
@@ -279,8 +283,12 @@ class QState:
     def status(self, stream=None) -> dict:
         c = Counters()
         _check("qstate_status", lib().qstate_status(self._h, ctypes.byref(c), _stream(stream)))
-        return {"nonfinite": int(c.nonfinite), "saturated": int(c.saturated),
-                "pipeline_timeouts": int(c.pipeline_timeouts)}
+        return {n: int(getattr(c, n)) for n, _ in Counters._fields_}
+
+    def set_taxonomy(self, on: bool = True):
+        """Count lost / moved / reversed elements of the following steps
+        (qstate_set_taxonomy)."""
+        _check("qstate_set_taxonomy", lib().qstate_set_taxonomy(self._h, 1 if on else 0))
 
     def debug_set(self, drop_from_tile=-1, wait_polls=1 << 24):
         """Fault injection for the bounded pipeline waits (see qstate_debug_set)."""

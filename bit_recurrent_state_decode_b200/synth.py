@@ -128,6 +128,7 @@ class Workload:
     v_sigma: float = 1.0
     head_bits_multiset: tuple = ()
     description: str = ""
+    rotation: int = 0            # 1: Hadamard-rotated state (INT4+Had)
 
     @property
     def seed(self) -> int:
@@ -180,6 +181,24 @@ WORKLOADS = {
                     "scales, dynamic + persistent + yoked side by side, BDR"),
 }
 BY_INDEX = {w.index: w for w in WORKLOADS.values()}
+
+# Layout variants the pages compare against, on the shapes above (not among
+# the five decode configurations).  INT4+Had: Table 2 of "Preserving Updates
+# in Low-Bit Recurrent State Quantization", INT4 at 4.50 bits (group 32,
+# binary16 scales) with a Hadamard rotation before quantization, on the
+# 24-layer Gated DeltaNet decode.
+VARIANTS = {
+    "gdn_l24_b256_h32_d128_int4g32_had": Workload(
+        "gdn_l24_b256_h32_d128_int4g32_had", 5, GDN, 256, 32, 128, 128, 2048, 4, 32,
+        (DYNAMIC,), RTN, BF16, BF16, F16, layers=24, rotation=1,
+        description="Gated DeltaNet x24 layers, Hadamard-rotated INT4 g32 fp16 dynamic scale "
+                    "(INT4+Had), RTN, bf16"),
+}
+
+
+def workload(name: str) -> Workload:
+    """A decode configuration or a layout variant, by name."""
+    return WORKLOADS[name] if name in WORKLOADS else VARIANTS[name]
 
 
 def _draw16(seed, layer, step, tiles, field, n):

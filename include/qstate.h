@@ -116,6 +116,15 @@ typedef struct qstate_layout {
     int32_t scale_dtype;      /* QSTATE_F16 or QSTATE_F32 */
     const uint8_t* head_bits; /* NULL, or host array [heads] of 2/4/6/8 (copied);
                                  overrides `bits` of qstate_create */
+    int32_t rotation;         /* 0: none; 1: the state is kept rotated by the
+                                 Hadamard matrix H along d_v (INT4+Had of Table 2
+                                 of "Preserving Updates in Low-Bit Recurrent State
+                                 Quantization"): the stored state is S H, each
+                                 step takes H v for v and emits o = H (S H)^T q
+                                 / d_v, H the Sylvester matrix (entries +-1)
+                                 applied by the butterfly of its order; the
+                                 outputs are those of S, qstate_dequant returns
+                                 the stored S H */
 } qstate_layout;
 
 typedef struct qstate qstate;
@@ -126,6 +135,16 @@ typedef struct qstate_counters {
     uint64_t saturated;       /* binary16 scale conversions that overflowed */
     uint64_t pipeline_timeouts; /* CTAs that gave up a bounded wait for their input
                                    copies (the step's results are then undefined) */
+    uint64_t exact_path_warps; /* warp-tiles that rounded element by element (the
+                                  general form, taken when the fast form's
+                                  conditions do not hold for every row of the warp) */
+    /* Rounding taxonomy (only while qstate_set_taxonomy is on): elements with a
+     * nonzero update d = x - a, classified on the grid of the new scale with
+     * u = a * inv, w = x * inv and c = clamp(RTN(w)): reversed when c lies
+     * strictly beyond u on the side away from the update, else lost when
+     * c = clamp(RTN(u)), else moved (Figure 4 of "Preserving Updates in
+     * Low-Bit Recurrent State Quantization"); and the BDR steps applied. */
+    uint64_t lost, moved, reversed, bdr_applied;
 } qstate_counters;
 
 typedef struct qstate_sizes {
@@ -236,6 +255,15 @@ int64_t qstate_bytes_per_step(const qstate* s);
 /* Read the sticky counters: copies them device->host on stream and
  * synchronises that stream (no counterpart on the pages). */
 int qstate_status(qstate* s, qstate_counters* out, qstate_stream stream);
+
+/* Count the rounding taxonomy of every element of every following step
+ * (on = 1) or stop (on = 0, the default) into the lost / moved / reversed /
+ * bdr_applied counters of qstate_status.  The counts are diagnostics of the
+ * error accounting of "Preserving Updates in Low-Bit Recurrent State
+ * Quantization" (Figure 4, Table 5: the lost fraction); while on, steps run
+ * the general kernel and classify each element again, so they are slower;
+ * the state and outputs are unchanged.  QSTATE_EINVAL for other values. */
+int qstate_set_taxonomy(qstate* s, int on);
 
 /* Fault injection for tests of the bounded waits (no counterpart on the
  * pages).  The step kernel stages each tile's inputs with asynchronous bulk

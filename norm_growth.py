@@ -1,6 +1,6 @@
 """Norm growth of the quantized state under the three scale modes.
 
-    python -m bit_recurrent_state_decode_b200.norm_growth [--steps 32768] [--every 64]
+    python norm_growth.py [--steps 32768] [--every 64]
 
 "When Dynamic Scaling Fails" (Abstract) reports that a scale re-derived from
 the state every step feeds back into the state and makes its norm explode,
@@ -28,8 +28,12 @@ import time
 import numpy as np
 import torch
 
-from . import qstate as Q
-from . import synth
+import os
+
+sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
+
+from bit_recurrent_state_decode_b200 import qstate as Q  # noqa: E402
+from bit_recurrent_state_decode_b200 import synth  # noqa: E402
 
 
 def run(steps: int, every: int, batch: int | None = None) -> dict:

@@ -34,13 +34,13 @@ def gpu_object(wl: synth.Workload, mode: int, batch: int, layers: int) -> Q.QSta
     return Q.QState(batch, wl.heads, wl.d_k, wl.d_v, wl.kind, bits=wl.bits or 4, group=wl.group,
                     scale_mode=mode, round_mode=wl.round_mode, eps_b=wl.eps_b, layers=layers,
                     gamma=wl.gamma, qkv_dtype=wl.qkv_dtype, gate_dtype=wl.gate_dtype,
-                    scale_dtype=wl.scale_dtype, head_bits=hb)
+                    scale_dtype=wl.scale_dtype, head_bits=hb, rotation=wl.rotation)
 
 
 def oracle_state(wl: synth.Workload, mode: int, tile_heads: np.ndarray, bits=None):
     cfg = oracle.Config(wl.d_k, wl.d_v, wl.kind, wl.group, scale_mode=mode,
                         round_mode=wl.round_mode, scale_f32=wl.scale_dtype == synth.F32,
-                        gamma=wl.gamma, eps_b=wl.eps_b)
+                        gamma=wl.gamma, eps_b=wl.eps_b, rotate=wl.rotation)
     hb = wl.head_bits()
     if bits is None:
         bits = wl.bits

@@ -24,7 +24,7 @@ def _declared():
 
 def test_exports_every_declared_symbol(q):
     declared = _declared()
-    assert len(declared) == 14
+    assert len(declared) == 15
     assert sorted(q.EXPORTS) == declared
     lib = q.lib()
     for name in declared:
@@ -102,6 +102,7 @@ def test_null_object_calls(q):
     assert lib.qstate_status(None, None, None) == q.EINVAL
     assert lib.qstate_reset(None, None) == q.EINVAL
     assert lib.qstate_debug_set(None, -1, 1) == q.EINVAL
+    assert lib.qstate_set_taxonomy(None, 1) == q.EINVAL
     assert lib.qstate_destroy(None) == q.EINVAL
 
 

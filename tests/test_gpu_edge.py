@@ -84,11 +84,11 @@ def test_yoked_non_square(dk, dv, kind):
 
 
 def test_stage_sizes_sharing_one_kernel():
-    """A GLA INT8 g32 object (group scales and the gate vector staged) is
+    """A GLA INT8 g16 object (group scales and the gate vector staged) is
     created before a Mamba2 INT8 per-token object (neither staged): both
     launch the same kernel.  Creating the second must not lower the
     kernel's shared-memory limit below what the first launches with."""
-    gla = C3.scaled(batch=2, heads=2, layers=1, bits=8, group=32, qkv_dtype=synth.F32,
+    gla = C3.scaled(batch=2, heads=2, layers=1, bits=8, group=16, qkv_dtype=synth.F32,
                     scale_modes=(synth.PERSISTENT,))
     mam = C2.scaled(batch=2, heads=2, layers=1, d_v=128)
     first = gpu_object(gla, synth.PERSISTENT, 2, 1)

@@ -65,7 +65,8 @@ def test_static_staging_matches_allocating_host_step():
     for x_, y_ in zip(a.export(), b.export()):
         if x_ is not None:
             assert torch.equal(x_, y_)
-    assert b.status() == {"nonfinite": 0, "saturated": 0, "pipeline_timeouts": 0}
+    st = b.status()
+    assert (st["nonfinite"], st["saturated"], st["pipeline_timeouts"]) == (0, 0, 0)
     a.close()
     b.close()
 
