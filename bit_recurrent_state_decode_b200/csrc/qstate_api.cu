@@ -12,6 +12,7 @@
 
 #include "qstate.h"
 #include "qstate_dispatch.h"
+#include "qstate_lrb.cuh"
 
 namespace qs {
 void launch_dequant_64_64(const StepParams&, float*, cudaStream_t);
@@ -62,6 +63,18 @@ struct qstate {
     int dyn_smem = 0;                 // bytes of pipeline stages per CTA
     unsigned wait_polls = qs::kWaitPolls;
     long long drop_from = -1;
+    // Low-Rank Bypass (qstate_set_lrb): bypass columns, coefficients, slot
+    // counts and the decay since the last merge, per tile
+    bool lrb = false;
+    int lrb_k = 0, lrb_m = 0;
+    float lrb_eps = 0.0f;
+    uint16_t* d_lu = nullptr;
+    uint16_t* d_lw = nullptr;
+    float* d_lg = nullptr;
+    int* d_ln = nullptr;
+    float* d_lD = nullptr;
+    const qs::LrbEntry* lrb_entry = nullptr;
+    int lrb_grid = 1, lrb_smem = 0;
     // set by qstate_import: the next step takes the general tile bodies (an
     // imported state may hold the code -2^(bits-1), which no step produces)
     bool import_pending = false;
@@ -141,6 +154,28 @@ void free_all(qstate* s) {
     cudaFree(s->st_v);
     cudaFree(s->st_g);
     cudaFree(s->st_out);
+    cudaFree(s->d_lu);
+    cudaFree(s->d_lw);
+    cudaFree(s->d_lg);
+    cudaFree(s->d_ln);
+    cudaFree(s->d_lD);
+}
+
+// bypass empty, D = 1 for every tile
+int zero_bypass(qstate* s, cudaStream_t st) {
+    if (!s->lrb || s->tiles == 0) return QSTATE_OK;
+    const int64_t K = s->lrb_k + s->lrb_m;
+    if (cudaMemsetAsync(s->d_lu, 0, s->tiles * K * s->L.d_k * 2, st) != cudaSuccess ||
+        cudaMemsetAsync(s->d_lw, 0, s->tiles * K * s->L.d_v * 2, st) != cudaSuccess ||
+        cudaMemsetAsync(s->d_lg, 0, s->tiles * K * 4, st) != cudaSuccess ||
+        cudaMemsetAsync(s->d_ln, 0, s->tiles * 2 * 4, st) != cudaSuccess)
+        return QSTATE_ECUDA;
+    // D = 1: copied from a host array (a copy from pageable memory has left
+    // the array when the call returns)
+    std::vector<float> ones((size_t)s->tiles, 1.0f);
+    if (cudaMemcpyAsync(s->d_lD, ones.data(), ones.size() * 4, cudaMemcpyHostToDevice, st) != cudaSuccess)
+        return QSTATE_ECUDA;
+    return QSTATE_OK;
 }
 
 int zero_state(qstate* s, cudaStream_t st) {
@@ -370,7 +405,9 @@ int qstate_destroy(qstate* s) {
 
 int qstate_reset(qstate* s, qstate_stream stream) {
     if (!s) return QSTATE_EINVAL;
-    return zero_state(s, (cudaStream_t)stream);
+    int rc = zero_state(s, (cudaStream_t)stream);
+    if (rc == QSTATE_OK) rc = zero_bypass(s, (cudaStream_t)stream);
+    return rc;
 }
 
 int qstate_step(qstate* s, const void* q, const void* k, const void* v, const void* gates,
@@ -389,6 +426,11 @@ int qstate_step(qstate* s, const void* q, const void* k, const void* v, const vo
     p.v = v;
     p.gates = gates;
     p.out = out;
+    if (s->lrb) {
+        qs::LrbParams Lp{s->d_lu, s->d_lw, s->d_lg, s->d_ln, s->d_lD, s->lrb_k, s->lrb_m, s->lrb_eps};
+        s->lrb_entry->launch(p, Lp, s->lrb_grid, s->lrb_smem, (cudaStream_t)stream);
+        return cudaGetLastError() == cudaSuccess ? QSTATE_OK : QSTATE_ECUDA;
+    }
     if (s->taxonomy)
         s->entry_general->launch(p, s->grid_general, s->dyn_smem, (cudaStream_t)stream);
     else
@@ -489,15 +531,85 @@ int qstate_import(qstate* s, const void* codes, const void* scales, const float*
         cudaMemcpyAsync(s->d_ref, ref, s->ref_bytes, cudaMemcpyDefault, st) != cudaSuccess)
         return QSTATE_ECUDA;
     s->import_pending = true;
-    return QSTATE_OK;
+    return zero_bypass(s, st);
 }
 
 int64_t qstate_bytes_per_step(const qstate* s) {
     if (!s) return -1;
     const int64_t dk = s->L.d_k, dv = s->L.d_v;
+    const int64_t ops = s->tiles * ((2 * dk + dv) * s->in_size + s->n_gate * s->gate_size + dv * 4);
+    if (s->lrb) {
+        // averaged over a merge cycle of m steps: the state is read every step
+        // and written at the merge; the columns held at the start of a step
+        // (k + (m - 1) / 2 on average) are read, one column and the
+        // coefficients written; the residual columns written at the merge
+        const int64_t k = s->lrb_k, m = s->lrb_m;
+        const int64_t col = (dk + dv) * 2 + 4;
+        int64_t b = m * (s->code_bytes + s->scale_bytes) + s->code_bytes + s->scale_bytes;
+        b += s->tiles * ((k * m + m * (m - 1) / 2) * col + m * col + k * col + m * 16);
+        return b / m + ops;
+    }
     int64_t b = 2 * s->code_bytes + 2 * s->scale_bytes + 2 * s->ref_bytes;
-    b += s->tiles * ((2 * dk + dv) * s->in_size + s->n_gate * s->gate_size + dv * 4);
-    return b;
+    return b + ops;
+}
+
+int qstate_set_lrb(qstate* s, int k, int m, float eps_l) {
+    if (!s || s->lrb) return QSTATE_EINVAL;
+    if (k < 0 || k > 1 || m < 1 || k + m > qs::kLrbMaxCols) return QSTATE_EINVAL;
+    if (!(eps_l >= 0.0f) || !std::isfinite(eps_l)) return QSTATE_EINVAL;
+    if (s->L.kind == QSTATE_GLA || s->scale_mode == QSTATE_YOKED || s->L.rotation ||
+        !s->head_bits.empty() || !(s->bits == 4 || s->bits == 8) || s->L.d_k != s->L.d_v)
+        return QSTATE_EUNSUPPORTED;
+    int rc = check_device(s);
+    if (rc != QSTATE_OK) return rc;
+    const int d = s->L.d_k;
+    const int idx = ((((d == 128) * 2 + (s->bits == 8)) * 2 + (s->L.kind == QSTATE_GDN)) * 2 +
+                     (s->round_mode == QSTATE_BDR)) * 2 + (s->L.qkv_dtype == QSTATE_BF16);
+    const qs::LrbEntry* e = &qs::lrb_table()[idx];
+    const int smem = k == 1 ? 64 * e->threads * 4 : 0;
+    const int per_sm = e->blocks_per_sm(smem);
+    if (per_sm < 1) { cudaGetLastError(); return QSTATE_EUNSUPPORTED; }
+    const int64_t K = k + m, T = s->tiles;
+    auto alloc = [&](void** p, size_t n) -> bool { return !n || cudaMalloc(p, n) == cudaSuccess; };
+    if (!alloc((void**)&s->d_lu, T * K * s->L.d_k * 2) || !alloc((void**)&s->d_lw, T * K * s->L.d_v * 2) ||
+        !alloc((void**)&s->d_lg, T * K * 4) || !alloc((void**)&s->d_ln, T * 2 * 4) ||
+        !alloc((void**)&s->d_lD, T * 4)) {
+        cudaGetLastError();
+        cudaFree(s->d_lu); cudaFree(s->d_lw); cudaFree(s->d_lg); cudaFree(s->d_ln); cudaFree(s->d_lD);
+        s->d_lu = s->d_lw = nullptr;
+        s->d_lg = s->d_lD = nullptr;
+        s->d_ln = nullptr;
+        return QSTATE_ENOMEM;
+    }
+    s->lrb = true;
+    s->lrb_k = k;
+    s->lrb_m = m;
+    s->lrb_eps = eps_l;
+    s->lrb_entry = e;
+    s->lrb_smem = smem;
+    int sms = 0;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, s->device);
+    int64_t g = (int64_t)sms * per_sm;
+    if (T < g) g = T > 0 ? T : 1;
+    s->lrb_grid = (int)g;
+    rc = zero_bypass(s, nullptr);
+    if (rc == QSTATE_OK && cudaDeviceSynchronize() != cudaSuccess) rc = QSTATE_ECUDA;
+    return rc;
+}
+
+int qstate_lrb_export(const qstate* s, uint16_t* u, uint16_t* w, float* g, int32_t* n, float* D,
+                      qstate_stream stream) {
+    if (!s || !s->lrb || !u || !w || !g || !n || !D) return QSTATE_EINVAL;
+    if (s->tiles == 0) return QSTATE_OK;
+    const int64_t K = s->lrb_k + s->lrb_m, T = s->tiles;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (cudaMemcpyAsync(u, s->d_lu, T * K * s->L.d_k * 2, cudaMemcpyDefault, st) != cudaSuccess ||
+        cudaMemcpyAsync(w, s->d_lw, T * K * s->L.d_v * 2, cudaMemcpyDefault, st) != cudaSuccess ||
+        cudaMemcpyAsync(g, s->d_lg, T * K * 4, cudaMemcpyDefault, st) != cudaSuccess ||
+        cudaMemcpyAsync(n, s->d_ln, T * 2 * 4, cudaMemcpyDefault, st) != cudaSuccess ||
+        cudaMemcpyAsync(D, s->d_lD, T * 4, cudaMemcpyDefault, st) != cudaSuccess)
+        return QSTATE_ECUDA;
+    return QSTATE_OK;
 }
 
 int qstate_debug_set(qstate* s, int64_t drop_from_tile, uint32_t wait_polls) {

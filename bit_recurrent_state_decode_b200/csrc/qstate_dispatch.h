@@ -34,6 +34,17 @@ const StepEntry* step_table_128_128_1();
 // ((((d_k == 128) * 2 + (bits == 8)) * 2 + (group == 64)) * 2 + gla) * 2 + bf16.
 const StepEntry* rows_table();
 
+// The decode step with a Low-Rank Bypass (d_k = d_v in {64, 128}, 4- or
+// 8-bit codes): 32 entries indexed by
+// ((((d == 128) * 2 + (bits == 8)) * 2 + gdn) * 2 + bdr) * 2 + bf16.
+struct LrbParams;
+struct LrbEntry {
+    void (*launch)(const StepParams&, const LrbParams&, int grid, int dyn_smem, cudaStream_t);
+    int (*blocks_per_sm)(int dyn_smem);
+    int threads;
+};
+const LrbEntry* lrb_table();
+
 // 0 = per-head widths, then 2, 4, 6, 8, 32 bits; -1 if invalid
 inline int bits_index(int bits) {
     switch (bits) {

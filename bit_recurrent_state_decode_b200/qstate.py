@@ -25,8 +25,8 @@ F32, BF16, F16 = 0, 1, 2
 # every symbol include/qstate.h declares
 EXPORTS = ("qstate_create", "qstate_destroy", "qstate_reset", "qstate_step", "qstate_step_host",
            "qstate_step_host_static", "qstate_dequant", "qstate_export", "qstate_import", "qstate_get_sizes",
-           "qstate_bytes_per_step", "qstate_status", "qstate_set_taxonomy", "qstate_debug_set",
-           "qstate_error_string")
+           "qstate_bytes_per_step", "qstate_status", "qstate_set_taxonomy", "qstate_set_lrb",
+           "qstate_lrb_export", "qstate_debug_set", "qstate_error_string")
 
 
 class QStateError(RuntimeError):
@@ -83,6 +83,8 @@ def lib():
         L.qstate_status.argtypes = [P, ctypes.POINTER(Counters), S]
         L.qstate_debug_set.argtypes = [P, ctypes.c_int64, ctypes.c_uint32]
         L.qstate_set_taxonomy.argtypes = [P, I]
+        L.qstate_set_lrb.argtypes = [P, I, I, ctypes.c_float]
+        L.qstate_lrb_export.argtypes = [P, P, P, P, P, P, S]
         L.qstate_error_string.argtypes = [I]
         L.qstate_error_string.restype = ctypes.c_char_p
         for name in EXPORTS:
@@ -146,6 +148,7 @@ class QState:
         self.qkv_dtype, self.gate_dtype, self.scale_dtype = qkv_dtype, gate_dtype, scale_dtype
         self.head_bits = None if head_bits is None else [int(b) for b in head_bits]
         self.rotation = int(rotation)
+        self.lrb = None
         z = Sizes()
         _check("qstate_get_sizes", lib().qstate_get_sizes(self._h, ctypes.byref(z)))
         self.sizes = {n: int(getattr(z, n)) for n, _ in Sizes._fields_}
@@ -289,6 +292,30 @@ class QState:
         """Count lost / moved / reversed elements of the following steps
         (qstate_set_taxonomy)."""
         _check("qstate_set_taxonomy", lib().qstate_set_taxonomy(self._h, 1 if on else 0))
+
+    def set_lrb(self, k: int, m: int, eps_l: float):
+        """Low-Rank Bypass with a rank-k residual, a merge every m steps and
+        the merge threshold eps_l (qstate_set_lrb); before the first step."""
+        _check("qstate_set_lrb", lib().qstate_set_lrb(self._h, int(k), int(m), float(eps_l)))
+        self.lrb = (int(k), int(m), float(eps_l))
+
+    def lrb_export(self, stream=None) -> dict:
+        """The bypass as new CUDA tensors: u [tiles, k+m, d_k] and
+        w [tiles, k+m, d_v] (float16), g [tiles, k+m], n [tiles, 2]
+        (residual and fresh columns held), D [tiles]."""
+        if self.lrb is None:
+            raise QStateError("qstate_lrb_export", 1)
+        K = self.lrb[0] + self.lrb[1]
+        T = self.tiles
+        dev = f"cuda:{self.device}"
+        u = torch.empty((T, K, self.d_k), dtype=torch.float16, device=dev)
+        w = torch.empty((T, K, self.d_v), dtype=torch.float16, device=dev)
+        g = torch.empty((T, K), dtype=torch.float32, device=dev)
+        n = torch.empty((T, 2), dtype=torch.int32, device=dev)
+        D = torch.empty((T,), dtype=torch.float32, device=dev)
+        _check("qstate_lrb_export", lib().qstate_lrb_export(self._h, _ptr(u), _ptr(w), _ptr(g), _ptr(n),
+                                                            _ptr(D), _stream(stream)))
+        return {"u": u, "w": w, "g": g, "n": n, "D": D}
 
     def debug_set(self, drop_from_tile=-1, wait_polls=1 << 24):
         """Fault injection for the bounded pipeline waits (see qstate_debug_set)."""

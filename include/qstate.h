@@ -237,7 +237,9 @@ int qstate_dequant(const qstate* s, float* S_out, qstate_stream stream);
 /* Copy the raw state out to / in from caller device buffers of
  * qstate_sizes() bytes (codes, scales, ref; ref may be NULL if not yoked).
  * Used for checkpoints and teacher-forced parity (no counterpart on the
- * pages; the layouts are the ones above). */
+ * pages; the layouts are the ones above).  With a Low-Rank Bypass these are
+ * the quantized part only (qstate_dequant likewise); import also empties the
+ * bypass and sets D = 1. */
 int qstate_export(const qstate* s, void* codes, void* scales, float* ref,
                   qstate_stream stream);
 int qstate_import(qstate* s, const void* codes, const void* scales, const float* ref,
@@ -264,6 +266,33 @@ int qstate_status(qstate* s, qstate_counters* out, qstate_stream stream);
  * the general kernel and classify each element again, so they are slower;
  * the state and outputs are unchanged.  QSTATE_EINVAL for other values. */
 int qstate_set_taxonomy(qstate* s, int on);
+
+/* Switch the object to steps with a Low-Rank Bypass (LRB) of "Preserving
+ * Updates in Low-Bit Recurrent State Quantization" (Abstract, Figure 3,
+ * Tables 6, 8, 9), before its first step.  Each tile keeps, next to its
+ * codes and scales, up to k + m bypass columns (u in binary16 [d_k], w in
+ * binary16 [d_v], a binary32 coefficient) and a binary32 decay D: every step
+ * decays D and the coefficients, adds the step's update as a new column
+ * (Gated DeltaNet: e = v - r with r over the whole state, codes plus bypass)
+ * and emits o from the whole state; codes and scales change only every m
+ * steps, when the bypass elements at least eps_l grid steps (of the decayed
+ * grid) large are merged into the state and it is requantized with the
+ * object's scale and rounding modes (BDR with the merged update as d), D
+ * reset to 1 and the rest kept as its leading singular pair (k = 1, found by
+ * power iteration) or dropped (k = 0).  The state a tile stands for is
+ * D * dequant(codes) + sum_l g_l u_l w_l^T.
+ * k in {0, 1}, m >= 1, k + m <= 32, eps_l >= 0.  Supported for RetNet,
+ * Mamba2 and Gated DeltaNet objects with one code width of 4 or 8 bits,
+ * d_k = d_v in {64, 128}, dynamic or persistent scales, no rotation
+ * (QSTATE_EUNSUPPORTED otherwise); allocates the bypass (QSTATE_ENOMEM).
+ * QSTATE_EINVAL if already set or for invalid k, m, eps_l. */
+int qstate_set_lrb(qstate* s, int k, int m, float eps_l);
+
+/* Copy an LRB object's bypass to caller buffers (device or host):
+ * u [tiles][k+m][d_k] and w [tiles][k+m][d_v] binary16 bit patterns,
+ * g [tiles][k+m], n [tiles][2] (residual and fresh columns held), D [tiles]. */
+int qstate_lrb_export(const qstate* s, uint16_t* u, uint16_t* w, float* g, int32_t* n, float* D,
+                      qstate_stream stream);
 
 /* Fault injection for tests of the bounded waits (no counterpart on the
  * pages).  The step kernel stages each tile's inputs with asynchronous bulk

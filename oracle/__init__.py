@@ -106,7 +106,7 @@ def lib():
         _lib.or_lrb_step.restype = ctypes.c_int
         _lib.or_lrb_step.argtypes = [ctypes.POINTER(_Cfg), ctypes.POINTER(LrbCfg), ctypes.c_int64,
                                      P, P, P, P, P, P, P, P, P, P, P, P, P, P, P,
-                                     ctypes.POINTER(Counts), P]
+                                     ctypes.POINTER(Counts), P, P]
         _lib.or_rank_k.argtypes = [ctypes.c_int, ctypes.c_int, P, ctypes.c_int, P, P, P]
         _lib.or_lrb_bits.restype = ctypes.c_double
         _lib.or_lrb_bits.argtypes = [ctypes.c_int] * 5 + [ctypes.c_double]
@@ -353,7 +353,8 @@ class LrbState(State):
     code): codes and scales as State, plus per tile u [k+m][d_k] and
     w [k+m][d_v] (binary16 patterns), g [k+m] and the slot counts."""
 
-    def __init__(self, cfg: Config, tile_bits, k: int, m: int, eps_l: float):
+    def __init__(self, cfg: Config, tile_bits, k: int, m: int, eps_l: float,
+                 keep_resid: bool = False):
         super().__init__(cfg, tile_bits)
         self.lcfg = LrbCfg(k, m, eps_l)
         T = self.ntiles
@@ -366,6 +367,8 @@ class LrbState(State):
         self.D = np.ones(T, np.float32)     # decay since the last merge
         self.merged = np.zeros(T, np.int32)
         self.peak_cols = 0                  # most columns held at once (before a merge)
+        # the unmerged rest of the bypass at each tile's last merge
+        self.resid = np.zeros((T, cfg.d_k, cfg.d_v), np.float32) if keep_resid else None
 
     def step(self, q, k, v, alpha=None, beta=None, threads: int = 1):
         cfg = self.cfg
@@ -383,7 +386,8 @@ class LrbState(State):
                                _ptr(self.u), _ptr(self.w), _ptr(self.g), _ptr(self.nres),
                                _ptr(self.nnew), _ptr(self.D), _ptr(q), _ptr(k), _ptr(v),
                                _ptr(alpha),
-                               _ptr(beta), _ptr(out), ctypes.byref(cnt), _ptr(self.merged))
+                               _ptr(beta), _ptr(out), ctypes.byref(cnt), _ptr(self.merged),
+                               _ptr(self.resid))
         if rc != 0:
             raise ValueError("oracle rejected the LRB configuration")
         self._add_counts(cnt)

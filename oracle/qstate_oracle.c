@@ -634,7 +634,8 @@ static void lrb_tile_step(const or_cfg* c, const or_lrb_cfg* L, int bits, int8_t
                           float* scales, uint16_t* u, uint16_t* w, float* g, int* nres, int* nnew,
                           float* D,
                           const float* q, const float* k, const float* v, const float* alpha,
-                          float beta, float* out, or_counts* cnt, int* merged_out)
+                          float beta, float* out, or_counts* cnt, int* merged_out,
+                          float* resid_out)
 {
     const int dk = c->d_k, dv = c->d_v;
     const int qmax = (1 << (bits - 1)) - 1;
@@ -745,6 +746,7 @@ static void lrb_tile_step(const or_cfg* c, const or_lrb_cfg* L, int bits, int8_t
             }
     }
     if (merge) {
+        if (resid_out) memcpy(resid_out, P, sizeof(float) * n_el);
         /* the unmerged residual as its best rank-k approximation */
         const int kk = L->k;
         if (kk > 0) {
@@ -779,7 +781,8 @@ static void lrb_tile_step(const or_cfg* c, const or_lrb_cfg* L, int bits, int8_t
 int or_lrb_step(const or_cfg* c, const or_lrb_cfg* L, int64_t ntiles, const int* tile_bits,
                 int8_t* codes, float* scales, uint16_t* u, uint16_t* w, float* g, int* nres,
                 int* nnew, float* D, const float* q, const float* k, const float* v,
-                const float* alpha, const float* beta, float* out, or_counts* cnt, int* merged)
+                const float* alpha, const float* beta, float* out, or_counts* cnt, int* merged,
+                float* resid)
 {
     if (!valid_lrb(c, L)) return -1;
     const int dk = c->d_k, dv = c->d_v, K = L->k + L->m, nsc = or_n_scales(c);
@@ -789,6 +792,7 @@ int or_lrb_step(const or_cfg* c, const or_lrb_cfg* L, int64_t ntiles, const int*
         lrb_tile_step(c, L, tile_bits[t], codes + t * dk * dv, scales + t * nsc,
                       u + t * K * dk, w + t * K * dv, g + t * K, nres + t, nnew + t, D + t,
                       q + t * dk, k + t * dk, v + t * dv, alpha ? alpha + t : NULL,
-                      beta ? beta[t] : 0.0f, out + t * dv, cnt, merged ? merged + t : NULL);
+                      beta ? beta[t] : 0.0f, out + t * dv, cnt, merged ? merged + t : NULL,
+                      resid ? resid + t * (int64_t)dk * dv : NULL);
     return 0;
 }

@@ -133,11 +133,14 @@ typedef struct {
  * [k+m][d_k] and w [k+m][d_v] binary16 bit patterns, g [k+m] binary32,
  * nres / nnew the residual and fresh slot counts, D [ntiles] the decay since
  * the last merge (1 at the start).  merged (may be NULL):
- * per tile, the number of elements merged by this step.  -1 if invalid. */
+ * per tile, the number of elements merged by this step.  resid (may be
+ * NULL): [ntiles][d_k][d_v], at a merge the unmerged rest of the bypass
+ * (before its rank-k approximation), untouched otherwise.  -1 if invalid. */
 int or_lrb_step(const or_cfg* c, const or_lrb_cfg* L, int64_t ntiles, const int* tile_bits,
                 int8_t* codes, float* scales, uint16_t* u, uint16_t* w, float* g, int* nres,
                 int* nnew, float* D, const float* q, const float* k, const float* v,
-                const float* alpha, const float* beta, float* out, or_counts* cnt, int* merged);
+                const float* alpha, const float* beta, float* out, or_counts* cnt, int* merged,
+                float* resid);
 
 /* Top-k singular triplets of a rows x cols fp64 matrix (Jacobi on R^T R). */
 void or_rank_k(int rows, int cols, const double* R, int k, double* s, double* U, double* V);

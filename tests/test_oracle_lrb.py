@@ -151,3 +151,47 @@ def test_lrb_tracks_the_unquantized_state_better(orc):
     e_plain = np.linalg.norm(plain.dequant() - S)
     e_lrb = np.linalg.norm(np.stack([lrb.state(t) for t in range(8)]) - S)
     assert e_lrb < 0.8 * e_plain, (e_lrb, e_plain)
+
+
+def test_residual_output_is_the_unmerged_bypass(orc):
+    """With a threshold nothing reaches, the residual handed out at a merge
+    is the whole decayed bypass (the fp64 sum of its columns, within fp32
+    rounding), and the kept rank-1 pair is numpy's leading singular pair of
+    it (within binary16 rounding).  The first merge finds no quantized state
+    (all scales 0: a grid step of 0), so everything merges there and the
+    residual is zero; the second merge is the one that keeps a residual.
+    With threshold 0 everything merges at every merge."""
+    wl = C1
+    cfg = oracle.Config(64, 64, synth.RETNET, 32, scale_mode=synth.DYNAMIC, gamma=wl.gamma)
+    st = oracle.LrbState(cfg, [4], k=1, m=3, eps_l=1e30, keep_resid=True)
+    gam = float(np.float32(wl.gamma))
+    for s in range(6):
+        nb = int(st.nres[0] + st.nnew[0])
+        u0 = st.u[0, :nb].view(np.float16).astype(np.float64).copy()
+        w0 = st.w[0, :nb].view(np.float16).astype(np.float64).copy()
+        g0 = st.g[0, :nb].astype(np.float64).copy()
+        x = synth.gen_step(wl, s, tiles=np.arange(1))
+        q, kk, v, _ = x.as_f32(wl)
+        st.step(q, kk, v)
+        if s == 2:
+            assert not st.resid.any() and not st.u[0, 0].any() and not st.w[0, 0].any()
+    assert nb == 3
+    un = st.u[0, nb].view(np.float16).astype(np.float64)
+    wn = st.w[0, nb].view(np.float16).astype(np.float64)
+    P = np.outer(un, wn)
+    for l in range(nb):
+        P = P + float(np.float32(gam * g0[l])) * np.outer(u0[l], w0[l])
+    R = st.resid[0].astype(np.float64)
+    assert np.abs(P).max() > 0 and np.abs(R - P).max() <= 1e-6 * np.abs(P).max()
+    U, S, Vt = np.linalg.svd(R)
+    best = S[0] * np.outer(U[:, 0], Vt[0])
+    kept = float(st.g[0, 0]) * np.outer(st.u[0, 0].view(np.float16).astype(np.float64),
+                                        st.w[0, 0].view(np.float16).astype(np.float64))
+    assert np.linalg.norm(kept - best) <= 2e-3 * np.linalg.norm(best)
+
+    st0 = oracle.LrbState(cfg, [4], k=1, m=3, eps_l=0.0, keep_resid=True)
+    for s in range(6):
+        x = synth.gen_step(wl, s, tiles=np.arange(1))
+        q, kk, v, _ = x.as_f32(wl)
+        st0.step(q, kk, v)
+    assert not st0.resid.any() and not st0.u[0, 0].any() and not st0.w[0, 0].any()
