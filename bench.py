@@ -50,7 +50,8 @@ def parse():
     ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
-                    help="a workload name, or 'all' for one line per workload in ALL_WORKLOADS")
+                    help="a workload name, 'all' for one line per workload in ALL_WORKLOADS, "
+                         "or 'variants' for one line per layout variant (synth.VARIANTS)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--replicas", type=int, default=0,
                     help="independent layer replicas (0: enough to exceed 4x L2)")
@@ -161,6 +162,13 @@ def cpu_oracle_rate(wl, seconds=10.0, threads=None, max_steps=None, tiles=None, 
     import oracle
     from bit_recurrent_state_decode_b200 import synth
     threads = threads or os.cpu_count() or 1
+    cycle = 1
+    if wl.lrb:
+        # whole merge cycles (m steps, one of them a merge), after one cycle
+        # that fills the residual; the bypass step is single-threaded
+        cycle = wl.lrb[1]
+        warmup = max(warmup, cycle)
+        tiles = tiles or 32
     # enough tiles per step that the worker threads, not their dispatch, set the rate
     tiles = tiles or max(threads * 64, 8)
     tiles = min(tiles, wl.tiles_per_layer)
@@ -171,8 +179,13 @@ def cpu_oracle_rate(wl, seconds=10.0, threads=None, max_steps=None, tiles=None, 
     for mode in wl.scale_modes:
         cfg = oracle.Config(wl.d_k, wl.d_v, wl.kind, wl.group, scale_mode=mode,
                             round_mode=wl.round_mode, scale_f32=wl.scale_dtype == synth.F32,
-                            gamma=wl.gamma, eps_b=wl.eps_b)
-        states.append(oracle.State(cfg, tile_bits))
+                            gamma=wl.gamma, eps_b=wl.eps_b, rotate=wl.rotation)
+        if wl.lrb:
+            # the oracle's bypass step runs its tiles on one host thread
+            states.append(oracle.LrbState(cfg, tile_bits, *wl.lrb))
+            threads = 1
+        else:
+            states.append(oracle.State(cfg, tile_bits))
     steps = 0
     busy = 0.0
     for w in range(warmup):
@@ -186,7 +199,8 @@ def cpu_oracle_rate(wl, seconds=10.0, threads=None, max_steps=None, tiles=None, 
         for st in states:
             st.step(q, k, v, alpha, beta, threads=threads)
     t_end = time.perf_counter() + seconds
-    while time.perf_counter() < t_end and (max_steps is None or steps < max_steps):
+    while ((time.perf_counter() < t_end or steps % cycle) and
+           (max_steps is None or steps < max_steps)):
         x = synth.gen_step(wl, warmup + steps, tiles=sel)
         q, k, v, g = x.as_f32(wl)
         alpha = beta = None
@@ -220,11 +234,14 @@ def run_ours(args, rank, world, local_rank):
     hb = wl0.head_bits()
 
     def make(mode, layers):
-        return Q.QState(wl0.batch, wl0.heads, wl0.d_k, wl0.d_v, wl0.kind, bits=wl0.bits or 4,
-                        group=wl0.group, scale_mode=mode, round_mode=wl0.round_mode,
-                        eps_b=wl0.eps_b, layers=layers, gamma=wl0.gamma,
-                        qkv_dtype=wl0.qkv_dtype, gate_dtype=wl0.gate_dtype,
-                        scale_dtype=wl0.scale_dtype, head_bits=hb)
+        o = Q.QState(wl0.batch, wl0.heads, wl0.d_k, wl0.d_v, wl0.kind, bits=wl0.bits or 4,
+                     group=wl0.group, scale_mode=mode, round_mode=wl0.round_mode,
+                     eps_b=wl0.eps_b, layers=layers, gamma=wl0.gamma,
+                     qkv_dtype=wl0.qkv_dtype, gate_dtype=wl0.gate_dtype,
+                     scale_dtype=wl0.scale_dtype, head_bits=hb, rotation=wl0.rotation)
+        if wl0.lrb:
+            o.set_lrb(*wl0.lrb)
+        return o
 
     probe = make(wl0.scale_modes[0], 1)
     per_layer = sum(probe.sizes[k] for k in ("code_bytes", "scale_bytes", "ref_bytes")) \
@@ -355,6 +372,7 @@ def run_ours(args, rank, world, local_rank):
                "steps": Ke}
 
     status = [o.status() for o in objs]
+    kernel_name = dom.kernel
     for o in objs:
         o.close()
 
@@ -395,7 +413,7 @@ def run_ours(args, rank, world, local_rank):
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_source": peak_kind,
                      "frac_of_nominal_8TBps": achieved / NOMINAL_HBM_GBS,
-                     "traffic": traffic, "kernel": "qs::step_kernel",
+                     "traffic": traffic, "kernel": "qs::" + kernel_name,
                      "bytes_per_launch": dom_bytes, "launch_ms": launch_ms},
         "gpu_launches": K * len(objs),
         "clocks": clk,
@@ -439,7 +457,7 @@ def read_traffic(workload, tiles=None):
 # ------------------------------------------------------------------ reference arm
 def run_reference(args):
     from bit_recurrent_state_decode_b200 import synth
-    wl = synth.workload(DEFAULT_WORKLOAD if args.workload == "all" else args.workload)
+    wl = synth.workload(DEFAULT_WORKLOAD if args.workload in ("all", "variants") else args.workload)
     K = args.steps or 50
     W = args.warmup
     threads = os.cpu_count() or 1
@@ -480,7 +498,13 @@ def main():
         torch.cuda.set_device(local_rank)
         tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                  device_id=torch.device("cuda", local_rank))
-    names = ALL_WORKLOADS if args.workload == "all" else (args.workload,)
+    if args.workload == "all":
+        names = ALL_WORKLOADS
+    elif args.workload == "variants":
+        from bit_recurrent_state_decode_b200 import synth
+        names = tuple(synth.VARIANTS)
+    else:
+        names = (args.workload,)
     for name in names:
         args.workload = name
         res = run_ours(args, rank, world, local_rank)

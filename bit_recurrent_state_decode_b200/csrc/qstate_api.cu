@@ -58,6 +58,7 @@ struct qstate {
     // the general kernel, when `entry` is a specialised one (the taxonomy
     // counts run in the general kernel only)
     const qs::StepEntry* entry_general = nullptr;
+    const char* entry_name = "step_kernel";
     int grid_general = 1;
     bool taxonomy = false;
     int dyn_smem = 0;                 // bytes of pipeline stages per CTA
@@ -320,6 +321,7 @@ int qstate_create(const qstate_layout* L, int bits, int group, qstate_scale_mode
         const int ridx = ((((dk == 128) * 2 + (bits == 8)) * 2 + (group == 64)) * 2 +
                           (L->kind == QSTATE_GLA)) * 2 + bf;
         s->entry = &qs::rows_table()[ridx];
+        s->entry_name = "rows_kernel";
     }
     if (!s->entry->launch) {
         free_all(s);
@@ -595,6 +597,13 @@ int qstate_set_lrb(qstate* s, int k, int m, float eps_l) {
     rc = zero_bypass(s, nullptr);
     if (rc == QSTATE_OK && cudaDeviceSynchronize() != cudaSuccess) rc = QSTATE_ECUDA;
     return rc;
+}
+
+const char* qstate_kernel(const qstate* s) {
+    if (!s) return "";
+    if (s->lrb) return "lrb_kernel";
+    if (s->taxonomy || s->L.rotation) return "step_kernel";
+    return s->entry_name;
 }
 
 int qstate_lrb_export(const qstate* s, uint16_t* u, uint16_t* w, float* g, int32_t* n, float* D,

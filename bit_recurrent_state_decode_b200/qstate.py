@@ -26,7 +26,7 @@ F32, BF16, F16 = 0, 1, 2
 EXPORTS = ("qstate_create", "qstate_destroy", "qstate_reset", "qstate_step", "qstate_step_host",
            "qstate_step_host_static", "qstate_dequant", "qstate_export", "qstate_import", "qstate_get_sizes",
            "qstate_bytes_per_step", "qstate_status", "qstate_set_taxonomy", "qstate_set_lrb",
-           "qstate_lrb_export", "qstate_debug_set", "qstate_error_string")
+           "qstate_lrb_export", "qstate_kernel", "qstate_debug_set", "qstate_error_string")
 
 
 class QStateError(RuntimeError):
@@ -85,10 +85,12 @@ def lib():
         L.qstate_set_taxonomy.argtypes = [P, I]
         L.qstate_set_lrb.argtypes = [P, I, I, ctypes.c_float]
         L.qstate_lrb_export.argtypes = [P, P, P, P, P, P, S]
+        L.qstate_kernel.argtypes = [P]
+        L.qstate_kernel.restype = ctypes.c_char_p
         L.qstate_error_string.argtypes = [I]
         L.qstate_error_string.restype = ctypes.c_char_p
         for name in EXPORTS:
-            if name not in ("qstate_bytes_per_step", "qstate_error_string"):
+            if name not in ("qstate_bytes_per_step", "qstate_error_string", "qstate_kernel"):
                 getattr(L, name).restype = I
         _lib = L
     return _lib
@@ -292,6 +294,11 @@ class QState:
         """Count lost / moved / reversed elements of the following steps
         (qstate_set_taxonomy)."""
         _check("qstate_set_taxonomy", lib().qstate_set_taxonomy(self._h, 1 if on else 0))
+
+    @property
+    def kernel(self) -> str:
+        """The kernel the next step launches (qstate_kernel)."""
+        return lib().qstate_kernel(self._h).decode()
 
     def set_lrb(self, k: int, m: int, eps_l: float):
         """Low-Rank Bypass with a rank-k residual, a merge every m steps and

@@ -129,6 +129,7 @@ class Workload:
     head_bits_multiset: tuple = ()
     description: str = ""
     rotation: int = 0            # 1: Hadamard-rotated state (INT4+Had)
+    lrb: tuple = ()              # (k, m, eps_L): Low-Rank Bypass
 
     @property
     def seed(self) -> int:
@@ -193,6 +194,13 @@ VARIANTS = {
         (DYNAMIC,), RTN, BF16, BF16, F16, layers=24, rotation=1,
         description="Gated DeltaNet x24 layers, Hadamard-rotated INT4 g32 fp16 dynamic scale "
                     "(INT4+Had), RTN, bf16"),
+    # LRB+BDR with the Gated DeltaNet configuration of Table 6 (k = 1,
+    # m = 15, eps_L = 0.50, eps_B = 0.30) on INT4 g32 binary16 scales
+    "gdn_l24_b256_h32_d128_int4g32_lrb": Workload(
+        "gdn_l24_b256_h32_d128_int4g32_lrb", 6, GDN, 256, 32, 128, 128, 2048, 4, 32,
+        (PERSISTENT,), BDR, BF16, BF16, F16, layers=24, eps_b=0.3, lrb=(1, 15, 0.5),
+        description="Gated DeltaNet x24 layers, INT4 g32 fp16 persistent scale with a Low-Rank "
+                    "Bypass (k=1, m=15, eps_L=0.5) and BDR (eps_B=0.3): LRB+BDR of Table 6"),
 }
 
 

@@ -288,6 +288,11 @@ int qstate_set_taxonomy(qstate* s, int on);
  * QSTATE_EINVAL if already set or for invalid k, m, eps_l. */
 int qstate_set_lrb(qstate* s, int k, int m, float eps_l);
 
+/* Name of the kernel the object's next step launches ("step_kernel",
+ * "rows_kernel" or "lrb_kernel"; "" for NULL): for reports and profiles, no
+ * counterpart on the pages.  The string is static. */
+const char* qstate_kernel(const qstate* s);
+
 /* Copy an LRB object's bypass to caller buffers (device or host):
  * u [tiles][k+m][d_k] and w [tiles][k+m][d_v] binary16 bit patterns,
  * g [tiles][k+m], n [tiles][2] (residual and fresh columns held), D [tiles]. */
