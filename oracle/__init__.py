@@ -107,6 +107,14 @@ def lib():
         _lib.or_lrb_step.argtypes = [ctypes.POINTER(_Cfg), ctypes.POINTER(LrbCfg), ctypes.c_int64,
                                      P, P, P, P, P, P, P, P, P, P, P, P, P, P, P,
                                      ctypes.POINTER(Counts), P, P]
+        _lib.or_e4m3_to_f32.restype = ctypes.c_float
+        _lib.or_e4m3_to_f32.argtypes = [ctypes.c_uint8]
+        _lib.or_f32_to_e4m3.restype = ctypes.c_uint8
+        _lib.or_f32_to_e4m3.argtypes = [ctypes.c_float]
+        _lib.or_pw_step.restype = ctypes.c_int
+        _lib.or_pw_step.argtypes = [ctypes.POINTER(_Cfg), ctypes.c_int, ctypes.c_int64,
+                                    P, P, P, P, P, P, P, P, P, P, P, P, P, P,
+                                    ctypes.POINTER(Counts)]
         _lib.or_rank_k.argtypes = [ctypes.c_int, ctypes.c_int, P, ctypes.c_int, P, P, P]
         _lib.or_lrb_bits.restype = ctypes.c_double
         _lib.or_lrb_bits.argtypes = [ctypes.c_int] * 5 + [ctypes.c_double]
@@ -407,6 +415,64 @@ class LrbState(State):
         u = self.u[t, :n].view(np.float16).astype(np.float64)
         w = self.w[t, :n].view(np.float16).astype(np.float64)
         return np.einsum("l,li,lj->ij", self.g[t, :n].astype(np.float64), u, w)
+
+
+def e4m3_to_f32(b: int) -> float:
+    return float(lib().or_e4m3_to_f32(int(b)))
+
+
+def f32_to_e4m3(x: float) -> int:
+    return int(lib().or_f32_to_e4m3(float(x)))
+
+
+class PwState(State):
+    """A Gated DeltaNet state with a pure-write sliding window of W FP8 pairs
+    (readings W1-W6 of the C code): the history as State (codes and scales,
+    or an fp32 S for 32-bit tiles), plus per tile A [W][d_k] and B [W][d_v]
+    (E4M3 bytes), the slot of the oldest pair and the pairs held."""
+
+    def __init__(self, cfg: Config, tile_bits, W: int):
+        super().__init__(cfg, tile_bits)
+        T = self.ntiles
+        self.W = int(W)
+        self.A = np.zeros((T, W, cfg.d_k), np.uint8)
+        self.B = np.zeros((T, W, cfg.d_v), np.uint8)
+        self.head = np.zeros(T, np.int32)
+        self.count = np.zeros(T, np.int32)
+
+    def step(self, q, k, v, alpha=None, beta=None, threads: int = 1):
+        cfg = self.cfg
+        T = self.ntiles
+        q, k, v = _f32(q).reshape(T, -1), _f32(k).reshape(T, -1), _f32(v).reshape(T, -1)
+        alpha = _f32(alpha).reshape(T, -1)[:, 0].copy()
+        beta = _f32(beta).reshape(T)
+        out = np.zeros((T, cfg.d_v), np.float32)
+        cnt = Counts()
+        rc = lib().or_pw_step(ctypes.byref(cfg.c), self.W, T, _ptr(self.tile_bits),
+                              _ptr(self.codes), _ptr(self.S), _ptr(self.scales), _ptr(self.A),
+                              _ptr(self.B), _ptr(self.head), _ptr(self.count), _ptr(q), _ptr(k),
+                              _ptr(v), _ptr(alpha), _ptr(beta), _ptr(out), ctypes.byref(cnt))
+        if rc != 0:
+            raise ValueError("oracle rejected the PW configuration")
+        self._add_counts(cnt)
+        return out
+
+    def pairs(self, t: int):
+        """(a, b) of tile t's pairs, oldest first, as fp64 [n, d_k], [n, d_v]."""
+        dec = np.vectorize(e4m3_to_f32, otypes=[np.float64])
+        n, h = int(self.count[t]), int(self.head[t])
+        sl = [(h + l) % self.W for l in range(n)]
+        return dec(self.A[t, sl]).reshape(n, -1), dec(self.B[t, sl]).reshape(n, -1)
+
+    def history(self, t: int) -> np.ndarray:
+        if int(self.tile_bits[t]) == 32:
+            return self.S[t].astype(np.float64)
+        return self.dequant()[t].astype(np.float64)
+
+    def state(self, t: int) -> np.ndarray:
+        """History plus the window's pairs (fp64)."""
+        a, b = self.pairs(t)
+        return self.history(t) + a.T @ b
 
 
 def step_many(work, threads: int = 1):

@@ -796,3 +796,178 @@ int or_lrb_step(const or_cfg* c, const or_lrb_cfg* L, int64_t ntiles, const int*
                       resid ? resid + t * (int64_t)dk * dv : NULL);
     return 0;
 }
+
+
+/* ------------------------------------------------------------------------
+ * Pure-write sliding window (PW) of "Low-Bit GDN Recurrent-State
+ * Quantization: Global Gradient-aware Allocation and Pure-Write Sliding
+ * Windows" (Abstract).  The page gives the method in one sentence: the
+ * recent pure writes are kept as FP8 vector pairs, carried through the full
+ * Gated DeltaNet transition, and merged into the low-bit history only once
+ * they leave the window.  Readings:
+ *  W1 the pure write of step t is beta_t k_t v_t^T (the update without its
+ *     erase term); its pair is (fp8(beta_t k_t), fp8(v_t)), beta_t k_t the
+ *     binary32 product;
+ *  W2 FP8 is OCP E4M3 without per-vector scales, encoded to nearest with
+ *     ties to even and saturating at 448;
+ *  W3 the transition A_t = alpha_t (I - beta_t k_t k_t^T) acts on every
+ *     part of the state: the history as the plain Gated DeltaNet step with
+ *     v = 0 (a = alpha (x) S_hat, r = a^T k, x = fma(beta k_i, -r_j, a_ij)),
+ *     and each stored pair on its key side:
+ *     s = canon(a_l . k), t_i = fma(-(beta (x) s), k_i, a_l,i),
+ *     a_l,i <- fp8(alpha (x) t_i), the value side unchanged;
+ *  W4 a window of W pairs: after the transition, when W pairs are held, the
+ *     oldest leaves and is merged into the history, x_ij = fma(a_i, b_j, x_ij);
+ *     then the step's own pair enters (in the slot the leaver freed);
+ *  W5 the output is the whole state's: o = canon(x^T q), then for every pair
+ *     held after the step, oldest first, o_j = fma(canon(a_l . q), b_l,j, o_j);
+ *  W6 the history is requantized every step with the object's scale and
+ *     rounding rules (BDR with d = x - a, a the decayed history).
+ * ---------------------------------------------------------------------- */
+float or_e4m3_to_f32(uint8_t b)
+{
+    int e = (b >> 3) & 15, m = b & 7;
+    if (e == 15 && m == 7) return NAN;
+    float v = e == 0 ? ldexpf((float)m, -9) : ldexpf((float)(8 + m), e - 10);
+    return (b & 0x80) ? -v : v;
+}
+
+uint8_t or_f32_to_e4m3(float x)
+{
+    if (isnan(x)) return 0x7F;
+    uint8_t s = signbit(x) ? 0x80 : 0;
+    double ax = fabs((double)x);
+    int best = 0;
+    double bd = INFINITY;
+    for (int c = 0; c < 127; c++) {      /* the finite non-negative codes, ascending */
+        double d = fabs((double)or_e4m3_to_f32((uint8_t)c) - ax);
+        if (d < bd || (d == bd && !(c & 1))) {
+            bd = d;
+            best = c;
+        }
+    }
+    return (uint8_t)(s | best);
+}
+
+static void pw_tile_step(const or_cfg* c, int W, int bits, int8_t* codes, float* S,
+                         float* scales, uint8_t* A, uint8_t* B, int* head, int* count,
+                         const float* q, const float* k, const float* v, float al, float be,
+                         float* out, or_counts* cnt)
+{
+    const int dk = c->d_k, dv = c->d_v;
+    const size_t n_el = (size_t)dk * dv;
+    const int gs = c->group ? c->group : dv, ng = dv / gs;
+    float* a = (float*)malloc(sizeof(float) * n_el);
+    float* x = (float*)malloc(sizeof(float) * n_el);
+    float al_[512], bl_[512];
+
+    /* W3: the history's transition */
+    for (int i = 0; i < dk; i++)
+        for (int j = 0; j < dv; j++) {
+            size_t e = (size_t)i * dv + j;
+            if (bits == 32) {
+                a[e] = S[e] * al;
+            } else {
+                float delta = c->group ? scales[i * ng + j / gs] : scales[0];
+                a[e] = (float)codes[e] * (al * delta);
+            }
+        }
+    for (int j = 0; j < dv; j++) {
+        float r = or_canon_dot(dk, a + j, dv, k);
+        float e = -r;
+        for (int i = 0; i < dk; i++) {
+            size_t idx = (size_t)i * dv + j;
+            x[idx] = fmaf(be * k[i], e, a[idx]);
+        }
+    }
+    /* W3: the pairs' key sides */
+    int h = *head, n = *count;
+    for (int l = 0; l < n; l++) {
+        uint8_t* Ak = A + (size_t)((h + l) % W) * dk;
+        for (int i = 0; i < dk; i++) al_[i] = or_e4m3_to_f32(Ak[i]);
+        float s = or_canon_dot(dk, al_, 1, k);
+        float cs = be * s;
+        for (int i = 0; i < dk; i++) Ak[i] = or_f32_to_e4m3(al * fmaf(-cs, k[i], al_[i]));
+    }
+    /* W4: the oldest leaves a full window into the history; the new pair */
+    int slot;
+    if (n == W) {
+        uint8_t* Ak = A + (size_t)h * dk;
+        uint8_t* Bv = B + (size_t)h * dv;
+        for (int i = 0; i < dk; i++) al_[i] = or_e4m3_to_f32(Ak[i]);
+        for (int j = 0; j < dv; j++) bl_[j] = or_e4m3_to_f32(Bv[j]);
+        for (int i = 0; i < dk; i++)
+            for (int j = 0; j < dv; j++) {
+                size_t idx = (size_t)i * dv + j;
+                x[idx] = fmaf(al_[i], bl_[j], x[idx]);
+            }
+        slot = h;
+        h = (h + 1) % W;
+    } else {
+        slot = (h + n) % W;
+        n++;
+    }
+    for (int i = 0; i < dk; i++) A[(size_t)slot * dk + i] = or_f32_to_e4m3(be * k[i]);
+    for (int j = 0; j < dv; j++) B[(size_t)slot * dv + j] = or_f32_to_e4m3(v[j]);
+    *head = h;
+    *count = n;
+
+    /* W5: the output of the whole state */
+    for (int j = 0; j < dv; j++) out[j] = or_canon_dot(dk, x + j, dv, q);
+    for (int l = 0; l < n; l++) {
+        int sl = (h + l) % W;
+        for (int i = 0; i < dk; i++) al_[i] = or_e4m3_to_f32(A[(size_t)sl * dk + i]);
+        float cq = or_canon_dot(dk, al_, 1, q);
+        for (int j = 0; j < dv; j++) out[j] = fmaf(cq, or_e4m3_to_f32(B[(size_t)sl * dv + j]), out[j]);
+    }
+
+    /* W6: requantize the history */
+    if (bits == 32) {
+        memcpy(S, x, sizeof(float) * n_el);
+    } else {
+        const int qmax = (1 << (bits - 1)) - 1;
+        const float fq = (float)qmax;
+        for (int g = 0; g < or_n_scales(c); g++) {
+            int i0 = c->group ? g / ng : 0, i1 = c->group ? i0 + 1 : dk;
+            int j0 = c->group ? (g % ng) * gs : 0, j1 = c->group ? j0 + gs : dv;
+            float m = 0.0f;
+            for (int i = i0; i < i1; i++)
+                for (int j = j0; j < j1; j++) m = fmaxf(m, fabsf(x[(size_t)i * dv + j]));
+            float delta;
+            if (c->scale_mode == OR_DYNAMIC) {
+                delta = to_stored_scale(c, m / fq, cnt);
+            } else {
+                float dp = scales[g];
+                delta = (m > fq * dp) ? to_stored_scale(c, m / fq, cnt) : dp;
+            }
+            scales[g] = delta;
+            float inv = delta == 0.0f ? 0.0f : 1.0f / delta;
+            for (int i = i0; i < i1; i++)
+                for (int j = j0; j < j1; j++) {
+                    size_t e = (size_t)i * dv + j;
+                    codes[e] = (int8_t)or_round(c, a[e], x[e], inv, qmax, cnt);
+                }
+        }
+    }
+    free(a);
+    free(x);
+}
+
+int or_pw_step(const or_cfg* c, int W, int64_t ntiles, const int* tile_bits,
+               int8_t* codes, float* S, float* scales, uint8_t* A, uint8_t* B, int* head,
+               int* count, const float* q, const float* k, const float* v,
+               const float* alpha, const float* beta, float* out, or_counts* cnt)
+{
+    if (!valid_cfg(c) || c->kind != OR_GDN || c->scale_mode == OR_YOKED || c->rotate) return -1;
+    if (W < 1 || W > OR_PW_MAX_W || c->d_k > 512 || c->d_v > 512) return -1;
+    const int dk = c->d_k, dv = c->d_v, nsc = or_n_scales(c);
+    for (int64_t t = 0; t < ntiles; t++) {
+        int b = tile_bits[t];
+        if (!(b == 32 || (b >= 2 && b <= 8 && b % 2 == 0))) return -1;
+    }
+    for (int64_t t = 0; t < ntiles; t++)
+        pw_tile_step(c, W, tile_bits[t], codes + t * dk * dv, S + t * dk * dv, scales + t * nsc,
+                     A + t * (int64_t)W * dk, B + t * (int64_t)W * dv, head + t, count + t,
+                     q + t * dk, k + t * dk, v + t * dv, alpha[t], beta[t], out + t * dv, cnt);
+    return 0;
+}

@@ -149,6 +149,25 @@ void or_rank_k(int rows, int cols, const double* R, int k, double* s, double* U,
  * bypass columns of (d_k + d_v) 16-bit values and a 32-bit coefficient. */
 double or_lrb_bits(int bits, int group, int scale_bits, int d_k, int d_v, double cols_used);
 
+/* ---- Pure-write sliding window (PW): readings W1-W6 in qstate_oracle.c -- */
+#define OR_PW_MAX_W 16
+
+/* OCP FP8 E4M3 ("E4M3FN"): 1 sign, 4 exponent bits (bias 7), 3 fraction bits,
+ * no infinities, 0x7F / 0xFF NaN, largest finite 448.  Encoding: nearest,
+ * ties to the even code; magnitudes beyond 448 give 448 (saturating). */
+float or_e4m3_to_f32(uint8_t b);
+uint8_t or_f32_to_e4m3(float x);
+
+/* One PW step of ntiles Gated DeltaNet tiles (history widths 2..8 quantized,
+ * or 32 = an fp32 history; dynamic or persistent scales).  Window per tile:
+ * A [W][d_k] and B [W][d_v] FP8 E4M3 bytes (key and value sides of the
+ * pairs), head the slot of the oldest pair, count the pairs held.  W in
+ * 1 .. OR_PW_MAX_W.  -1 if invalid. */
+int or_pw_step(const or_cfg* c, int W, int64_t ntiles, const int* tile_bits,
+               int8_t* codes, float* S, float* scales, uint8_t* A, uint8_t* B, int* head,
+               int* count, const float* q, const float* k, const float* v,
+               const float* alpha, const float* beta, float* out, or_counts* cnt);
+
 #ifdef __cplusplus
 }
 #endif
