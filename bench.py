@@ -163,6 +163,8 @@ def cpu_oracle_rate(wl, seconds=10.0, threads=None, max_steps=None, tiles=None, 
     from bit_recurrent_state_decode_b200 import synth
     threads = threads or os.cpu_count() or 1
     cycle = 1
+    if wl.pw:
+        tiles = tiles or 32
     if wl.lrb:
         # whole merge cycles (m steps, one of them a merge), after one cycle
         # that fills the residual; the bypass step is single-threaded
@@ -183,6 +185,10 @@ def cpu_oracle_rate(wl, seconds=10.0, threads=None, max_steps=None, tiles=None, 
         if wl.lrb:
             # the oracle's bypass step runs its tiles on one host thread
             states.append(oracle.LrbState(cfg, tile_bits, *wl.lrb))
+            threads = 1
+        elif wl.pw:
+            # so does its windowed step
+            states.append(oracle.PwState(cfg, tile_bits, wl.pw))
             threads = 1
         else:
             states.append(oracle.State(cfg, tile_bits))
@@ -241,6 +247,8 @@ def run_ours(args, rank, world, local_rank):
                      scale_dtype=wl0.scale_dtype, head_bits=hb, rotation=wl0.rotation)
         if wl0.lrb:
             o.set_lrb(*wl0.lrb)
+        if wl0.pw:
+            o.set_pw(wl0.pw)
         return o
 
     probe = make(wl0.scale_modes[0], 1)

@@ -13,6 +13,7 @@
 #include "qstate.h"
 #include "qstate_dispatch.h"
 #include "qstate_lrb.cuh"
+#include "qstate_pw.cuh"
 
 namespace qs {
 void launch_dequant_64_64(const StepParams&, float*, cudaStream_t);
@@ -76,6 +77,16 @@ struct qstate {
     float* d_lD = nullptr;
     const qs::LrbEntry* lrb_entry = nullptr;
     int lrb_grid = 1, lrb_smem = 0;
+    // pure-write sliding window (qstate_set_pw): the pairs, the slot of the
+    // oldest pair and the pairs held, per tile
+    bool pw = false;
+    int pw_W = 0;
+    uint8_t* d_pa = nullptr;
+    uint8_t* d_pb = nullptr;
+    int* d_phead = nullptr;
+    int* d_pcount = nullptr;
+    const qs::PwEntry* pw_entry = nullptr;
+    int pw_grid = 1;
     // set by qstate_import: the next step takes the general tile bodies (an
     // imported state may hold the code -2^(bits-1), which no step produces)
     bool import_pending = false;
@@ -160,6 +171,22 @@ void free_all(qstate* s) {
     cudaFree(s->d_lg);
     cudaFree(s->d_ln);
     cudaFree(s->d_lD);
+    cudaFree(s->d_pa);
+    cudaFree(s->d_pb);
+    cudaFree(s->d_phead);
+    cudaFree(s->d_pcount);
+}
+
+// an empty window
+int zero_window(qstate* s, cudaStream_t st) {
+    if (!s->pw || s->tiles == 0) return QSTATE_OK;
+    const int64_t T = s->tiles, W = s->pw_W;
+    if (cudaMemsetAsync(s->d_pa, 0, T * W * s->L.d_k, st) != cudaSuccess ||
+        cudaMemsetAsync(s->d_pb, 0, T * W * s->L.d_v, st) != cudaSuccess ||
+        cudaMemsetAsync(s->d_phead, 0, T * 4, st) != cudaSuccess ||
+        cudaMemsetAsync(s->d_pcount, 0, T * 4, st) != cudaSuccess)
+        return QSTATE_ECUDA;
+    return QSTATE_OK;
 }
 
 // bypass empty, D = 1 for every tile
@@ -409,6 +436,7 @@ int qstate_reset(qstate* s, qstate_stream stream) {
     if (!s) return QSTATE_EINVAL;
     int rc = zero_state(s, (cudaStream_t)stream);
     if (rc == QSTATE_OK) rc = zero_bypass(s, (cudaStream_t)stream);
+    if (rc == QSTATE_OK) rc = zero_window(s, (cudaStream_t)stream);
     return rc;
 }
 
@@ -428,6 +456,11 @@ int qstate_step(qstate* s, const void* q, const void* k, const void* v, const vo
     p.v = v;
     p.gates = gates;
     p.out = out;
+    if (s->pw) {
+        qs::PwParams Pp{s->d_pa, s->d_pb, s->d_phead, s->d_pcount, s->pw_W};
+        s->pw_entry->launch(p, Pp, s->pw_grid, 0, (cudaStream_t)stream);
+        return cudaGetLastError() == cudaSuccess ? QSTATE_OK : QSTATE_ECUDA;
+    }
     if (s->lrb) {
         qs::LrbParams Lp{s->d_lu, s->d_lw, s->d_lg, s->d_ln, s->d_lD, s->lrb_k, s->lrb_m, s->lrb_eps};
         s->lrb_entry->launch(p, Lp, s->lrb_grid, s->lrb_smem, (cudaStream_t)stream);
@@ -533,13 +566,22 @@ int qstate_import(qstate* s, const void* codes, const void* scales, const float*
         cudaMemcpyAsync(s->d_ref, ref, s->ref_bytes, cudaMemcpyDefault, st) != cudaSuccess)
         return QSTATE_ECUDA;
     s->import_pending = true;
-    return zero_bypass(s, st);
+    int rc = zero_bypass(s, st);
+    if (rc == QSTATE_OK) rc = zero_window(s, st);
+    return rc;
 }
 
 int64_t qstate_bytes_per_step(const qstate* s) {
     if (!s) return -1;
     const int64_t dk = s->L.d_k, dv = s->L.d_v;
     const int64_t ops = s->tiles * ((2 * dk + dv) * s->in_size + s->n_gate * s->gate_size + dv * 4);
+    if (s->pw) {
+        // state and scales read and written; every pair read, every key side
+        // and the new value side written
+        const int64_t W = s->pw_W;
+        return 2 * s->code_bytes + 2 * s->scale_bytes + ops +
+               s->tiles * (W * (dk + dv) + W * dk + dv + 16);
+    }
     if (s->lrb) {
         // averaged over a merge cycle of m steps: the state is read every step
         // and written at the merge; the columns held at the start of a step
@@ -555,8 +597,59 @@ int64_t qstate_bytes_per_step(const qstate* s) {
     return b + ops;
 }
 
+int qstate_set_pw(qstate* s, int W) {
+    if (!s || s->pw || s->lrb) return QSTATE_EINVAL;
+    if (W < 1 || W > qs::kPwMaxW) return QSTATE_EINVAL;
+    if (s->L.kind != QSTATE_GDN || s->scale_mode == QSTATE_YOKED || s->L.rotation ||
+        !s->head_bits.empty() || !(s->bits == 4 || s->bits == 8) || s->L.d_k != s->L.d_v)
+        return QSTATE_EUNSUPPORTED;
+    int rc = check_device(s);
+    if (rc != QSTATE_OK) return rc;
+    const int d = s->L.d_k;
+    const int idx = (((d == 128) * 2 + (s->bits == 8)) * 2 + (s->round_mode == QSTATE_BDR)) * 2 +
+                    (s->L.qkv_dtype == QSTATE_BF16);
+    const qs::PwEntry* e = &qs::pw_table()[idx];
+    const int per_sm = e->blocks_per_sm(0);
+    if (per_sm < 1) { cudaGetLastError(); return QSTATE_EUNSUPPORTED; }
+    const int64_t T = s->tiles;
+    auto alloc = [&](void** p, size_t n) -> bool { return !n || cudaMalloc(p, n) == cudaSuccess; };
+    if (!alloc((void**)&s->d_pa, T * W * d) || !alloc((void**)&s->d_pb, T * W * d) ||
+        !alloc((void**)&s->d_phead, T * 4) || !alloc((void**)&s->d_pcount, T * 4)) {
+        cudaGetLastError();
+        cudaFree(s->d_pa); cudaFree(s->d_pb); cudaFree(s->d_phead); cudaFree(s->d_pcount);
+        s->d_pa = s->d_pb = nullptr;
+        s->d_phead = s->d_pcount = nullptr;
+        return QSTATE_ENOMEM;
+    }
+    s->pw = true;
+    s->pw_W = W;
+    s->pw_entry = e;
+    int sms = 0;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, s->device);
+    int64_t g = (int64_t)sms * per_sm;
+    if (T < g) g = T > 0 ? T : 1;
+    s->pw_grid = (int)g;
+    rc = zero_window(s, nullptr);
+    if (rc == QSTATE_OK && cudaDeviceSynchronize() != cudaSuccess) rc = QSTATE_ECUDA;
+    return rc;
+}
+
+int qstate_pw_export(const qstate* s, uint8_t* A, uint8_t* B, int32_t* head, int32_t* count,
+                     qstate_stream stream) {
+    if (!s || !s->pw || !A || !B || !head || !count) return QSTATE_EINVAL;
+    if (s->tiles == 0) return QSTATE_OK;
+    const int64_t T = s->tiles, W = s->pw_W;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (cudaMemcpyAsync(A, s->d_pa, T * W * s->L.d_k, cudaMemcpyDefault, st) != cudaSuccess ||
+        cudaMemcpyAsync(B, s->d_pb, T * W * s->L.d_v, cudaMemcpyDefault, st) != cudaSuccess ||
+        cudaMemcpyAsync(head, s->d_phead, T * 4, cudaMemcpyDefault, st) != cudaSuccess ||
+        cudaMemcpyAsync(count, s->d_pcount, T * 4, cudaMemcpyDefault, st) != cudaSuccess)
+        return QSTATE_ECUDA;
+    return QSTATE_OK;
+}
+
 int qstate_set_lrb(qstate* s, int k, int m, float eps_l) {
-    if (!s || s->lrb) return QSTATE_EINVAL;
+    if (!s || s->lrb || s->pw) return QSTATE_EINVAL;
     if (k < 0 || k > 1 || m < 1 || k + m > qs::kLrbMaxCols) return QSTATE_EINVAL;
     if (!(eps_l >= 0.0f) || !std::isfinite(eps_l)) return QSTATE_EINVAL;
     if (s->L.kind == QSTATE_GLA || s->scale_mode == QSTATE_YOKED || s->L.rotation ||
@@ -602,6 +695,7 @@ int qstate_set_lrb(qstate* s, int k, int m, float eps_l) {
 const char* qstate_kernel(const qstate* s) {
     if (!s) return "";
     if (s->lrb) return "lrb_kernel";
+    if (s->pw) return "pw_kernel";
     if (s->taxonomy || s->L.rotation) return "step_kernel";
     return s->entry_name;
 }

@@ -45,6 +45,17 @@ struct LrbEntry {
 };
 const LrbEntry* lrb_table();
 
+// The Gated DeltaNet decode step with a pure-write sliding window (d_k = d_v
+// in {64, 128}, 4- or 8-bit codes): 16 entries indexed by
+// (((d == 128) * 2 + (bits == 8)) * 2 + bdr) * 2 + bf16.
+struct PwParams;
+struct PwEntry {
+    void (*launch)(const StepParams&, const PwParams&, int grid, int dyn_smem, cudaStream_t);
+    int (*blocks_per_sm)(int dyn_smem);
+    int threads;
+};
+const PwEntry* pw_table();
+
 // 0 = per-head widths, then 2, 4, 6, 8, 32 bits; -1 if invalid
 inline int bits_index(int bits) {
     switch (bits) {

@@ -29,7 +29,7 @@
 namespace qs {
 
 constexpr int kLrbMaxCols = 32;
-constexpr int kLrbPowerIters = 24;
+constexpr int kLrbPowerIters = 16;
 
 struct LrbParams {
     uint16_t* u;      // [tiles][k + m][d_k] binary16
@@ -47,7 +47,8 @@ __device__ __forceinline__ float f16r(float x) { return __half2float(__float2hal
 
 // Canonical sum over i < DK of x_i y_i (blocks of 8 rows, ascending fma from
 // +0, then the adjacent-pairs tree), by one warp: lane b < DK/8 sums block b,
-// the xor butterfly over those lanes is the tree.  Every lane gets the sum.
+// the xor butterfly over those lanes is the tree, and lane 0's total goes to
+// every lane (the lanes above DK/8 hold only their own zeros).
 template <int DK, class X, class Y>
 __device__ __forceinline__ float warp_canon_dot(X x, Y y, int lane) {
     constexpr int NB = DK / 8;
@@ -58,7 +59,7 @@ __device__ __forceinline__ float warp_canon_dot(X x, Y y, int lane) {
     }
 #pragma unroll
     for (int off = 1; off < NB; off <<= 1) p = __fadd_rn(p, __shfl_xor_sync(0xFFFFFFFFu, p, off));
-    return p;
+    return __shfl_sync(0xFFFFFFFFu, p, 0);
 }
 
 template <int DK, int DV>
@@ -74,7 +75,18 @@ struct __align__(16) LrbShared {
     float unew[DK], wnew[DV];        // the new column (binary16 values)
     // the tile's scales before the step, in their stored format
     __align__(16) uint8_t sprev[DK * (DV / 8) * 4];
+    // the columns held at the start of the step (binary16 patterns)
+    __align__(16) uint16_t ucol[kLrbMaxCols * DK];
+    __align__(16) uint16_t wcol[kLrbMaxCols * DV];
 };
+
+// Ask L2 for [p, p + bytes) (128-byte lines, spread over the CTA's threads)
+template <int NT>
+__device__ __forceinline__ void prefetch_l2(const void* p, long long bytes) {
+    const char* c = static_cast<const char*>(p);
+    for (long long o = (long long)threadIdx.x * 128; o < bytes; o += (long long)NT * 128)
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(c + o));
+}
 
 // Round x with the scale's reciprocal: code = clamp(RTN(x * inv)); with BDR
 // a reversed element (d = x - a, s = fma(a, inv, -code), d > 0 and s > eps_B,
@@ -111,6 +123,93 @@ __device__ __forceinline__ void colsum_any(float (&p)[8], float* red, float* tot
     colsum_finish<DK, DV>(p, red, tot, warp, rbl, j0, res);
 }
 
+// Requantize a tile's updated state x (a: the decayed state before the
+// update, for BDR) with the object's scale rule (dynamic or persistent,
+// per-group or per-token; previous scales in `sprev`, in their stored
+// format): new scales and codes written to HBM, saturated scales and
+// non-finite group maxima counted.  Every thread of the CTA calls it.
+template <int DK, int DV, int BITS, bool BDR, class XS>
+__device__ __forceinline__ void requantize(const StepParams& p, XS& xs, const uint8_t* sprev,
+                                           long long sbase, uint8_t* ct, const float (&a)[8][8],
+                                           const float (&x)[8][8], int lane, int warp, int cb,
+                                           int i0, int ng, int gcol) {
+    using G = Geo<DK, DV>;
+    constexpr int QMAX = (1 << (BITS - 1)) - 1;
+    constexpr float fq = float(QMAX);
+    constexpr float rq = QMAX == 7 ? 0x1.24924ap-3f : 0x1.020408p-7f;
+    const bool sf32 = p.scale_f32 != 0;
+    const int group = p.group;
+    auto prev_scale = [&](int idx) -> float {
+        if (sf32) return reinterpret_cast<const float*>(sprev)[idx];
+        return __half2float(reinterpret_cast<const __half*>(sprev)[idx]);
+    };
+    // group maxima of |x| and the new scales
+    float m[8];
+#pragma unroll
+    for (int r = 0; r < 8; r++) {
+        float mx = 0.0f;
+#pragma unroll
+        for (int c = 0; c < 8; c++) mx = fmaxf(mx, fabsf(x[r][c]));
+        m[r] = mx;
+    }
+    if (group) {
+        float4* r4 = reinterpret_cast<float4*>(&xs.rmax[cb][i0]);
+        r4[0] = make_float4(m[0], m[1], m[2], m[3]);
+        r4[1] = make_float4(m[4], m[5], m[6], m[7]);
+    } else {
+        float t = m[0];
+#pragma unroll
+        for (int r = 1; r < 8; r++) t = fmaxf(t, m[r]);
+        t = __uint_as_float(__reduce_max_sync(0xFFFFFFFFu, __float_as_uint(t)));
+        if (lane == 0) xs.wred[0][warp] = t;
+    }
+    __syncthreads();
+    float inv[8];
+    unsigned nsat = 0;
+    bool bad = false;
+    auto new_scale = [&](float mm, float, float dp, bool& sat, auto sfc) -> float {
+        const bool F = as_bool(sfc);
+        sat = false;
+        if (p.scale_mode == M_PERSISTENT)
+            return (mm > __fmul_rn(fq, dp)) ? to_stored(div_by_qmax(mm, fq, rq), F, sat) : dp;
+        return to_stored(div_by_qmax(mm, fq, rq), F, sat);
+    };
+    if (group) {
+        auto gs = [&](auto lc, auto sfc) {
+            group_scales<DK, DV, decltype(lc)::value, decltype(sfc)::value>(
+                cb, lane, i0, xs, false, inv, nsat, bad, new_scale, sprev, p, sbase, ng, gcol);
+        };
+        auto gs_l = [&](auto lc) {
+            if (sf32) gs(lc, std::true_type{});
+            else gs(lc, std::false_type{});
+        };
+        switch (group / 8) {
+            case 1: gs_l(std::integral_constant<int, 1>{}); break;
+            case 2: gs_l(std::integral_constant<int, 2>{}); break;
+            case 4: gs_l(std::integral_constant<int, 4>{}); break;
+            case 8: gs_l(std::integral_constant<int, 8>{}); break;
+            default: gs_l(std::integral_constant<int, 16>{}); break;
+        }
+    } else {
+        float tmax = xs.wred[0][0];
+#pragma unroll
+        for (int w2 = 1; w2 < G::NWARPS; w2++) tmax = fmaxf(tmax, xs.wred[0][w2]);
+        bool sat;
+        const float d = new_scale(tmax, 0.0f, prev_scale(0), sat, sf32);
+        const float iv = d == 0.0f ? 0.0f : __frcp_rn(d);
+#pragma unroll
+        for (int r = 0; r < 8; r++) inv[r] = iv;
+        bad |= !isfinite(tmax);
+        if (threadIdx.x == G::NT - 1) {
+            store_scale(p.scales, sbase, sf32, d);
+            nsat += sat ? 1u : 0u;
+        }
+    }
+    if (nsat) atomicAdd(p.counters + 1, (unsigned long long)nsat);
+    if (bad && threadIdx.x == 0) atomicAdd(p.counters, 1ull);
+    round_pack_ax<DK, DV, BITS, BDR>(a, x, inv, p.eps_b, ct, i0, cb);
+}
+
 template <int DK, int DV, int BITS, bool GDN, bool BDR, bool BF>
 __global__ void __launch_bounds__(Geo<DK, DV>::NT, 1) lrb_kernel(const StepParams p, const LrbParams L) {
     using G = Geo<DK, DV>;
@@ -142,11 +241,41 @@ __global__ void __launch_bounds__(Geo<DK, DV>::NT, 1) lrb_kernel(const StepParam
         const float beta = GDN ? ldg1(p.gates, tile * p.n_gate + 1, p.gate_bf16 != 0) : 0.0f;
         const float Dn = __fmul_rn(alpha, L.D[tile]);
 
-        // the tile's scales before the step, and the decayed coefficients
+        // the next tile's bytes on their way to L2 while this one is stepped
+        {
+            const long long nt = tile + gridDim.x;
+            if (nt < p.ntiles) {
+                const int ssz = sf32 ? 4 : 2;
+                const int isz = BF ? 2 : 4;
+                prefetch_l2<G::NT>(p.codes + nt * p.tile_bytes, p.tile_bytes);
+                prefetch_l2<G::NT>(static_cast<const uint8_t*>(p.scales) + nt * p.n_scales * ssz,
+                                   (long long)p.n_scales * ssz);
+                prefetch_l2<G::NT>(L.u + nt * K * DK, (long long)K * DK * 2);
+                prefetch_l2<G::NT>(L.w + nt * K * DV, (long long)K * DV * 2);
+                if (threadIdx.x == 0) {
+                    asm volatile("prefetch.global.L2 [%0];" ::"l"(static_cast<const uint8_t*>(p.q) + nt * DK * isz));
+                    asm volatile("prefetch.global.L2 [%0];" ::"l"(static_cast<const uint8_t*>(p.k) + nt * DK * isz));
+                    asm volatile("prefetch.global.L2 [%0];" ::"l"(static_cast<const uint8_t*>(p.v) + nt * DV * isz));
+                }
+            }
+        }
+        // the tile's scales before the step, its columns, and the decayed
+        // coefficients (16-byte loads: every region starts on a 16-byte
+        // boundary and holds a multiple of 16 bytes, or is copied bytewise)
         {
             const int ssz = sf32 ? 4 : 2;
             const uint8_t* src = static_cast<const uint8_t*>(p.scales) + sbase * ssz;
-            for (int i = threadIdx.x; i < p.n_scales * ssz; i += G::NT) sh.sprev[i] = src[i];
+            const int sb = p.n_scales * ssz;
+            if ((sb & 15) == 0 && ((sbase * ssz) & 15) == 0) {
+                for (int i = threadIdx.x; i < sb / 16; i += G::NT)
+                    reinterpret_cast<uint4*>(sh.sprev)[i] = reinterpret_cast<const uint4*>(src)[i];
+            } else {
+                for (int i = threadIdx.x; i < sb; i += G::NT) sh.sprev[i] = src[i];
+            }
+            for (int i = threadIdx.x; i < n * DK / 8; i += G::NT)
+                reinterpret_cast<uint4*>(sh.ucol)[i] = reinterpret_cast<const uint4*>(U)[i];
+            for (int i = threadIdx.x; i < n * DV / 8; i += G::NT)
+                reinterpret_cast<uint4*>(sh.wcol)[i] = reinterpret_cast<const uint4*>(Wc)[i];
         }
         auto prev_scale = [&](int idx) -> float {
             if (sf32) return reinterpret_cast<const float*>(sh.sprev)[idx];
@@ -160,7 +289,7 @@ __global__ void __launch_bounds__(Geo<DK, DV>::NT, 1) lrb_kernel(const StepParam
         auto kval = [&](int i) { return ldg1(kin, i, BF); };
         auto qval = [&](int i) { return ldg1(qin, i, BF); };
         for (int l = warp; l < n; l += G::NWARPS) {
-            auto uval = [&](int i) { return h2f(U[l * DK + i]); };
+            auto uval = [&](int i) { return h2f(sh.ucol[l * DK + i]); };
             const float dk_ = warp_canon_dot<DK>(uval, kval, lane);
             const float dq_ = warp_canon_dot<DK>(uval, qval, lane);
             if (lane == 0) {
@@ -208,7 +337,7 @@ __global__ void __launch_bounds__(Geo<DK, DV>::NT, 1) lrb_kernel(const StepParam
             colsum_finish<DK, DV>(pr, sh.red, sh.tot, warp, rbl, j0, rr);
             for (int l = 0; l < n; l++) {
 #pragma unroll
-                for (int c = 0; c < 8; c++) rr[c] = __fmaf_rn(sh.ck[l], h2f(Wc[l * DV + j0 + c]), rr[c]);
+                for (int c = 0; c < 8; c++) rr[c] = __fmaf_rn(sh.ck[l], h2f(sh.wcol[l * DV + j0 + c]), rr[c]);
             }
 #pragma unroll
             for (int c = 0; c < 8; c++) wn[c] = f16r(__fsub_rn(vv[c], rr[c]));
@@ -247,7 +376,7 @@ __global__ void __launch_bounds__(Geo<DK, DV>::NT, 1) lrb_kernel(const StepParam
             colsum_finish<DK, DV>(po, sh.red, sh.tot, warp, rbl, j0, oo);    // syncs: cq[n] visible
             for (int l = 0; l < n; l++) {
 #pragma unroll
-                for (int c = 0; c < 8; c++) oo[c] = __fmaf_rn(sh.cq[l], h2f(Wc[l * DV + j0 + c]), oo[c]);
+                for (int c = 0; c < 8; c++) oo[c] = __fmaf_rn(sh.cq[l], h2f(sh.wcol[l * DV + j0 + c]), oo[c]);
             }
 #pragma unroll
             for (int c = 0; c < 8; c++) oo[c] = __fmaf_rn(sh.cq[n], sh.wnew[j0 + c], oo[c]);
@@ -283,11 +412,11 @@ __global__ void __launch_bounds__(Geo<DK, DV>::NT, 1) lrb_kernel(const StepParam
                 const float gl = sh.gco[l];
 #pragma unroll
                 for (int r = 0; r < 8; r++) {
-                    const float ul = l < n ? h2f(U[l * DK + i0 + r]) : sh.unew[i0 + r];
+                    const float ul = l < n ? h2f(sh.ucol[l * DK + i0 + r]) : sh.unew[i0 + r];
                     const float gu = __fmul_rn(gl, ul);
 #pragma unroll
                     for (int c = 0; c < 8; c++) {
-                        const float wl = l < n ? h2f(Wc[l * DV + j0 + c]) : sh.wnew[j0 + c];
+                        const float wl = l < n ? h2f(sh.wcol[l * DV + j0 + c]) : sh.wnew[j0 + c];
                         P[r][c] = __fmaf_rn(gu, wl, P[r][c]);
                     }
                 }
@@ -303,72 +432,8 @@ __global__ void __launch_bounds__(Geo<DK, DV>::NT, 1) lrb_kernel(const StepParam
                 }
             }
         }
-        // group maxima of |x| and the new scales
-        float m[8];
-#pragma unroll
-        for (int r = 0; r < 8; r++) {
-            float mx = 0.0f;
-#pragma unroll
-            for (int c = 0; c < 8; c++) mx = fmaxf(mx, fabsf(x[r][c]));
-            m[r] = mx;
-        }
-        auto& xs = sh.xs;
-        if (group) {
-            float4* r4 = reinterpret_cast<float4*>(&xs.rmax[cb][i0]);
-            r4[0] = make_float4(m[0], m[1], m[2], m[3]);
-            r4[1] = make_float4(m[4], m[5], m[6], m[7]);
-        } else {
-            float t = m[0];
-#pragma unroll
-            for (int r = 1; r < 8; r++) t = fmaxf(t, m[r]);
-            t = __uint_as_float(__reduce_max_sync(0xFFFFFFFFu, __float_as_uint(t)));
-            if (lane == 0) xs.wred[0][warp] = t;
-        }
-        __syncthreads();
-        float inv[8];
-        unsigned nsat = 0;
-        bool bad = false;
-        auto new_scale = [&](float mm, float, float dp, bool& sat, auto sfc) -> float {
-            const bool F = as_bool(sfc);
-            sat = false;
-            if (p.scale_mode == M_PERSISTENT)
-                return (mm > __fmul_rn(fq, dp)) ? to_stored(div_by_qmax(mm, fq, rq), F, sat) : dp;
-            return to_stored(div_by_qmax(mm, fq, rq), F, sat);
-        };
-        if (group) {
-            auto gs = [&](auto lc, auto sfc) {
-                group_scales<DK, DV, decltype(lc)::value, decltype(sfc)::value>(
-                    cb, lane, i0, xs, false, inv, nsat, bad, new_scale, sh.sprev, p, sbase, ng, gcol);
-            };
-            auto gs_l = [&](auto lc) {
-                if (sf32) gs(lc, std::true_type{});
-                else gs(lc, std::false_type{});
-            };
-            switch (group / 8) {
-                case 1: gs_l(std::integral_constant<int, 1>{}); break;
-                case 2: gs_l(std::integral_constant<int, 2>{}); break;
-                case 4: gs_l(std::integral_constant<int, 4>{}); break;
-                case 8: gs_l(std::integral_constant<int, 8>{}); break;
-                default: gs_l(std::integral_constant<int, 16>{}); break;
-            }
-        } else {
-            float tmax = xs.wred[0][0];
-#pragma unroll
-            for (int w2 = 1; w2 < G::NWARPS; w2++) tmax = fmaxf(tmax, xs.wred[0][w2]);
-            bool sat;
-            const float d = new_scale(tmax, 0.0f, prev_scale(0), sat, sf32);
-            const float iv = d == 0.0f ? 0.0f : __frcp_rn(d);
-#pragma unroll
-            for (int r = 0; r < 8; r++) inv[r] = iv;
-            bad |= !isfinite(tmax);
-            if (threadIdx.x == G::NT - 1) {
-                store_scale(p.scales, sbase, sf32, d);
-                nsat += sat ? 1u : 0u;
-            }
-        }
-        if (nsat) atomicAdd(p.counters + 1, (unsigned long long)nsat);
-        if (bad && threadIdx.x == 0) atomicAdd(p.counters, 1ull);
-        round_pack_ax<DK, DV, BITS, BDR>(a, x, inv, p.eps_b, ct, i0, cb);
+        requantize<DK, DV, BITS, BDR>(p, sh.xs, sh.sprev, sbase, ct, a, x, lane, warp, cb, i0, ng,
+                                      gcol);
 
         // the unmerged rest: its leading singular pair (k = 1) or nothing
         if (L.k == 1) {
@@ -379,7 +444,7 @@ __global__ void __launch_bounds__(Geo<DK, DV>::NT, 1) lrb_kernel(const StepParam
             // rows sum to zero, as all ones would be)
             bool nz = false;
             for (int j = threadIdx.x; j < DV; j += G::NT) {
-                const float v0 = nres > 0 ? h2f(Wc[j]) : 0.0f;
+                const float v0 = nres > 0 ? h2f(sh.wcol[j]) : 0.0f;
                 sh.vec[j] = v0;
                 nz |= v0 != 0.0f;
             }
@@ -388,9 +453,9 @@ __global__ void __launch_bounds__(Geo<DK, DV>::NT, 1) lrb_kernel(const StepParam
             }
             __syncthreads();
             float y[8], vj[8];
-            for (int itp = 0; itp <= kLrbPowerIters; itp++) {
 #pragma unroll
-                for (int c = 0; c < 8; c++) vj[c] = sh.vec[j0 + c];
+            for (int c = 0; c < 8; c++) vj[c] = sh.vec[j0 + c];
+            for (int itp = 0; itp <= kLrbPowerIters; itp++) {
                 // y = R v over this thread's rows, joined across its row's lanes
 #pragma unroll
                 for (int r = 0; r < 8; r++) {
@@ -401,7 +466,8 @@ __global__ void __launch_bounds__(Geo<DK, DV>::NT, 1) lrb_kernel(const StepParam
                     y[r] = t;
                 }
                 if (itp == kLrbPowerIters) break;
-                // z = R^T y, normalised
+                // v = R^T y / |R^T y|: every warp forms the norm from the column
+                // totals itself (same values, same order), so v stays in registers
                 float z[8], zt[8];
 #pragma unroll
                 for (int c = 0; c < 8; c++) {
@@ -412,20 +478,16 @@ __global__ void __launch_bounds__(Geo<DK, DV>::NT, 1) lrb_kernel(const StepParam
                 }
                 colsum_any<DK, DV>(z, sh.red, sh.tot, warp, rbl, j0, zt);
                 float s2 = 0.0f;
-                if (threadIdx.x < 32) {
-                    for (int j = lane; j < DV; j += 32) s2 = __fmaf_rn(sh.tot[j], sh.tot[j], s2);
+                for (int j = lane; j < DV; j += 32) s2 = __fmaf_rn(sh.tot[j], sh.tot[j], s2);
 #pragma unroll
-                    for (int off = 16; off >= 1; off >>= 1) s2 += __shfl_xor_sync(0xFFFFFFFFu, s2, off);
-                    if (lane == 0) sh.nrm[0] = s2;
-                }
-                __syncthreads();
-                const float nz = sqrtf(sh.nrm[0]);
-                const float iz = nz > 0.0f ? 1.0f / nz : 0.0f;
-                if (rbl == 0 && warp == 0) {
+                for (int off = 16; off >= 1; off >>= 1) s2 += __shfl_xor_sync(0xFFFFFFFFu, s2, off);
+                const float iz = s2 > 0.0f ? rsqrtf(s2) : 0.0f;
 #pragma unroll
-                    for (int c = 0; c < 8; c++) sh.vec[j0 + c] = zt[c] * iz;
-                }
-                __syncthreads();
+                for (int c = 0; c < 8; c++) vj[c] = zt[c] * iz;
+            }
+            if (rbl == 0 && warp == 0) {
+#pragma unroll
+                for (int c = 0; c < 8; c++) sh.vec[j0 + c] = vj[c];
             }
             // sigma = |R v|, u = R v / sigma: columns of the new residual slot 0
             float s2 = 0.0f;

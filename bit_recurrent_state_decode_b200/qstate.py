@@ -26,7 +26,7 @@ F32, BF16, F16 = 0, 1, 2
 EXPORTS = ("qstate_create", "qstate_destroy", "qstate_reset", "qstate_step", "qstate_step_host",
            "qstate_step_host_static", "qstate_dequant", "qstate_export", "qstate_import", "qstate_get_sizes",
            "qstate_bytes_per_step", "qstate_status", "qstate_set_taxonomy", "qstate_set_lrb",
-           "qstate_lrb_export", "qstate_kernel", "qstate_debug_set", "qstate_error_string")
+           "qstate_lrb_export", "qstate_set_pw", "qstate_pw_export", "qstate_kernel", "qstate_debug_set", "qstate_error_string")
 
 
 class QStateError(RuntimeError):
@@ -85,6 +85,8 @@ def lib():
         L.qstate_set_taxonomy.argtypes = [P, I]
         L.qstate_set_lrb.argtypes = [P, I, I, ctypes.c_float]
         L.qstate_lrb_export.argtypes = [P, P, P, P, P, P, S]
+        L.qstate_set_pw.argtypes = [P, I]
+        L.qstate_pw_export.argtypes = [P, P, P, P, P, S]
         L.qstate_kernel.argtypes = [P]
         L.qstate_kernel.restype = ctypes.c_char_p
         L.qstate_error_string.argtypes = [I]
@@ -151,6 +153,7 @@ class QState:
         self.head_bits = None if head_bits is None else [int(b) for b in head_bits]
         self.rotation = int(rotation)
         self.lrb = None
+        self.pw = None
         z = Sizes()
         _check("qstate_get_sizes", lib().qstate_get_sizes(self._h, ctypes.byref(z)))
         self.sizes = {n: int(getattr(z, n)) for n, _ in Sizes._fields_}
@@ -299,6 +302,27 @@ class QState:
     def kernel(self) -> str:
         """The kernel the next step launches (qstate_kernel)."""
         return lib().qstate_kernel(self._h).decode()
+
+    def set_pw(self, W: int):
+        """Gated DeltaNet steps with a pure-write sliding window of W FP8
+        pairs (qstate_set_pw); before the first step."""
+        _check("qstate_set_pw", lib().qstate_set_pw(self._h, int(W)))
+        self.pw = int(W)
+
+    def pw_export(self, stream=None) -> dict:
+        """The window as new CUDA tensors: A [tiles, W, d_k], B [tiles, W, d_v]
+        (E4M3 bytes, uint8, by slot), head and count [tiles] (int32)."""
+        if self.pw is None:
+            raise QStateError("qstate_pw_export", 1)
+        T, W = self.tiles, self.pw
+        dev = f"cuda:{self.device}"
+        A = torch.empty((T, W, self.d_k), dtype=torch.uint8, device=dev)
+        B = torch.empty((T, W, self.d_v), dtype=torch.uint8, device=dev)
+        head = torch.empty((T,), dtype=torch.int32, device=dev)
+        count = torch.empty((T,), dtype=torch.int32, device=dev)
+        _check("qstate_pw_export", lib().qstate_pw_export(self._h, _ptr(A), _ptr(B), _ptr(head),
+                                                          _ptr(count), _stream(stream)))
+        return {"A": A, "B": B, "head": head, "count": count}
 
     def set_lrb(self, k: int, m: int, eps_l: float):
         """Low-Rank Bypass with a rank-k residual, a merge every m steps and

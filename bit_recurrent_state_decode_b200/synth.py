@@ -130,6 +130,7 @@ class Workload:
     description: str = ""
     rotation: int = 0            # 1: Hadamard-rotated state (INT4+Had)
     lrb: tuple = ()              # (k, m, eps_L): Low-Rank Bypass
+    pw: int = 0                  # W > 0: pure-write sliding window of W FP8 pairs
 
     @property
     def seed(self) -> int:
@@ -201,6 +202,13 @@ VARIANTS = {
         (PERSISTENT,), BDR, BF16, BF16, F16, layers=24, eps_b=0.3, lrb=(1, 15, 0.5),
         description="Gated DeltaNet x24 layers, INT4 g32 fp16 persistent scale with a Low-Rank "
                     "Bypass (k=1, m=15, eps_L=0.5) and BDR (eps_B=0.3): LRB+BDR of Table 6"),
+    # the 24-layer Gated DeltaNet decode with the pure-write window of
+    # "Low-Bit GDN Recurrent-State Quantization ..." at 8 pairs (PW-S8)
+    "gdn_l24_b256_h32_d128_int4g64_pw8": Workload(
+        "gdn_l24_b256_h32_d128_int4g64_pw8", 7, GDN, 256, 32, 128, 128, 2048, 4, 64,
+        (PERSISTENT,), BDR, BF16, BF16, F16, layers=24, pw=8,
+        description="Gated DeltaNet x24 layers, INT4 g64 fp16 persistent scale, BDR, with a "
+                    "pure-write window of 8 FP8 E4M3 pairs (PW-S8)"),
 }
 
 

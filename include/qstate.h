@@ -239,7 +239,8 @@ int qstate_dequant(const qstate* s, float* S_out, qstate_stream stream);
  * Used for checkpoints and teacher-forced parity (no counterpart on the
  * pages; the layouts are the ones above).  With a Low-Rank Bypass these are
  * the quantized part only (qstate_dequant likewise); import also empties the
- * bypass and sets D = 1. */
+ * bypass and sets D = 1.  With a pure-write window they are the history
+ * only; import also empties the window. */
 int qstate_export(const qstate* s, void* codes, void* scales, float* ref,
                   qstate_stream stream);
 int qstate_import(qstate* s, const void* codes, const void* scales, const float* ref,
@@ -285,11 +286,37 @@ int qstate_set_taxonomy(qstate* s, int on);
  * Mamba2 and Gated DeltaNet objects with one code width of 4 or 8 bits,
  * d_k = d_v in {64, 128}, dynamic or persistent scales, no rotation
  * (QSTATE_EUNSUPPORTED otherwise); allocates the bypass (QSTATE_ENOMEM).
- * QSTATE_EINVAL if already set or for invalid k, m, eps_l. */
+ * QSTATE_EINVAL if a bypass or a window is already set or for invalid k, m,
+ * eps_l. */
 int qstate_set_lrb(qstate* s, int k, int m, float eps_l);
 
+/* Switch a Gated DeltaNet object to steps with a pure-write sliding window
+ * (PW) of "Low-Bit GDN Recurrent-State Quantization: Global Gradient-aware
+ * Allocation and Pure-Write Sliding Windows" (Abstract), before its first
+ * step.  Each tile keeps, next to its quantized history (codes, scales), the
+ * W most recent pure writes beta k v^T as pairs of FP8 E4M3 vectors
+ * (a = beta k, b = v; OCP E4M3, nearest-even, saturating at 448).  Every
+ * step applies the transition alpha (I - beta k k^T) to the history (a
+ * Gated DeltaNet step without a write, requantized with the object's scale
+ * and rounding rules) and to every pair's key side (re-encoded in E4M3);
+ * when W pairs are held the oldest then leaves into the history before the
+ * step's own pair takes its slot; o is the whole state's output.  The state
+ * a tile stands for is dequant(codes) + sum over the pairs of a b^T.
+ * 1 <= W <= 16.  Supported for Gated DeltaNet objects with one code width
+ * of 4 or 8 bits, d_k = d_v in {64, 128}, dynamic or persistent scales, no
+ * rotation (QSTATE_EUNSUPPORTED otherwise); allocates the window
+ * (QSTATE_ENOMEM).  QSTATE_EINVAL if a window or a bypass is already set,
+ * or for an invalid W.  qstate_reset and qstate_import empty the window. */
+int qstate_set_pw(qstate* s, int W);
+
+/* Copy a PW object's window to caller buffers (device or host): A
+ * [tiles][W][d_k] and B [tiles][W][d_v] E4M3 bytes by slot, head [tiles]
+ * the slot of the oldest pair, count [tiles] the pairs held. */
+int qstate_pw_export(const qstate* s, uint8_t* A, uint8_t* B, int32_t* head, int32_t* count,
+                     qstate_stream stream);
+
 /* Name of the kernel the object's next step launches ("step_kernel",
- * "rows_kernel" or "lrb_kernel"; "" for NULL): for reports and profiles, no
+ * "rows_kernel", "lrb_kernel" or "pw_kernel"; "" for NULL): for reports and profiles, no
  * counterpart on the pages.  The string is static. */
 const char* qstate_kernel(const qstate* s);
 
