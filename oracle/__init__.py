@@ -115,6 +115,10 @@ def lib():
         _lib.or_pw_step.argtypes = [ctypes.POINTER(_Cfg), ctypes.c_int, ctypes.c_int64,
                                     P, P, P, P, P, P, P, P, P, P, P, P, P, P,
                                     ctypes.POINTER(Counts)]
+        _lib.or_rc_step.restype = ctypes.c_int
+        _lib.or_rc_step.argtypes = [ctypes.POINTER(_Cfg), ctypes.c_int64, P, P, P, P, P, P, P, P,
+                                    P, ctypes.POINTER(Counts)]
+        _lib.or_rc_dequant.argtypes = [ctypes.POINTER(_Cfg), P, P, P]
         _lib.or_rank_k.argtypes = [ctypes.c_int, ctypes.c_int, P, ctypes.c_int, P, P, P]
         _lib.or_lrb_bits.restype = ctypes.c_double
         _lib.or_lrb_bits.argtypes = [ctypes.c_int] * 5 + [ctypes.c_double]
@@ -473,6 +477,42 @@ class PwState(State):
         """History plus the window's pairs (fp64)."""
         a, b = self.pairs(t)
         return self.history(t) + a.T @ b
+
+
+class RcState(State):
+    """A quantized state with key-row x value-column scales (readings R1-R5
+    of the C code): codes as State, scales [T][d_k + d_v] (rho, then
+    kappa)."""
+
+    def __init__(self, cfg: Config, tile_bits):
+        super().__init__(cfg, tile_bits)
+        self.scales = np.zeros((self.ntiles, cfg.d_k + cfg.d_v), np.float32)
+
+    def step(self, q, k, v, alpha=None, beta=None, threads: int = 1):
+        cfg = self.cfg
+        T = self.ntiles
+        q, k, v = _f32(q).reshape(T, -1), _f32(k).reshape(T, -1), _f32(v).reshape(T, -1)
+        if alpha is not None:
+            alpha = _f32(alpha).reshape(T, -1)
+        if beta is not None:
+            beta = _f32(beta).reshape(T)
+        out = np.zeros((T, cfg.d_v), np.float32)
+        cnt = Counts()
+        rc = lib().or_rc_step(ctypes.byref(cfg.c), T, _ptr(self.tile_bits), _ptr(self.codes),
+                              _ptr(self.scales), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
+                              _ptr(beta), _ptr(out), ctypes.byref(cnt))
+        if rc != 0:
+            raise ValueError("oracle rejected the row x column configuration")
+        self._add_counts(cnt)
+        return out
+
+    def dequant(self) -> np.ndarray:
+        T = self.ntiles
+        out = np.zeros((T, self.cfg.d_k, self.cfg.d_v), np.float32)
+        for t in range(T):
+            lib().or_rc_dequant(ctypes.byref(self.cfg.c), _ptr(self.codes[t]),
+                                _ptr(self.scales[t]), _ptr(out[t]))
+        return out
 
 
 def step_many(work, threads: int = 1):

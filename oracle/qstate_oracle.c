@@ -971,3 +971,120 @@ int or_pw_step(const or_cfg* c, int W, int64_t ntiles, const int* tile_bits,
                      q + t * dk, k + t * dk, v + t * dv, alpha[t], beta[t], out + t * dv, cnt);
     return 0;
 }
+
+
+/* ------------------------------------------------------------------------
+ * Key-row x value-column scales ("STEPQuant: When and Where Errors Matter
+ * in Delta-Rule Recurrent State Quantization", Abstract: key-row and
+ * value-column scales fitted jointly from the state's distribution, the
+ * state's magnitudes varying along both rows and columns).  The page fits
+ * them offline against trained models' output error (out of scope here);
+ * this is the plainest joint fit from the state alone.  Readings:
+ *  R1 a tile holds row scales rho_i (i < d_k) and column scales kappa_j
+ *     (j < d_v) in the object's scale format; the grid step of element
+ *     (i, j) is Delta_ij = rho_i * kappa_j (a binary32 product, exact for
+ *     binary16 scales);
+ *  R2 fitted every step from the updated state x before rounding: kappa_j =
+ *     cvt(max_i |x_ij|) (the column maxima), ikappa_j = 1/kappa_j (0 for
+ *     0); rho_i = cvt(max_j(|x_ij| * ikappa_j) / Qmax) (each row's largest
+ *     column-normalised magnitude spread over the code range), irho_i =
+ *     1/rho_i (0 for 0);
+ *  R3 c_ij = clamp(rne(x_ij * inv_ij)), inv_ij = irho_i * ikappa_j (the
+ *     exact product x * inv rounded to nearest even, as the plain step);
+ *     BDR with a = the decayed state and the same inv;
+ *  R4 the decay of a quantized tile: a_ij = code_ij * ((alpha_i * rho_i) *
+ *     kappa_j), alpha_i the row's decay (GLA) or the scalar one;
+ *  R5 dynamic scales only (a carried or yoked rule is not defined for a
+ *     two-factor scale).
+ * ---------------------------------------------------------------------- */
+static void rc_tile_step(const or_cfg* c, int bits, int8_t* codes, float* scales,
+                         const float* q, const float* k, const float* v, const float* alpha,
+                         float beta, float* out, or_counts* cnt)
+{
+    const int dk = c->d_k, dv = c->d_v;
+    const size_t n_el = (size_t)dk * dv;
+    const int qmax = (1 << (bits - 1)) - 1;
+    const float fq = (float)qmax;
+    float* rho = scales;
+    float* kap = scales + dk;
+    float* a = (float*)malloc(sizeof(float) * n_el);
+    float* x = (float*)malloc(sizeof(float) * n_el);
+
+    /* R4: decay */
+    for (int i = 0; i < dk; i++) {
+        float al = c->kind == OR_RETNET ? c->gamma : c->kind == OR_GLA ? alpha[i] : alpha[0];
+        float ar = al * rho[i];
+        for (int j = 0; j < dv; j++) {
+            size_t e = (size_t)i * dv + j;
+            a[e] = (float)codes[e] * (ar * kap[j]);
+        }
+    }
+    /* update and output: the plain step's */
+    if (c->kind == OR_GDN) {
+        for (int j = 0; j < dv; j++) {
+            float r = or_canon_dot(dk, a + j, dv, k);
+            float e = v[j] - r;
+            for (int i = 0; i < dk; i++) {
+                size_t idx = (size_t)i * dv + j;
+                x[idx] = fmaf(beta * k[i], e, a[idx]);
+            }
+        }
+    } else {
+        for (int i = 0; i < dk; i++)
+            for (int j = 0; j < dv; j++) {
+                size_t idx = (size_t)i * dv + j;
+                x[idx] = fmaf(k[i], v[j], a[idx]);
+            }
+    }
+    for (int j = 0; j < dv; j++) out[j] = or_canon_dot(dk, x + j, dv, q);
+
+    /* R2: the scales */
+    float ikap[512], irho[512];
+    for (int j = 0; j < dv; j++) {
+        float m = 0.0f;
+        for (int i = 0; i < dk; i++) m = fmaxf(m, fabsf(x[(size_t)i * dv + j]));
+        kap[j] = to_stored_scale(c, m, cnt);
+        ikap[j] = kap[j] == 0.0f ? 0.0f : 1.0f / kap[j];
+    }
+    for (int i = 0; i < dk; i++) {
+        float m = 0.0f;
+        for (int j = 0; j < dv; j++) m = fmaxf(m, fabsf(x[(size_t)i * dv + j]) * ikap[j]);
+        rho[i] = to_stored_scale(c, m / fq, cnt);
+        irho[i] = rho[i] == 0.0f ? 0.0f : 1.0f / rho[i];
+    }
+    /* R3: rounding */
+    for (int i = 0; i < dk; i++)
+        for (int j = 0; j < dv; j++) {
+            size_t e = (size_t)i * dv + j;
+            codes[e] = (int8_t)or_round(c, a[e], x[e], irho[i] * ikap[j], qmax, cnt);
+        }
+    int bad = !finite_all(out, dv) || !finite_all(x, (int)n_el);
+    if (bad && cnt) cnt->nonfinite++;
+    free(a);
+    free(x);
+}
+
+int or_rc_step(const or_cfg* c, int64_t ntiles, const int* tile_bits, int8_t* codes,
+               float* scales, const float* q, const float* k, const float* v,
+               const float* alpha, const float* beta, float* out, or_counts* cnt)
+{
+    if (!valid_cfg(c) || c->scale_mode != OR_DYNAMIC || c->rotate) return -1;
+    if (c->d_k > 512 || c->d_v > 512) return -1;
+    const int dk = c->d_k, dv = c->d_v;
+    for (int64_t t = 0; t < ntiles; t++)
+        if (tile_bits[t] < 2 || tile_bits[t] > 8 || tile_bits[t] % 2) return -1;
+    const int na = c->kind == OR_GLA ? dk : 1;
+    for (int64_t t = 0; t < ntiles; t++)
+        rc_tile_step(c, tile_bits[t], codes + t * dk * dv, scales + t * (dk + dv), q + t * dk,
+                     k + t * dk, v + t * dv, alpha ? alpha + t * na : NULL,
+                     beta ? beta[t] : 0.0f, out + t * dv, cnt);
+    return 0;
+}
+
+void or_rc_dequant(const or_cfg* c, const int8_t* codes, const float* scales, float* S_out)
+{
+    const int dk = c->d_k, dv = c->d_v;
+    for (int i = 0; i < dk; i++)
+        for (int j = 0; j < dv; j++)
+            S_out[(size_t)i * dv + j] = (float)codes[(size_t)i * dv + j] * (scales[i] * scales[dk + j]);
+}

@@ -168,6 +168,19 @@ int or_pw_step(const or_cfg* c, int W, int64_t ntiles, const int* tile_bits,
                int* count, const float* q, const float* k, const float* v,
                const float* alpha, const float* beta, float* out, or_counts* cnt);
 
+/* ---- Key-row x value-column scales: readings R1-R5 in qstate_oracle.c --- */
+
+/* One step of ntiles tiles whose scales are a row vector rho [d_k] and a
+ * column vector kappa [d_v] per tile (scales [ntiles][d_k + d_v], rho
+ * first, in the configuration's scale format); widths 2..8, dynamic scales,
+ * all four kinds, RTN or BDR.  -1 if invalid. */
+int or_rc_step(const or_cfg* c, int64_t ntiles, const int* tile_bits, int8_t* codes,
+               float* scales, const float* q, const float* k, const float* v,
+               const float* alpha, const float* beta, float* out, or_counts* cnt);
+
+/* Dequantized tile of a row x column-scaled state: code * (rho_i * kappa_j). */
+void or_rc_dequant(const or_cfg* c, const int8_t* codes, const float* scales, float* S_out);
+
 #ifdef __cplusplus
 }
 #endif
