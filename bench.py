@@ -163,7 +163,7 @@ def cpu_oracle_rate(wl, seconds=10.0, threads=None, max_steps=None, tiles=None, 
     from bit_recurrent_state_decode_b200 import synth
     threads = threads or os.cpu_count() or 1
     cycle = 1
-    if wl.pw:
+    if wl.pw or wl.rowcol:
         tiles = tiles or 32
     if wl.lrb:
         # whole merge cycles (m steps, one of them a merge), after one cycle
@@ -189,6 +189,10 @@ def cpu_oracle_rate(wl, seconds=10.0, threads=None, max_steps=None, tiles=None, 
         elif wl.pw:
             # so does its windowed step
             states.append(oracle.PwState(cfg, tile_bits, wl.pw))
+            threads = 1
+        elif wl.rowcol:
+            # and its row x column step
+            states.append(oracle.RcState(cfg, tile_bits))
             threads = 1
         else:
             states.append(oracle.State(cfg, tile_bits))
@@ -249,6 +253,8 @@ def run_ours(args, rank, world, local_rank):
             o.set_lrb(*wl0.lrb)
         if wl0.pw:
             o.set_pw(wl0.pw)
+        if wl0.rowcol:
+            o.set_rowcol()
         return o
 
     probe = make(wl0.scale_modes[0], 1)

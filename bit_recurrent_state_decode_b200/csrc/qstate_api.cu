@@ -14,6 +14,7 @@
 #include "qstate_dispatch.h"
 #include "qstate_lrb.cuh"
 #include "qstate_pw.cuh"
+#include "qstate_rc.cuh"
 
 namespace qs {
 void launch_dequant_64_64(const StepParams&, float*, cudaStream_t);
@@ -77,6 +78,11 @@ struct qstate {
     float* d_lD = nullptr;
     const qs::LrbEntry* lrb_entry = nullptr;
     int lrb_grid = 1, lrb_smem = 0;
+    // key-row x value-column scales (qstate_set_rowcol): scales
+    // [tiles][d_k + d_v], rho then kappa
+    bool rowcol = false;
+    const qs::RcEntry* rc_entry = nullptr;
+    int rc_grid = 1;
     // pure-write sliding window (qstate_set_pw): the pairs, the slot of the
     // oldest pair and the pairs held, per tile
     bool pw = false;
@@ -456,6 +462,10 @@ int qstate_step(qstate* s, const void* q, const void* k, const void* v, const vo
     p.v = v;
     p.gates = gates;
     p.out = out;
+    if (s->rowcol) {
+        s->rc_entry->launch(p, s->rc_grid, 0, (cudaStream_t)stream);
+        return cudaGetLastError() == cudaSuccess ? QSTATE_OK : QSTATE_ECUDA;
+    }
     if (s->pw) {
         qs::PwParams Pp{s->d_pa, s->d_pb, s->d_phead, s->d_pcount, s->pw_W};
         s->pw_entry->launch(p, Pp, s->pw_grid, 0, (cudaStream_t)stream);
@@ -533,7 +543,10 @@ int qstate_dequant(const qstate* s, float* S_out, qstate_stream stream) {
     if (s->tiles == 0) return QSTATE_OK;
     int rc = check_device(s);
     if (rc != QSTATE_OK) return rc;
-    qs::launch_dequant(s->L.d_k, s->L.d_v, params_of(s), S_out, (cudaStream_t)stream);
+    if (s->rowcol)
+        s->rc_entry->dequant(params_of(s), S_out, s->rc_grid, (cudaStream_t)stream);
+    else
+        qs::launch_dequant(s->L.d_k, s->L.d_v, params_of(s), S_out, (cudaStream_t)stream);
     return cudaGetLastError() == cudaSuccess ? QSTATE_OK : QSTATE_ECUDA;
 }
 
@@ -597,8 +610,43 @@ int64_t qstate_bytes_per_step(const qstate* s) {
     return b + ops;
 }
 
+int qstate_set_rowcol(qstate* s) {
+    if (!s || s->rowcol || s->pw || s->lrb) return QSTATE_EINVAL;
+    const int dk = s->L.d_k, dv = s->L.d_v;
+    if (s->scale_mode != QSTATE_DYNAMIC || s->L.rotation || !s->head_bits.empty() ||
+        !(s->bits == 4 || s->bits == 8))
+        return QSTATE_EUNSUPPORTED;
+    int rc = check_device(s);
+    if (rc != QSTATE_OK) return rc;
+    const qs::RcEntry* tab = dk == 64 ? (dv == 64 ? qs::rc_table_64_64() : qs::rc_table_64_128())
+                                      : (dv == 64 ? qs::rc_table_128_64() : qs::rc_table_128_128());
+    const int idx = (((s->bits == 8) * 2 + (s->L.kind == QSTATE_GDN)) * 2 +
+                     (s->round_mode == QSTATE_BDR)) * 2 + (s->L.qkv_dtype == QSTATE_BF16);
+    const qs::RcEntry* e = &tab[idx];
+    const int per_sm = e->blocks_per_sm(0);
+    if (per_sm < 1) { cudaGetLastError(); return QSTATE_EUNSUPPORTED; }
+    const int64_t n_scales = dk + dv;
+    const int64_t bytes = s->tiles * n_scales * s->scale_size;
+    void* ns = nullptr;
+    if (bytes && cudaMalloc(&ns, bytes) != cudaSuccess) { cudaGetLastError(); return QSTATE_ENOMEM; }
+    cudaFree(s->d_scales);
+    s->d_scales = ns;
+    s->n_scales = n_scales;
+    s->scale_bytes = bytes;
+    s->rowcol = true;
+    s->rc_entry = e;
+    int sms = 0;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, s->device);
+    int64_t g = (int64_t)sms * per_sm;
+    if (s->tiles < g) g = s->tiles > 0 ? s->tiles : 1;
+    s->rc_grid = (int)g;
+    rc = zero_state(s, nullptr);
+    if (rc == QSTATE_OK && cudaDeviceSynchronize() != cudaSuccess) rc = QSTATE_ECUDA;
+    return rc;
+}
+
 int qstate_set_pw(qstate* s, int W) {
-    if (!s || s->pw || s->lrb) return QSTATE_EINVAL;
+    if (!s || s->pw || s->lrb || s->rowcol) return QSTATE_EINVAL;
     if (W < 1 || W > qs::kPwMaxW) return QSTATE_EINVAL;
     if (s->L.kind != QSTATE_GDN || s->scale_mode == QSTATE_YOKED || s->L.rotation ||
         !s->head_bits.empty() || !(s->bits == 4 || s->bits == 8) || s->L.d_k != s->L.d_v)
@@ -649,7 +697,7 @@ int qstate_pw_export(const qstate* s, uint8_t* A, uint8_t* B, int32_t* head, int
 }
 
 int qstate_set_lrb(qstate* s, int k, int m, float eps_l) {
-    if (!s || s->lrb || s->pw) return QSTATE_EINVAL;
+    if (!s || s->lrb || s->pw || s->rowcol) return QSTATE_EINVAL;
     if (k < 0 || k > 1 || m < 1 || k + m > qs::kLrbMaxCols) return QSTATE_EINVAL;
     if (!(eps_l >= 0.0f) || !std::isfinite(eps_l)) return QSTATE_EINVAL;
     if (s->L.kind == QSTATE_GLA || s->scale_mode == QSTATE_YOKED || s->L.rotation ||
@@ -696,6 +744,7 @@ const char* qstate_kernel(const qstate* s) {
     if (!s) return "";
     if (s->lrb) return "lrb_kernel";
     if (s->pw) return "pw_kernel";
+    if (s->rowcol) return "rc_kernel";
     if (s->taxonomy || s->L.rotation) return "step_kernel";
     return s->entry_name;
 }

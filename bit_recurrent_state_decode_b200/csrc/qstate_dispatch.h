@@ -56,6 +56,19 @@ struct PwEntry {
 };
 const PwEntry* pw_table();
 
+// The decode step with key-row x value-column scales: per shape 16 entries
+// indexed by (((bits == 8) * 2 + gdn) * 2 + bdr) * 2 + bf16.
+struct RcEntry {
+    void (*launch)(const StepParams&, int grid, int dyn_smem, cudaStream_t);
+    int (*blocks_per_sm)(int dyn_smem);
+    void (*dequant)(const StepParams&, float* S, int grid, cudaStream_t);
+    int threads;
+};
+const RcEntry* rc_table_64_64();
+const RcEntry* rc_table_64_128();
+const RcEntry* rc_table_128_64();
+const RcEntry* rc_table_128_128();
+
 // 0 = per-head widths, then 2, 4, 6, 8, 32 bits; -1 if invalid
 inline int bits_index(int bits) {
     switch (bits) {

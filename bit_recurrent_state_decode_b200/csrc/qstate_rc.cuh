@@ -1,0 +1,270 @@
+// qstate_rc.cuh -- the decode step of a state quantized with key-row x
+// value-column scales ("STEPQuant: When and Where Errors Matter in
+// Delta-Rule Recurrent State Quantization", Abstract), fitted every step
+// from the state itself: kappa_j = cvt(max_i |x_ij|), rho_i =
+// cvt(max_j(|x_ij| / kappa_j) / Qmax), grid step rho_i * kappa_j.
+//
+// Per tile: a_ij = code * ((alpha_i * rho_i) * kappa_j); the update and the
+// output are the plain step's (rank-1, or the delta rule with r = a^T k);
+// then the column maxima, the column scales and their reciprocals, the row
+// maxima of the column-normalised magnitudes, the row scales, and
+// c = clamp(rne(x * (1/rho_i * 1/kappa_j))) (BDR with d = x - a).  Every
+// result is defined element by element and matches the definition bit for
+// bit.  One tile per CTA at a time, plain loads with the next tile's bytes
+// prefetched to L2 (like the bypass and window steps).
+#pragma once
+
+#include "qstate_lrb.cuh"
+
+namespace qs {
+
+template <int DK, int DV>
+struct __align__(16) RcShared {
+    using G = Geo<DK, DV>;
+    float red[G::NWARPS * DV];
+    float tot[DV];
+    float rho[DK];                   // the previous row scales
+    float kap[DV];                   // the previous column scales
+    int bad;
+};
+
+// Maximum over the row blocks of a warp and then over the warps of a
+// per-thread 8-column partial (max is exact: any order); every thread gets
+// its 8 column maxima.
+template <int DK, int DV>
+__device__ __forceinline__ void colmax_finish(float (&p)[8], float* red, float* tot, int warp,
+                                              int rbl, int j0, float (&res)[8]) {
+    using G = Geo<DK, DV>;
+#pragma unroll
+    for (int off = G::CBW; off < 32; off <<= 1) {
+#pragma unroll
+        for (int c = 0; c < 8; c++) p[c] = fmaxf(p[c], __shfl_xor_sync(0xFFFFFFFFu, p[c], off));
+    }
+    if (rbl == 0) {
+#pragma unroll
+        for (int c = 0; c < 8; c++) red[warp * DV + j0 + c] = p[c];
+    }
+    __syncthreads();
+    for (int j = threadIdx.x; j < DV; j += G::NT) {
+        float t = red[j];
+#pragma unroll
+        for (int w2 = 1; w2 < G::NWARPS; w2++) t = fmaxf(t, red[w2 * DV + j]);
+        tot[j] = t;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int c = 0; c < 8; c++) res[c] = tot[j0 + c];
+}
+
+template <int DK, int DV, int BITS, bool GDN, bool BDR, bool BF>
+__global__ void __launch_bounds__(Geo<DK, DV>::NT, 1) rc_kernel(const StepParams p) {
+    using G = Geo<DK, DV>;
+    static_assert(BITS == 4 || BITS == 8, "4- or 8-bit codes");
+    constexpr int QMAX = (1 << (BITS - 1)) - 1;
+    constexpr float fq = float(QMAX);
+    constexpr float rq = QMAX == 7 ? 0x1.24924ap-3f : 0x1.020408p-7f;
+    __shared__ RcShared<DK, DV> sh;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int cb = lane % G::CBW, rbl = lane / G::CBW;
+    const int i0 = (warp * G::RBW + rbl) * 8, j0 = cb * 8;
+    const bool sf32 = p.scale_f32 != 0;
+    const int isz = BF ? 2 : 4;
+
+    for (long long tile = blockIdx.x; tile < p.ntiles; tile += gridDim.x) {
+        uint8_t* ct = p.codes + tile * p.tile_bytes;
+        const long long sbase = tile * (long long)(DK + DV);
+        {
+            const long long nt = tile + gridDim.x;
+            if (nt < p.ntiles) {
+                const int ssz = sf32 ? 4 : 2;
+                prefetch_l2<G::NT>(p.codes + nt * p.tile_bytes, p.tile_bytes);
+                prefetch_l2<G::NT>(static_cast<const uint8_t*>(p.scales) + nt * (DK + DV) * ssz,
+                                   (long long)(DK + DV) * ssz);
+                if (threadIdx.x < 3) {
+                    const void* src = threadIdx.x == 0 ? p.q : threadIdx.x == 1 ? p.k : p.v;
+                    const int n = threadIdx.x == 2 ? DV : DK;
+                    const char* b = static_cast<const char*>(src) + nt * n * isz;
+                    for (int o = 0; o < n * isz; o += 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(b + o));
+                }
+            }
+        }
+        for (int i = threadIdx.x; i < DK + DV; i += G::NT) {
+            const float s = scale_at(p.scales, sbase + i, sf32);
+            if (i < DK) sh.rho[i] = s;
+            else sh.kap[i - DK] = s;
+        }
+        if (threadIdx.x == 0) sh.bad = 0;
+        const uint8_t* kin = static_cast<const uint8_t*>(p.k) + tile * DK * isz;
+        const uint8_t* qin = static_cast<const uint8_t*>(p.q) + tile * DK * isz;
+        const uint8_t* vin = static_cast<const uint8_t*>(p.v) + tile * DV * isz;
+        float kk[8], qq[8], vv[8], al[8];
+#pragma unroll
+        for (int r = 0; r < 8; r++) {
+            kk[r] = ldg1(kin, i0 + r, BF);
+            qq[r] = ldg1(qin, i0 + r, BF);
+            al[r] = p.kind == K_RETNET ? p.gamma
+                  : p.kind == K_GLA    ? ldg1(p.gates, tile * p.n_gate + i0 + r, p.gate_bf16 != 0)
+                                       : ldg1(p.gates, tile * p.n_gate, p.gate_bf16 != 0);
+        }
+#pragma unroll
+        for (int c = 0; c < 8; c++) vv[c] = ldg1(vin, j0 + c, BF);
+        const float beta = GDN ? ldg1(p.gates, tile * p.n_gate + 1, p.gate_bf16 != 0) : 0.0f;
+        __syncthreads();
+
+        // the decayed state: a = code * ((alpha_i * rho_i) * kappa_j)
+        float a[8][8];
+        {
+            float kp[8];
+#pragma unroll
+            for (int c = 0; c < 8; c++) kp[c] = sh.kap[j0 + c];
+#pragma unroll
+            for (int r = 0; r < 8; r++) {
+                float c8[8];
+                if constexpr (BITS == 4) Decode<4>::run(ct + (i0 + r) * (DV / 2), cb, c8);
+                else Decode<8>::run(ct + (i0 + r) * DV, cb, c8);
+                const float ar = __fmul_rn(al[r], sh.rho[i0 + r]);
+#pragma unroll
+                for (int c = 0; c < 8; c++) a[r][c] = __fmul_rn(c8[c], __fmul_rn(ar, kp[c]));
+            }
+        }
+        // the update
+        float x[8][8];
+        if constexpr (GDN) {
+            float pr[8];
+#pragma unroll
+            for (int c = 0; c < 8; c++) pr[c] = 0.0f;
+#pragma unroll
+            for (int r = 0; r < 8; r++)
+#pragma unroll
+                for (int c = 0; c < 8; c++) pr[c] = __fmaf_rn(a[r][c], kk[r], pr[c]);
+            float rr[8];
+            colsum_finish<DK, DV>(pr, sh.red, sh.tot, warp, rbl, j0, rr);
+#pragma unroll
+            for (int r = 0; r < 8; r++) {
+                const float kap = __fmul_rn(beta, kk[r]);
+#pragma unroll
+                for (int c = 0; c < 8; c++) x[r][c] = __fmaf_rn(kap, __fsub_rn(vv[c], rr[c]), a[r][c]);
+            }
+        } else {
+#pragma unroll
+            for (int r = 0; r < 8; r++)
+#pragma unroll
+                for (int c = 0; c < 8; c++) x[r][c] = __fmaf_rn(kk[r], vv[c], a[r][c]);
+        }
+        // the output from the state before rounding
+        bool bad = false;
+        {
+            float po[8];
+#pragma unroll
+            for (int c = 0; c < 8; c++) po[c] = 0.0f;
+#pragma unroll
+            for (int r = 0; r < 8; r++)
+#pragma unroll
+                for (int c = 0; c < 8; c++) po[c] = __fmaf_rn(x[r][c], qq[r], po[c]);
+            float oo[8];
+            colsum_finish<DK, DV>(po, sh.red, sh.tot, warp, rbl, j0, oo);
+            if (rbl == 0 && warp == 0) {
+#pragma unroll
+                for (int c = 0; c < 8; c++) {
+                    p.out[tile * DV + j0 + c] = oo[c];
+                    bad |= !isfinite(oo[c]);
+                }
+            }
+        }
+        // the column scales and their reciprocals
+        float ik[8];
+        unsigned nsat = 0;
+        {
+            float m[8];
+#pragma unroll
+            for (int c = 0; c < 8; c++) {
+                float t = 0.0f;
+#pragma unroll
+                for (int r = 0; r < 8; r++) {
+                    t = fmaxf(t, fabsf(x[r][c]));
+                    bad |= !isfinite(x[r][c]);
+                }
+                m[c] = t;
+            }
+            float cm[8];
+            colmax_finish<DK, DV>(m, sh.red, sh.tot, warp, rbl, j0, cm);
+#pragma unroll
+            for (int c = 0; c < 8; c++) {
+                bool sat = false;
+                const float kap = to_stored(cm[c], sf32, sat);
+                ik[c] = kap == 0.0f ? 0.0f : __frcp_rn(kap);
+                if (rbl == 0 && warp == 0) {
+                    store_scale(p.scales, sbase + DK + j0 + c, sf32, kap);
+                    nsat += sat ? 1u : 0u;
+                }
+            }
+        }
+        // the row scales from the column-normalised magnitudes
+        float ir[8];
+#pragma unroll
+        for (int r = 0; r < 8; r++) {
+            float t = 0.0f;
+#pragma unroll
+            for (int c = 0; c < 8; c++) t = fmaxf(t, __fmul_rn(fabsf(x[r][c]), ik[c]));
+#pragma unroll
+            for (int off = 1; off < G::CBW; off <<= 1) t = fmaxf(t, __shfl_xor_sync(0xFFFFFFFFu, t, off));
+            bool sat = false;
+            const float rho = to_stored(div_by_qmax(t, fq, rq), sf32, sat);
+            ir[r] = rho == 0.0f ? 0.0f : __frcp_rn(rho);
+            if (cb == 0) {
+                store_scale(p.scales, sbase + i0 + r, sf32, rho);
+                nsat += sat ? 1u : 0u;
+            }
+        }
+        if (nsat) atomicAdd(p.counters + 1, (unsigned long long)nsat);
+        if (bad) sh.bad = 1;
+        // round (BDR: a reversed element moves one code toward its update) and pack
+#pragma unroll
+        for (int r = 0; r < 8; r++) {
+            float t8[8];
+#pragma unroll
+            for (int c = 0; c < 8; c++) {
+                const float inv = __fmul_rn(ir[r], ik[c]);
+                float t = fminf(fmaxf(__fmaf_rn(x[r][c], inv, kMagic), kMagic - fq), kMagic + fq);
+                if (BDR) {
+                    const float d = __fsub_rn(x[r][c], a[r][c]);
+                    const float s = __fmaf_rn(a[r][c], inv, -__fsub_rn(t, kMagic));
+                    if (d > 0.0f && s > p.eps_b) t = fminf(__fadd_rn(t, 1.0f), kMagic + fq);
+                    else if (d < 0.0f && s < -p.eps_b) t = fmaxf(__fsub_rn(t, 1.0f), kMagic - fq);
+                }
+                t8[c] = t;
+            }
+            pack_row<DK, DV, BITS>(ct, i0 + r, cb, t8);
+        }
+        __syncthreads();
+        if (threadIdx.x == 0 && sh.bad) atomicAdd(p.counters, 1ull);
+    }
+}
+
+// Dequantized state of a row x column-scaled object: code * (rho_i * kappa_j).
+template <int DK, int DV, int BITS>
+__global__ void __launch_bounds__(Geo<DK, DV>::NT) rc_dequant_kernel(const StepParams p, float* S) {
+    using G = Geo<DK, DV>;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int cb = lane % G::CBW, rbl = lane / G::CBW;
+    const int i0 = (warp * G::RBW + rbl) * 8, j0 = cb * 8;
+    const bool sf32 = p.scale_f32 != 0;
+    for (long long tile = blockIdx.x; tile < p.ntiles; tile += gridDim.x) {
+        const uint8_t* ct = p.codes + tile * p.tile_bytes;
+        const long long sbase = tile * (long long)(DK + DV);
+#pragma unroll
+        for (int r = 0; r < 8; r++) {
+            float c8[8];
+            if constexpr (BITS == 4) Decode<4>::run(ct + (i0 + r) * (DV / 2), cb, c8);
+            else Decode<8>::run(ct + (i0 + r) * DV, cb, c8);
+            const float rho = scale_at(p.scales, sbase + i0 + r, sf32);
+#pragma unroll
+            for (int c = 0; c < 8; c++) {
+                const float kap = scale_at(p.scales, sbase + DK + j0 + c, sf32);
+                S[(tile * DK + i0 + r) * DV + j0 + c] = __fmul_rn(c8[c], __fmul_rn(rho, kap));
+            }
+        }
+    }
+}
+
+}  // namespace qs

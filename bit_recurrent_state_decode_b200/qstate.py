@@ -26,7 +26,8 @@ F32, BF16, F16 = 0, 1, 2
 EXPORTS = ("qstate_create", "qstate_destroy", "qstate_reset", "qstate_step", "qstate_step_host",
            "qstate_step_host_static", "qstate_dequant", "qstate_export", "qstate_import", "qstate_get_sizes",
            "qstate_bytes_per_step", "qstate_status", "qstate_set_taxonomy", "qstate_set_lrb",
-           "qstate_lrb_export", "qstate_set_pw", "qstate_pw_export", "qstate_kernel", "qstate_debug_set", "qstate_error_string")
+           "qstate_lrb_export", "qstate_set_pw", "qstate_pw_export", "qstate_set_rowcol",
+           "qstate_kernel", "qstate_debug_set", "qstate_error_string")
 
 
 class QStateError(RuntimeError):
@@ -87,6 +88,7 @@ def lib():
         L.qstate_lrb_export.argtypes = [P, P, P, P, P, P, S]
         L.qstate_set_pw.argtypes = [P, I]
         L.qstate_pw_export.argtypes = [P, P, P, P, P, S]
+        L.qstate_set_rowcol.argtypes = [P]
         L.qstate_kernel.argtypes = [P]
         L.qstate_kernel.restype = ctypes.c_char_p
         L.qstate_error_string.argtypes = [I]
@@ -154,6 +156,7 @@ class QState:
         self.rotation = int(rotation)
         self.lrb = None
         self.pw = None
+        self.rowcol = False
         z = Sizes()
         _check("qstate_get_sizes", lib().qstate_get_sizes(self._h, ctypes.byref(z)))
         self.sizes = {n: int(getattr(z, n)) for n, _ in Sizes._fields_}
@@ -302,6 +305,15 @@ class QState:
     def kernel(self) -> str:
         """The kernel the next step launches (qstate_kernel)."""
         return lib().qstate_kernel(self._h).decode()
+
+    def set_rowcol(self):
+        """Key-row x value-column scales (qstate_set_rowcol); before the
+        first step.  The scales become [tiles, d_k + d_v] (rho, then kappa)."""
+        _check("qstate_set_rowcol", lib().qstate_set_rowcol(self._h))
+        self.rowcol = True
+        z = Sizes()
+        _check("qstate_get_sizes", lib().qstate_get_sizes(self._h, ctypes.byref(z)))
+        self.sizes = {n: int(getattr(z, n)) for n, _ in Sizes._fields_}
 
     def set_pw(self, W: int):
         """Gated DeltaNet steps with a pure-write sliding window of W FP8

@@ -131,6 +131,7 @@ class Workload:
     rotation: int = 0            # 1: Hadamard-rotated state (INT4+Had)
     lrb: tuple = ()              # (k, m, eps_L): Low-Rank Bypass
     pw: int = 0                  # W > 0: pure-write sliding window of W FP8 pairs
+    rowcol: bool = False         # key-row x value-column scales
 
     @property
     def seed(self) -> int:
@@ -209,6 +210,13 @@ VARIANTS = {
         (PERSISTENT,), BDR, BF16, BF16, F16, layers=24, pw=8,
         description="Gated DeltaNet x24 layers, INT4 g64 fp16 persistent scale, BDR, with a "
                     "pure-write window of 8 FP8 E4M3 pairs (PW-S8)"),
+    # the same decode with key-row x value-column scales (STEPQuant's layout,
+    # fitted from the state every step): 4.25 bits per element
+    "gdn_l24_b256_h32_d128_int4rc": Workload(
+        "gdn_l24_b256_h32_d128_int4rc", 8, GDN, 256, 32, 128, 128, 2048, 4, 0,
+        (DYNAMIC,), BDR, BF16, BF16, F16, layers=24, rowcol=True,
+        description="Gated DeltaNet x24 layers, INT4 with fp16 key-row x value-column scales "
+                    "fitted every step, BDR, bf16"),
 }
 
 

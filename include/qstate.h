@@ -286,8 +286,8 @@ int qstate_set_taxonomy(qstate* s, int on);
  * Mamba2 and Gated DeltaNet objects with one code width of 4 or 8 bits,
  * d_k = d_v in {64, 128}, dynamic or persistent scales, no rotation
  * (QSTATE_EUNSUPPORTED otherwise); allocates the bypass (QSTATE_ENOMEM).
- * QSTATE_EINVAL if a bypass or a window is already set or for invalid k, m,
- * eps_l. */
+ * QSTATE_EINVAL if a bypass, a window or row x column scales are already set
+ * or for invalid k, m, eps_l. */
 int qstate_set_lrb(qstate* s, int k, int m, float eps_l);
 
 /* Switch a Gated DeltaNet object to steps with a pure-write sliding window
@@ -305,8 +305,9 @@ int qstate_set_lrb(qstate* s, int k, int m, float eps_l);
  * 1 <= W <= 16.  Supported for Gated DeltaNet objects with one code width
  * of 4 or 8 bits, d_k = d_v in {64, 128}, dynamic or persistent scales, no
  * rotation (QSTATE_EUNSUPPORTED otherwise); allocates the window
- * (QSTATE_ENOMEM).  QSTATE_EINVAL if a window or a bypass is already set,
- * or for an invalid W.  qstate_reset and qstate_import empty the window. */
+ * (QSTATE_ENOMEM).  QSTATE_EINVAL if a window, a bypass or row x column
+ * scales are already set, or for an invalid W.  qstate_reset and
+ * qstate_import empty the window. */
 int qstate_set_pw(qstate* s, int W);
 
 /* Copy a PW object's window to caller buffers (device or host): A
@@ -315,8 +316,26 @@ int qstate_set_pw(qstate* s, int W);
 int qstate_pw_export(const qstate* s, uint8_t* A, uint8_t* B, int32_t* head, int32_t* count,
                      qstate_stream stream);
 
+/* Switch the object to key-row x value-column scales ("STEPQuant: When and
+ * Where Errors Matter in Delta-Rule Recurrent State Quantization",
+ * Abstract), before its first step: the scales become, per tile, row scales
+ * rho [d_k] then column scales kappa [d_v] (scales [tiles][d_k + d_v] in the
+ * layout's scale format; qstate_get_sizes reports the new size), the grid
+ * step of element (i, j) is rho_i * kappa_j, and every step fits them from
+ * the updated state x before rounding: kappa_j = cvt(max_i |x_ij|),
+ * rho_i = cvt(max_j(|x_ij| * (1/kappa_j)) / Qmax), codes
+ * c = clamp(rne(x * ((1/rho_i) * (1/kappa_j)))) (BDR with d = x - a), the
+ * decay a = code * ((alpha_i * rho_i) * kappa_j).  The update and output
+ * are the plain step's.  The page fits these scales offline against trained
+ * models; this joint fit from the state alone is this library's reading.
+ * Supported for all four kinds, one code width of 4 or 8 bits, dynamic
+ * scales, no rotation (QSTATE_EUNSUPPORTED otherwise); the state is reset.
+ * QSTATE_EINVAL if already set or with a bypass or window.  The taxonomy
+ * counts are not kept for such objects. */
+int qstate_set_rowcol(qstate* s);
+
 /* Name of the kernel the object's next step launches ("step_kernel",
- * "rows_kernel", "lrb_kernel" or "pw_kernel"; "" for NULL): for reports and profiles, no
+ * "rows_kernel", "lrb_kernel", "pw_kernel" or "rc_kernel"; "" for NULL): for reports and profiles, no
  * counterpart on the pages.  The string is static. */
 const char* qstate_kernel(const qstate* s);
 

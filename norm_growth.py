@@ -3,9 +3,9 @@
     python norm_growth.py [--steps 32768] [--every 64]
 
 "When Dynamic Scaling Fails" (Abstract) reports that a scale re-derived from
-the state every step feeds back into the state and makes its norm explode,
-and that yoking the scale to a full-precision reference removes the
-explosion.  This runs the long-horizon Gated DeltaNet workload (batch 32,
+the state at every step forms a loop with the state that can make its norm
+grow without bound, and that tying the scale to an unquantized copy of the
+state prevents that.  This runs the long-horizon Gated DeltaNet workload (batch 32,
 16 heads, d_k = d_v = 128, per-head widths {2, 4, 6, 8} with mean 4, group 64,
 binary32 scales, BDR) with the three scale modes side by side on the same
 seeded inputs and reports, every `--every` steps,
@@ -91,7 +91,7 @@ def main(argv=None):
     ap.add_argument("--every", type=int, default=64)
     ap.add_argument("--batch", type=int, default=0)
     a = ap.parse_args(argv)
-    from . import build
+    from bit_recurrent_state_decode_b200 import build
     build.build()
     print(json.dumps(run(a.steps, a.every, a.batch or None)))
 

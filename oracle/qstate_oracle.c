@@ -174,8 +174,9 @@ float or_canon_dot(int n, const float* a, int stride, const float* b)
 }
 
 /* ------------------------------------------------------------------------
- * Hadamard rotation ("INT4+Had applies a Hadamard rotation before INT4
- * quantization", Table 2 of "Preserving Updates ...").
+ * Hadamard rotation (INT4+Had of Table 2 of "Preserving Updates ...": the
+ * state is rotated by a Hadamard matrix before it is quantized to INT4; the
+ * page says no more).
  * Reading: the rotation acts on the value axis of the state (the axis the
  * scale groups run along), S_rot = S H with H the Sylvester Hadamard matrix of
  * order d_v (entries +-1, symmetric, H H = d_v I).  Every decay A_t acts on the
@@ -217,8 +218,8 @@ int or_round_rtn(float x, float inv, int qmax)
     return (int)r;
 }
 
-/* BDR.  Reading of "rounds reversed elements toward their updates" with the
- * threshold eps_B of Table 6: the update of the element is d = x - a (a is
+/* BDR.  Reading of its rule (a reversed element is rounded in the direction
+ * of its update instead) with the threshold eps_B of Table 6: the update of the element is d = x - a (a is
  * the decayed state before the update), u = a * inv is where the element
  * sits on the new grid without the update.  The element is reversed when its
  * RTN code lies on the far side of u from the update by more than eps_B grid
@@ -490,9 +491,9 @@ void or_dequant(const or_cfg* c, int bits, const int8_t* codes, const float* sca
 
 /* ========================================================================
  * Low-Rank Bypass (LRB), "Preserving Updates in Low-Bit Recurrent State
- * Quantization": the Abstract (small updates are accumulated in a compact
- * low-rank buffer whose sufficiently large elements are periodically merged
- * into the state), Figure 3 (updates go to the bypass and are written into
+ * Quantization": the Abstract (small updates collect in a low-rank buffer,
+ * and the buffer's large elements go into the state from time to time),
+ * Figure 3 (updates go to the bypass and are written into
  * the quantized state every m steps), Table 6 (k, m, eps_L per model, and
  * the average / peak storage per state element) and Tables 8-9 (the rank k
  * and the number k + m of bypass columns).
