@@ -91,20 +91,24 @@ __device__ __forceinline__ void prefetch_l2(const void* p, long long bytes) {
 // Round x with the scale's reciprocal: code = clamp(RTN(x * inv)); with BDR
 // a reversed element (d = x - a, s = fma(a, inv, -code), d > 0 and s > eps_B,
 // or d < 0 and s < -eps_B) moves one code toward its update, clamped.
-template <int DK, int DV, int BITS, bool BDR>
-__device__ __forceinline__ void round_pack_ax(const float (&a)[8][8], const float (&x)[8][8],
+// arow(r, a8) gives row r of this thread's decayed state a (read only with
+// BDR, before row r's codes are written).
+template <int DK, int DV, int BITS, bool BDR, class ARow>
+__device__ __forceinline__ void round_pack_ax(ARow arow, const float (&x)[8][8],
                                               const float (&inv)[8], float eps_b, uint8_t* ct,
                                               int i0, int cb) {
     constexpr float fq = float((1 << (BITS - 1)) - 1);
 #pragma unroll
     for (int r = 0; r < 8; r++) {
         float t8[8];
+        float ar[8];
+        if (BDR) arow(r, ar);
 #pragma unroll
         for (int c = 0; c < 8; c++) {
             float t = fminf(fmaxf(__fmaf_rn(x[r][c], inv[r], kMagic), kMagic - fq), kMagic + fq);
             if (BDR) {
-                const float d = __fsub_rn(x[r][c], a[r][c]);
-                const float s = __fmaf_rn(a[r][c], inv[r], -__fsub_rn(t, kMagic));
+                const float d = __fsub_rn(x[r][c], ar[c]);
+                const float s = __fmaf_rn(ar[c], inv[r], -__fsub_rn(t, kMagic));
                 if (d > 0.0f && s > eps_b) t = fminf(__fadd_rn(t, 1.0f), kMagic + fq);
                 else if (d < 0.0f && s < -eps_b) t = fmaxf(__fsub_rn(t, 1.0f), kMagic - fq);
             }
@@ -123,14 +127,14 @@ __device__ __forceinline__ void colsum_any(float (&p)[8], float* red, float* tot
     colsum_finish<DK, DV>(p, red, tot, warp, rbl, j0, res);
 }
 
-// Requantize a tile's updated state x (a: the decayed state before the
-// update, for BDR) with the object's scale rule (dynamic or persistent,
-// per-group or per-token; previous scales in `sprev`, in their stored
-// format): new scales and codes written to HBM, saturated scales and
+// Requantize a tile's updated state x (arow: rows of the decayed state a
+// before the update, for BDR) with the object's scale rule (dynamic or
+// persistent, per-group or per-token; previous scales in `sprev`, in their
+// stored format): new scales and codes written to HBM, saturated scales and
 // non-finite group maxima counted.  Every thread of the CTA calls it.
-template <int DK, int DV, int BITS, bool BDR, class XS>
+template <int DK, int DV, int BITS, bool BDR, class XS, class ARow>
 __device__ __forceinline__ void requantize(const StepParams& p, XS& xs, const uint8_t* sprev,
-                                           long long sbase, uint8_t* ct, const float (&a)[8][8],
+                                           long long sbase, uint8_t* ct, ARow arow,
                                            const float (&x)[8][8], int lane, int warp, int cb,
                                            int i0, int ng, int gcol) {
     using G = Geo<DK, DV>;
@@ -207,11 +211,14 @@ __device__ __forceinline__ void requantize(const StepParams& p, XS& xs, const ui
     }
     if (nsat) atomicAdd(p.counters + 1, (unsigned long long)nsat);
     if (bad && threadIdx.x == 0) atomicAdd(p.counters, 1ull);
-    round_pack_ax<DK, DV, BITS, BDR>(a, x, inv, p.eps_b, ct, i0, cb);
+    round_pack_ax<DK, DV, BITS, BDR>(arow, x, inv, p.eps_b, ct, i0, cb);
 }
 
+// Two CTAs per SM: the decayed quantized part a is re-derived from the codes
+// (an L1 hit after the first read) wherever the step needs it, so only the
+// merge's 8 x 8 block stays in registers.
 template <int DK, int DV, int BITS, bool GDN, bool BDR, bool BF>
-__global__ void __launch_bounds__(Geo<DK, DV>::NT, 1) lrb_kernel(const StepParams p, const LrbParams L) {
+__global__ void __launch_bounds__(Geo<DK, DV>::NT, 2) lrb_kernel(const StepParams p, const LrbParams L) {
     using G = Geo<DK, DV>;
     static_assert(DK == DV, "square tiles");
     static_assert(BITS == 4 || BITS == 8, "4- or 8-bit codes");
@@ -312,15 +319,14 @@ __global__ void __launch_bounds__(Geo<DK, DV>::NT, 1) lrb_kernel(const StepParam
 #pragma unroll
             for (int c = 0; c < 8; c++) vv[c] = ldg1(vin, j0 + c, BF);
         }
-        float a[8][8];
-#pragma unroll
-        for (int r = 0; r < 8; r++) {
+        // row r of this thread's a = code * (D * scale)
+        auto arow = [&](int r, float (&ar)[8]) {
             float c8[8];
             if constexpr (BITS == 4) Decode<4>::run(ct + (i0 + r) * (DV / 2), cb, c8);
             else Decode<8>::run(ct + (i0 + r) * DV, cb, c8);
 #pragma unroll
-            for (int c = 0; c < 8; c++) a[r][c] = __fmul_rn(c8[c], eta[r]);
-        }
+            for (int c = 0; c < 8; c++) ar[c] = __fmul_rn(c8[c], eta[r]);
+        };
         __syncthreads();                                   // ck, cq complete
 
         // the update: GDN e = v - r over the whole state; the new column
@@ -330,9 +336,12 @@ __global__ void __launch_bounds__(Geo<DK, DV>::NT, 1) lrb_kernel(const StepParam
 #pragma unroll
             for (int c = 0; c < 8; c++) pr[c] = 0.0f;
 #pragma unroll
-            for (int r = 0; r < 8; r++)
+            for (int r = 0; r < 8; r++) {
+                float ar[8];
+                arow(r, ar);
 #pragma unroll
-                for (int c = 0; c < 8; c++) pr[c] = __fmaf_rn(a[r][c], kk[r], pr[c]);
+                for (int c = 0; c < 8; c++) pr[c] = __fmaf_rn(ar[c], kk[r], pr[c]);
+            }
             float rr[8];
             colsum_finish<DK, DV>(pr, sh.red, sh.tot, warp, rbl, j0, rr);
             for (int l = 0; l < n; l++) {
@@ -369,9 +378,12 @@ __global__ void __launch_bounds__(Geo<DK, DV>::NT, 1) lrb_kernel(const StepParam
 #pragma unroll
             for (int c = 0; c < 8; c++) po[c] = 0.0f;
 #pragma unroll
-            for (int r = 0; r < 8; r++)
+            for (int r = 0; r < 8; r++) {
+                float ar[8];
+                arow(r, ar);
 #pragma unroll
-                for (int c = 0; c < 8; c++) po[c] = __fmaf_rn(a[r][c], qq[r], po[c]);
+                for (int c = 0; c < 8; c++) po[c] = __fmaf_rn(ar[c], qq[r], po[c]);
+            }
             float oo[8];
             colsum_finish<DK, DV>(po, sh.red, sh.tot, warp, rbl, j0, oo);    // syncs: cq[n] visible
             for (int l = 0; l < n; l++) {
@@ -400,10 +412,11 @@ __global__ void __launch_bounds__(Geo<DK, DV>::NT, 1) lrb_kernel(const StepParam
             continue;
         }
 
-        // ---- merge: the dense bypass, the threshold, requantization
+        // ---- merge: the dense bypass, the threshold, requantization (x is
+        // formed in place of the bypass block P)
         float x[8][8];
         {
-            float P[8][8];
+            auto& P = x;
 #pragma unroll
             for (int r = 0; r < 8; r++)
 #pragma unroll
@@ -424,15 +437,18 @@ __global__ void __launch_bounds__(Geo<DK, DV>::NT, 1) lrb_kernel(const StepParam
 #pragma unroll
             for (int r = 0; r < 8; r++) {
                 const float thr = __fmul_rn(L.eps_l, eta[r]);
+                float ar[8];
+                arow(r, ar);
 #pragma unroll
                 for (int c = 0; c < 8; c++) {
-                    const bool mg = fabsf(P[r][c]) >= thr;
-                    x[r][c] = mg ? __fadd_rn(a[r][c], P[r][c]) : a[r][c];
-                    if (L.k == 1) resid[(r * 8 + c) * G::NT + threadIdx.x] = mg ? 0.0f : P[r][c];
+                    const float pc = P[r][c];
+                    const bool mg = fabsf(pc) >= thr;
+                    if (L.k == 1) resid[(r * 8 + c) * G::NT + threadIdx.x] = mg ? 0.0f : pc;
+                    x[r][c] = mg ? __fadd_rn(ar[c], pc) : ar[c];
                 }
             }
         }
-        requantize<DK, DV, BITS, BDR>(p, sh.xs, sh.sprev, sbase, ct, a, x, lane, warp, cb, i0, ng,
+        requantize<DK, DV, BITS, BDR>(p, sh.xs, sh.sprev, sbase, ct, arow, x, lane, warp, cb, i0, ng,
                                       gcol);
 
         // the unmerged rest: its leading singular pair (k = 1) or nothing

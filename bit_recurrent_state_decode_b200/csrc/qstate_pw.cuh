@@ -56,8 +56,10 @@ struct __align__(16) PwShared {
     __align__(16) uint8_t sb[kPwMaxW * DV];    // value sides by slot
 };
 
+// Two CTAs per SM: the decayed history a is re-derived from the codes (an L1
+// hit after the first read) wherever the step needs it.
 template <int DK, int DV, int BITS, bool BDR, bool BF>
-__global__ void __launch_bounds__(Geo<DK, DV>::NT, 1) pw_kernel(const StepParams p, const PwParams P) {
+__global__ void __launch_bounds__(Geo<DK, DV>::NT, 2) pw_kernel(const StepParams p, const PwParams P) {
     using G = Geo<DK, DV>;
     static_assert(DK == DV, "square tiles");
     static_assert(BITS == 4 || BITS == 8, "4- or 8-bit codes");
@@ -151,31 +153,34 @@ __global__ void __launch_bounds__(Geo<DK, DV>::NT, 1) pw_kernel(const StepParams
             qq[r] = qval(i0 + r);
             eta[r] = __fmul_rn(alpha, prev_scale(group ? (i0 + r) * ng + gcol : 0));
         }
-        float a[8][8];
-#pragma unroll
-        for (int r = 0; r < 8; r++) {
+        auto arow = [&](int r, float (&ar)[8]) {
             float c8[8];
             if constexpr (BITS == 4) Decode<4>::run(ct + (i0 + r) * (DV / 2), cb, c8);
             else Decode<8>::run(ct + (i0 + r) * DV, cb, c8);
 #pragma unroll
-            for (int c = 0; c < 8; c++) a[r][c] = __fmul_rn(c8[c], eta[r]);
-        }
+            for (int c = 0; c < 8; c++) ar[c] = __fmul_rn(c8[c], eta[r]);
+        };
         float x[8][8];
         {
             float pr[8];
 #pragma unroll
             for (int c = 0; c < 8; c++) pr[c] = 0.0f;
 #pragma unroll
-            for (int r = 0; r < 8; r++)
+            for (int r = 0; r < 8; r++) {
+                float ar[8];
+                arow(r, ar);
 #pragma unroll
-                for (int c = 0; c < 8; c++) pr[c] = __fmaf_rn(a[r][c], kk[r], pr[c]);
+                for (int c = 0; c < 8; c++) pr[c] = __fmaf_rn(ar[c], kk[r], pr[c]);
+            }
             float rr[8];
             colsum_finish<DK, DV>(pr, sh.red, sh.tot, warp, rbl, j0, rr);    // syncs: pairs propagated
 #pragma unroll
             for (int r = 0; r < 8; r++) {
                 const float kap = __fmul_rn(beta, kk[r]);
+                float ar[8];
+                arow(r, ar);
 #pragma unroll
-                for (int c = 0; c < 8; c++) x[r][c] = __fmaf_rn(kap, -rr[c], a[r][c]);
+                for (int c = 0; c < 8; c++) x[r][c] = __fmaf_rn(kap, -rr[c], ar[c]);
             }
         }
         // the oldest pair leaves a full window into the history
@@ -247,7 +252,7 @@ __global__ void __launch_bounds__(Geo<DK, DV>::NT, 1) pw_kernel(const StepParams
         }
 
         // the history requantized
-        requantize<DK, DV, BITS, BDR>(p, sh.xs, sh.sprev, sbase, ct, a, x, lane, warp, cb, i0, ng,
+        requantize<DK, DV, BITS, BDR>(p, sh.xs, sh.sprev, sbase, ct, arow, x, lane, warp, cb, i0, ng,
                                       gcol);
         __syncthreads();
     }

@@ -23,7 +23,7 @@ struct __align__(16) RcShared {
     using G = Geo<DK, DV>;
     float red[G::NWARPS * DV];
     float tot[DV];
-    float rho[DK];                   // the previous row scales
+    float rho[DK];                   // alpha_i * the previous row scale
     float kap[DV];                   // the previous column scales
     int bad;
 };
@@ -56,8 +56,11 @@ __device__ __forceinline__ void colmax_finish(float (&p)[8], float* red, float* 
     for (int c = 0; c < 8; c++) res[c] = tot[j0 + c];
 }
 
+// Two CTAs per SM: only the updated state x stays in registers; the decayed
+// state a is re-derived from the codes (an L1 hit after the first read)
+// wherever a step needs it.
 template <int DK, int DV, int BITS, bool GDN, bool BDR, bool BF>
-__global__ void __launch_bounds__(Geo<DK, DV>::NT, 1) rc_kernel(const StepParams p) {
+__global__ void __launch_bounds__(Geo<DK, DV>::NT, 2) rc_kernel(const StepParams p) {
     using G = Geo<DK, DV>;
     static_assert(BITS == 4 || BITS == 8, "4- or 8-bit codes");
     constexpr int QMAX = (1 << (BITS - 1)) - 1;
@@ -90,66 +93,63 @@ __global__ void __launch_bounds__(Geo<DK, DV>::NT, 1) rc_kernel(const StepParams
         }
         for (int i = threadIdx.x; i < DK + DV; i += G::NT) {
             const float s = scale_at(p.scales, sbase + i, sf32);
-            if (i < DK) sh.rho[i] = s;
-            else sh.kap[i - DK] = s;
+            if (i < DK) {
+                const float al = p.kind == K_RETNET ? p.gamma
+                               : p.kind == K_GLA    ? ldg1(p.gates, tile * p.n_gate + i, p.gate_bf16 != 0)
+                                                    : ldg1(p.gates, tile * p.n_gate, p.gate_bf16 != 0);
+                sh.rho[i] = __fmul_rn(al, s);            // alpha_i * rho_i
+            } else {
+                sh.kap[i - DK] = s;
+            }
         }
         if (threadIdx.x == 0) sh.bad = 0;
         const uint8_t* kin = static_cast<const uint8_t*>(p.k) + tile * DK * isz;
         const uint8_t* qin = static_cast<const uint8_t*>(p.q) + tile * DK * isz;
         const uint8_t* vin = static_cast<const uint8_t*>(p.v) + tile * DV * isz;
-        float kk[8], qq[8], vv[8], al[8];
+        float kk[8];
 #pragma unroll
-        for (int r = 0; r < 8; r++) {
-            kk[r] = ldg1(kin, i0 + r, BF);
-            qq[r] = ldg1(qin, i0 + r, BF);
-            al[r] = p.kind == K_RETNET ? p.gamma
-                  : p.kind == K_GLA    ? ldg1(p.gates, tile * p.n_gate + i0 + r, p.gate_bf16 != 0)
-                                       : ldg1(p.gates, tile * p.n_gate, p.gate_bf16 != 0);
-        }
-#pragma unroll
-        for (int c = 0; c < 8; c++) vv[c] = ldg1(vin, j0 + c, BF);
+        for (int r = 0; r < 8; r++) kk[r] = ldg1(kin, i0 + r, BF);
         const float beta = GDN ? ldg1(p.gates, tile * p.n_gate + 1, p.gate_bf16 != 0) : 0.0f;
         __syncthreads();
 
-        // the decayed state: a = code * ((alpha_i * rho_i) * kappa_j)
-        float a[8][8];
-        {
-            float kp[8];
+        // a_ij = code * ((alpha_i * rho_i) * kappa_j) of row r of this thread
+        auto decayed_row = [&](int r, float (&ar)[8]) {
+            float c8[8];
+            if constexpr (BITS == 4) Decode<4>::run(ct + (i0 + r) * (DV / 2), cb, c8);
+            else Decode<8>::run(ct + (i0 + r) * DV, cb, c8);
+            const float arho = sh.rho[i0 + r];
 #pragma unroll
-            for (int c = 0; c < 8; c++) kp[c] = sh.kap[j0 + c];
-#pragma unroll
-            for (int r = 0; r < 8; r++) {
-                float c8[8];
-                if constexpr (BITS == 4) Decode<4>::run(ct + (i0 + r) * (DV / 2), cb, c8);
-                else Decode<8>::run(ct + (i0 + r) * DV, cb, c8);
-                const float ar = __fmul_rn(al[r], sh.rho[i0 + r]);
-#pragma unroll
-                for (int c = 0; c < 8; c++) a[r][c] = __fmul_rn(c8[c], __fmul_rn(ar, kp[c]));
-            }
-        }
+            for (int c = 0; c < 8; c++) ar[c] = __fmul_rn(c8[c], __fmul_rn(arho, sh.kap[j0 + c]));
+        };
         // the update
         float x[8][8];
+        float e[8];
         if constexpr (GDN) {
             float pr[8];
 #pragma unroll
             for (int c = 0; c < 8; c++) pr[c] = 0.0f;
 #pragma unroll
-            for (int r = 0; r < 8; r++)
+            for (int r = 0; r < 8; r++) {
+                float ar[8];
+                decayed_row(r, ar);
 #pragma unroll
-                for (int c = 0; c < 8; c++) pr[c] = __fmaf_rn(a[r][c], kk[r], pr[c]);
+                for (int c = 0; c < 8; c++) pr[c] = __fmaf_rn(ar[c], kk[r], pr[c]);
+            }
             float rr[8];
             colsum_finish<DK, DV>(pr, sh.red, sh.tot, warp, rbl, j0, rr);
 #pragma unroll
-            for (int r = 0; r < 8; r++) {
-                const float kap = __fmul_rn(beta, kk[r]);
-#pragma unroll
-                for (int c = 0; c < 8; c++) x[r][c] = __fmaf_rn(kap, __fsub_rn(vv[c], rr[c]), a[r][c]);
-            }
+            for (int c = 0; c < 8; c++) e[c] = __fsub_rn(ldg1(vin, j0 + c, BF), rr[c]);
         } else {
 #pragma unroll
-            for (int r = 0; r < 8; r++)
+            for (int c = 0; c < 8; c++) e[c] = ldg1(vin, j0 + c, BF);
+        }
 #pragma unroll
-                for (int c = 0; c < 8; c++) x[r][c] = __fmaf_rn(kk[r], vv[c], a[r][c]);
+        for (int r = 0; r < 8; r++) {
+            float ar[8];
+            decayed_row(r, ar);
+            const float kr = GDN ? __fmul_rn(beta, kk[r]) : kk[r];
+#pragma unroll
+            for (int c = 0; c < 8; c++) x[r][c] = __fmaf_rn(kr, e[c], ar[c]);
         }
         // the output from the state before rounding
         bool bad = false;
@@ -158,9 +158,11 @@ __global__ void __launch_bounds__(Geo<DK, DV>::NT, 1) rc_kernel(const StepParams
 #pragma unroll
             for (int c = 0; c < 8; c++) po[c] = 0.0f;
 #pragma unroll
-            for (int r = 0; r < 8; r++)
+            for (int r = 0; r < 8; r++) {
+                const float qr = ldg1(qin, i0 + r, BF);
 #pragma unroll
-                for (int c = 0; c < 8; c++) po[c] = __fmaf_rn(x[r][c], qq[r], po[c]);
+                for (int c = 0; c < 8; c++) po[c] = __fmaf_rn(x[r][c], qr, po[c]);
+            }
             float oo[8];
             colsum_finish<DK, DV>(po, sh.red, sh.tot, warp, rbl, j0, oo);
             if (rbl == 0 && warp == 0) {
@@ -199,8 +201,8 @@ __global__ void __launch_bounds__(Geo<DK, DV>::NT, 1) rc_kernel(const StepParams
                 }
             }
         }
-        // the row scales from the column-normalised magnitudes
-        float ir[8];
+        // row by row: the row scale from the column-normalised magnitudes, then
+        // round (BDR: a reversed element moves one code toward its update) and pack
 #pragma unroll
         for (int r = 0; r < 8; r++) {
             float t = 0.0f;
@@ -210,32 +212,30 @@ __global__ void __launch_bounds__(Geo<DK, DV>::NT, 1) rc_kernel(const StepParams
             for (int off = 1; off < G::CBW; off <<= 1) t = fmaxf(t, __shfl_xor_sync(0xFFFFFFFFu, t, off));
             bool sat = false;
             const float rho = to_stored(div_by_qmax(t, fq, rq), sf32, sat);
-            ir[r] = rho == 0.0f ? 0.0f : __frcp_rn(rho);
+            const float ir = rho == 0.0f ? 0.0f : __frcp_rn(rho);
             if (cb == 0) {
                 store_scale(p.scales, sbase + i0 + r, sf32, rho);
                 nsat += sat ? 1u : 0u;
             }
-        }
-        if (nsat) atomicAdd(p.counters + 1, (unsigned long long)nsat);
-        if (bad) sh.bad = 1;
-        // round (BDR: a reversed element moves one code toward its update) and pack
-#pragma unroll
-        for (int r = 0; r < 8; r++) {
+            float ar[8];
+            if (BDR) decayed_row(r, ar);
             float t8[8];
 #pragma unroll
             for (int c = 0; c < 8; c++) {
-                const float inv = __fmul_rn(ir[r], ik[c]);
-                float t = fminf(fmaxf(__fmaf_rn(x[r][c], inv, kMagic), kMagic - fq), kMagic + fq);
+                const float inv = __fmul_rn(ir, ik[c]);
+                float tc = fminf(fmaxf(__fmaf_rn(x[r][c], inv, kMagic), kMagic - fq), kMagic + fq);
                 if (BDR) {
-                    const float d = __fsub_rn(x[r][c], a[r][c]);
-                    const float s = __fmaf_rn(a[r][c], inv, -__fsub_rn(t, kMagic));
-                    if (d > 0.0f && s > p.eps_b) t = fminf(__fadd_rn(t, 1.0f), kMagic + fq);
-                    else if (d < 0.0f && s < -p.eps_b) t = fmaxf(__fsub_rn(t, 1.0f), kMagic - fq);
+                    const float d = __fsub_rn(x[r][c], ar[c]);
+                    const float s = __fmaf_rn(ar[c], inv, -__fsub_rn(tc, kMagic));
+                    if (d > 0.0f && s > p.eps_b) tc = fminf(__fadd_rn(tc, 1.0f), kMagic + fq);
+                    else if (d < 0.0f && s < -p.eps_b) tc = fmaxf(__fsub_rn(tc, 1.0f), kMagic - fq);
                 }
-                t8[c] = t;
+                t8[c] = tc;
             }
             pack_row<DK, DV, BITS>(ct, i0 + r, cb, t8);
         }
+        if (nsat) atomicAdd(p.counters + 1, (unsigned long long)nsat);
+        if (bad) sh.bad = 1;
         __syncthreads();
         if (threadIdx.x == 0 && sh.bad) atomicAdd(p.counters, 1ull);
     }
