@@ -45,6 +45,18 @@ __device__ __forceinline__ float h2f(uint16_t h) { return __half2float(__ushort_
 __device__ __forceinline__ uint16_t f2h(float x) { return __half_as_ushort(__float2half_rn(x)); }
 __device__ __forceinline__ float f16r(float x) { return __half2float(__float2half_rn(x)); }
 
+// Eight consecutive binary16 values (16-byte aligned) as binary32
+__device__ __forceinline__ void h8(const uint16_t* p, float (&v)[8]) {
+    const uint4 u = *reinterpret_cast<const uint4*>(p);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[i]));
+        v[2 * i] = f.x;
+        v[2 * i + 1] = f.y;
+    }
+}
+
 // Canonical sum over i < DK of x_i y_i (blocks of 8 rows, ascending fma from
 // +0, then the adjacent-pairs tree), by one warp: lane b < DK/8 sums block b,
 // the xor butterfly over those lanes is the tree, and lane 0's total goes to
@@ -104,15 +116,21 @@ __device__ __forceinline__ void round_pack_ax(ARow arow, const float (&x)[8][8],
         float ar[8];
         if (BDR) arow(r, ar);
 #pragma unroll
-        for (int c = 0; c < 8; c++) {
-            float t = fminf(fmaxf(__fmaf_rn(x[r][c], inv[r], kMagic), kMagic - fq), kMagic + fq);
+        for (int c = 0; c < 8; c += 2) {
+            const float2 x2 = f2(x[r][c], x[r][c + 1]);
+            float2 t2 = rtn2(x2, inv[r]);
+            t2.x = fminf(fmaxf(t2.x, kMagic - fq), kMagic + fq);
+            t2.y = fminf(fmaxf(t2.y, kMagic - fq), kMagic + fq);
             if (BDR) {
-                const float d = __fsub_rn(x[r][c], ar[c]);
-                const float s = __fmaf_rn(ar[c], inv[r], -__fsub_rn(t, kMagic));
-                if (d > 0.0f && s > eps_b) t = fminf(__fadd_rn(t, 1.0f), kMagic + fq);
-                else if (d < 0.0f && s < -eps_b) t = fmaxf(__fsub_rn(t, 1.0f), kMagic - fq);
+                const float2 a2 = f2(ar[c], ar[c + 1]);
+                const float2 d2 = ffma2(a2, f2(-1.0f, -1.0f), x2);                  // x - a
+                const float2 cn = ffma2(t2, f2(-1.0f, -1.0f), f2(kMagic, kMagic));  // -code
+                const float2 s2 = ffma2(a2, f2(inv[r], inv[r]), cn);
+                t2.x = fminf(fmaxf(bdr1(t2.x, s2.x, d2.x, eps_b), kMagic - fq), kMagic + fq);
+                t2.y = fminf(fmaxf(bdr1(t2.y, s2.y, d2.y, eps_b), kMagic - fq), kMagic + fq);
             }
-            t8[c] = t;
+            t8[c] = t2.x;
+            t8[c + 1] = t2.y;
         }
         pack_row<DK, DV, BITS>(ct, i0 + r, cb, t8);
     }
@@ -325,7 +343,11 @@ __global__ void __launch_bounds__(Geo<DK, DV>::NT, 2) lrb_kernel(const StepParam
             if constexpr (BITS == 4) Decode<4>::run(ct + (i0 + r) * (DV / 2), cb, c8);
             else Decode<8>::run(ct + (i0 + r) * DV, cb, c8);
 #pragma unroll
-            for (int c = 0; c < 8; c++) ar[c] = __fmul_rn(c8[c], eta[r]);
+            for (int c = 0; c < 8; c += 2) {
+                const float2 a2 = fmul2(f2(c8[c], c8[c + 1]), f2(eta[r], eta[r]));
+                ar[c] = a2.x;
+                ar[c + 1] = a2.y;
+            }
         };
         __syncthreads();                                   // ck, cq complete
 
@@ -340,13 +362,24 @@ __global__ void __launch_bounds__(Geo<DK, DV>::NT, 2) lrb_kernel(const StepParam
                 float ar[8];
                 arow(r, ar);
 #pragma unroll
-                for (int c = 0; c < 8; c++) pr[c] = __fmaf_rn(ar[c], kk[r], pr[c]);
+                for (int c = 0; c < 8; c += 2) {
+                    const float2 p2 = ffma2(f2(ar[c], ar[c + 1]), f2(kk[r], kk[r]), f2(pr[c], pr[c + 1]));
+                    pr[c] = p2.x;
+                    pr[c + 1] = p2.y;
+                }
             }
             float rr[8];
             colsum_finish<DK, DV>(pr, sh.red, sh.tot, warp, rbl, j0, rr);
             for (int l = 0; l < n; l++) {
+                float w8[8];
+                h8(sh.wcol + l * DV + j0, w8);
+                const float cl = sh.ck[l];
 #pragma unroll
-                for (int c = 0; c < 8; c++) rr[c] = __fmaf_rn(sh.ck[l], h2f(sh.wcol[l * DV + j0 + c]), rr[c]);
+                for (int c = 0; c < 8; c += 2) {
+                    const float2 r2 = ffma2(f2(cl, cl), f2(w8[c], w8[c + 1]), f2(rr[c], rr[c + 1]));
+                    rr[c] = r2.x;
+                    rr[c + 1] = r2.y;
+                }
             }
 #pragma unroll
             for (int c = 0; c < 8; c++) wn[c] = f16r(__fsub_rn(vv[c], rr[c]));
@@ -382,13 +415,24 @@ __global__ void __launch_bounds__(Geo<DK, DV>::NT, 2) lrb_kernel(const StepParam
                 float ar[8];
                 arow(r, ar);
 #pragma unroll
-                for (int c = 0; c < 8; c++) po[c] = __fmaf_rn(ar[c], qq[r], po[c]);
+                for (int c = 0; c < 8; c += 2) {
+                    const float2 p2 = ffma2(f2(ar[c], ar[c + 1]), f2(qq[r], qq[r]), f2(po[c], po[c + 1]));
+                    po[c] = p2.x;
+                    po[c + 1] = p2.y;
+                }
             }
             float oo[8];
             colsum_finish<DK, DV>(po, sh.red, sh.tot, warp, rbl, j0, oo);    // syncs: cq[n] visible
             for (int l = 0; l < n; l++) {
+                float w8[8];
+                h8(sh.wcol + l * DV + j0, w8);
+                const float cl = sh.cq[l];
 #pragma unroll
-                for (int c = 0; c < 8; c++) oo[c] = __fmaf_rn(sh.cq[l], h2f(sh.wcol[l * DV + j0 + c]), oo[c]);
+                for (int c = 0; c < 8; c += 2) {
+                    const float2 o2 = ffma2(f2(cl, cl), f2(w8[c], w8[c + 1]), f2(oo[c], oo[c + 1]));
+                    oo[c] = o2.x;
+                    oo[c + 1] = o2.y;
+                }
             }
 #pragma unroll
             for (int c = 0; c < 8; c++) oo[c] = __fmaf_rn(sh.cq[n], sh.wnew[j0 + c], oo[c]);
@@ -423,14 +467,25 @@ __global__ void __launch_bounds__(Geo<DK, DV>::NT, 2) lrb_kernel(const StepParam
                 for (int c = 0; c < 8; c++) P[r][c] = 0.0f;
             for (int l = 0; l <= n; l++) {
                 const float gl = sh.gco[l];
+                float u8[8], w8[8];
+                if (l < n) {
+                    h8(sh.ucol + l * DK + i0, u8);
+                    h8(sh.wcol + l * DV + j0, w8);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 8; i++) {
+                        u8[i] = sh.unew[i0 + i];
+                        w8[i] = sh.wnew[j0 + i];
+                    }
+                }
 #pragma unroll
                 for (int r = 0; r < 8; r++) {
-                    const float ul = l < n ? h2f(sh.ucol[l * DK + i0 + r]) : sh.unew[i0 + r];
-                    const float gu = __fmul_rn(gl, ul);
+                    const float gu = __fmul_rn(gl, u8[r]);
 #pragma unroll
-                    for (int c = 0; c < 8; c++) {
-                        const float wl = l < n ? h2f(sh.wcol[l * DV + j0 + c]) : sh.wnew[j0 + c];
-                        P[r][c] = __fmaf_rn(gu, wl, P[r][c]);
+                    for (int c = 0; c < 8; c += 2) {
+                        const float2 p2 = ffma2(f2(gu, gu), f2(w8[c], w8[c + 1]), f2(P[r][c], P[r][c + 1]));
+                        P[r][c] = p2.x;
+                        P[r][c + 1] = p2.y;
                     }
                 }
             }

@@ -158,29 +158,42 @@ __global__ void __launch_bounds__(Geo<DK, DV>::NT, 2) pw_kernel(const StepParams
             if constexpr (BITS == 4) Decode<4>::run(ct + (i0 + r) * (DV / 2), cb, c8);
             else Decode<8>::run(ct + (i0 + r) * DV, cb, c8);
 #pragma unroll
-            for (int c = 0; c < 8; c++) ar[c] = __fmul_rn(c8[c], eta[r]);
+            for (int c = 0; c < 8; c += 2) {
+                const float2 a2 = fmul2(f2(c8[c], c8[c + 1]), f2(eta[r], eta[r]));
+                ar[c] = a2.x;
+                ar[c + 1] = a2.y;
+            }
         };
         float x[8][8];
         {
-            float pr[8];
+            float2 pr[4];
 #pragma unroll
-            for (int c = 0; c < 8; c++) pr[c] = 0.0f;
+            for (int c = 0; c < 4; c++) pr[c] = f2(0.0f, 0.0f);
 #pragma unroll
             for (int r = 0; r < 8; r++) {
                 float ar[8];
                 arow(r, ar);
 #pragma unroll
-                for (int c = 0; c < 8; c++) pr[c] = __fmaf_rn(ar[c], kk[r], pr[c]);
+                for (int c = 0; c < 4; c++) pr[c] = ffma2(f2(ar[2 * c], ar[2 * c + 1]), f2(kk[r], kk[r]), pr[c]);
             }
-            float rr[8];
-            colsum_finish<DK, DV>(pr, sh.red, sh.tot, warp, rbl, j0, rr);    // syncs: pairs propagated
+            float p8[8], rr[8];
+#pragma unroll
+            for (int c = 0; c < 4; c++) {
+                p8[2 * c] = pr[c].x;
+                p8[2 * c + 1] = pr[c].y;
+            }
+            colsum_finish<DK, DV>(p8, sh.red, sh.tot, warp, rbl, j0, rr);    // syncs: pairs propagated
 #pragma unroll
             for (int r = 0; r < 8; r++) {
                 const float kap = __fmul_rn(beta, kk[r]);
                 float ar[8];
                 arow(r, ar);
 #pragma unroll
-                for (int c = 0; c < 8; c++) x[r][c] = __fmaf_rn(kap, -rr[c], ar[c]);
+                for (int c = 0; c < 8; c += 2) {
+                    const float2 x2 = ffma2(f2(kap, kap), f2(-rr[c], -rr[c + 1]), f2(ar[c], ar[c + 1]));
+                    x[r][c] = x2.x;
+                    x[r][c + 1] = x2.y;
+                }
             }
         }
         // the oldest pair leaves a full window into the history
@@ -198,7 +211,11 @@ __global__ void __launch_bounds__(Geo<DK, DV>::NT, 2) pw_kernel(const StepParams
             for (int r = 0; r < 8; r++) {
                 const float ao = e4m3_to_f32(a8[i0 + r]);
 #pragma unroll
-                for (int c = 0; c < 8; c++) x[r][c] = __fmaf_rn(ao, bo[c], x[r][c]);
+                for (int c = 0; c < 8; c += 2) {
+                    const float2 x2 = ffma2(f2(ao, ao), f2(bo[c], bo[c + 1]), f2(x[r][c], x[r][c + 1]));
+                    x[r][c] = x2.x;
+                    x[r][c + 1] = x2.y;
+                }
             }
         }
         __syncthreads();                                   // the leaver is read
@@ -218,14 +235,20 @@ __global__ void __launch_bounds__(Geo<DK, DV>::NT, 2) pw_kernel(const StepParams
 
         // the output: o = x^T q, then the pairs oldest first
         {
-            float po[8];
+            float2 po2[4];
 #pragma unroll
-            for (int c = 0; c < 8; c++) po[c] = 0.0f;
+            for (int c = 0; c < 4; c++) po2[c] = f2(0.0f, 0.0f);
 #pragma unroll
             for (int r = 0; r < 8; r++)
 #pragma unroll
-                for (int c = 0; c < 8; c++) po[c] = __fmaf_rn(x[r][c], qq[r], po[c]);
-            float oo[8];
+                for (int c = 0; c < 4; c++)
+                    po2[c] = ffma2(f2(x[r][2 * c], x[r][2 * c + 1]), f2(qq[r], qq[r]), po2[c]);
+            float po[8], oo[8];
+#pragma unroll
+            for (int c = 0; c < 4; c++) {
+                po[2 * c] = po2[c].x;
+                po[2 * c + 1] = po2[c].y;
+            }
             colsum_finish<DK, DV>(po, sh.red, sh.tot, warp, rbl, j0, oo);    // syncs: cq visible
             for (int l = 0; l < n2; l++) {
                 const uint8_t* b8 = sh.sb + ((h2 + l) % W) * DV;

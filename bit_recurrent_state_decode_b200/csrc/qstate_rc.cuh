@@ -112,6 +112,9 @@ __global__ void __launch_bounds__(Geo<DK, DV>::NT, 2) rc_kernel(const StepParams
         const float beta = GDN ? ldg1(p.gates, tile * p.n_gate + 1, p.gate_bf16 != 0) : 0.0f;
         __syncthreads();
 
+        float kp[8];
+#pragma unroll
+        for (int c = 0; c < 8; c++) kp[c] = sh.kap[j0 + c];
         // a_ij = code * ((alpha_i * rho_i) * kappa_j) of row r of this thread
         auto decayed_row = [&](int r, float (&ar)[8]) {
             float c8[8];
@@ -119,24 +122,33 @@ __global__ void __launch_bounds__(Geo<DK, DV>::NT, 2) rc_kernel(const StepParams
             else Decode<8>::run(ct + (i0 + r) * DV, cb, c8);
             const float arho = sh.rho[i0 + r];
 #pragma unroll
-            for (int c = 0; c < 8; c++) ar[c] = __fmul_rn(c8[c], __fmul_rn(arho, sh.kap[j0 + c]));
+            for (int c = 0; c < 8; c += 2) {
+                const float2 a2 = fmul2(f2(c8[c], c8[c + 1]), fmul2(f2(arho, arho), f2(kp[c], kp[c + 1])));
+                ar[c] = a2.x;
+                ar[c + 1] = a2.y;
+            }
         };
         // the update
         float x[8][8];
         float e[8];
         if constexpr (GDN) {
-            float pr[8];
+            float2 pr[4];
 #pragma unroll
-            for (int c = 0; c < 8; c++) pr[c] = 0.0f;
+            for (int c = 0; c < 4; c++) pr[c] = f2(0.0f, 0.0f);
 #pragma unroll
             for (int r = 0; r < 8; r++) {
                 float ar[8];
                 decayed_row(r, ar);
 #pragma unroll
-                for (int c = 0; c < 8; c++) pr[c] = __fmaf_rn(ar[c], kk[r], pr[c]);
+                for (int c = 0; c < 4; c++) pr[c] = ffma2(f2(ar[2 * c], ar[2 * c + 1]), f2(kk[r], kk[r]), pr[c]);
             }
-            float rr[8];
-            colsum_finish<DK, DV>(pr, sh.red, sh.tot, warp, rbl, j0, rr);
+            float p8[8], rr[8];
+#pragma unroll
+            for (int c = 0; c < 4; c++) {
+                p8[2 * c] = pr[c].x;
+                p8[2 * c + 1] = pr[c].y;
+            }
+            colsum_finish<DK, DV>(p8, sh.red, sh.tot, warp, rbl, j0, rr);
 #pragma unroll
             for (int c = 0; c < 8; c++) e[c] = __fsub_rn(ldg1(vin, j0 + c, BF), rr[c]);
         } else {
@@ -149,22 +161,31 @@ __global__ void __launch_bounds__(Geo<DK, DV>::NT, 2) rc_kernel(const StepParams
             decayed_row(r, ar);
             const float kr = GDN ? __fmul_rn(beta, kk[r]) : kk[r];
 #pragma unroll
-            for (int c = 0; c < 8; c++) x[r][c] = __fmaf_rn(kr, e[c], ar[c]);
+            for (int c = 0; c < 8; c += 2) {
+                const float2 x2 = ffma2(f2(kr, kr), f2(e[c], e[c + 1]), f2(ar[c], ar[c + 1]));
+                x[r][c] = x2.x;
+                x[r][c + 1] = x2.y;
+            }
         }
         // the output from the state before rounding
         bool bad = false;
         {
-            float po[8];
+            float2 po[4];
 #pragma unroll
-            for (int c = 0; c < 8; c++) po[c] = 0.0f;
+            for (int c = 0; c < 4; c++) po[c] = f2(0.0f, 0.0f);
 #pragma unroll
             for (int r = 0; r < 8; r++) {
                 const float qr = ldg1(qin, i0 + r, BF);
 #pragma unroll
-                for (int c = 0; c < 8; c++) po[c] = __fmaf_rn(x[r][c], qr, po[c]);
+                for (int c = 0; c < 4; c++) po[c] = ffma2(f2(x[r][2 * c], x[r][2 * c + 1]), f2(qr, qr), po[c]);
             }
-            float oo[8];
-            colsum_finish<DK, DV>(po, sh.red, sh.tot, warp, rbl, j0, oo);
+            float p8[8], oo[8];
+#pragma unroll
+            for (int c = 0; c < 4; c++) {
+                p8[2 * c] = po[c].x;
+                p8[2 * c + 1] = po[c].y;
+            }
+            colsum_finish<DK, DV>(p8, sh.red, sh.tot, warp, rbl, j0, oo);
             if (rbl == 0 && warp == 0) {
 #pragma unroll
                 for (int c = 0; c < 8; c++) {
@@ -180,14 +201,19 @@ __global__ void __launch_bounds__(Geo<DK, DV>::NT, 2) rc_kernel(const StepParams
             float m[8];
 #pragma unroll
             for (int c = 0; c < 8; c++) {
-                float t = 0.0f;
+                float t = fmaxf(fabsf(x[0][c]), fabsf(x[1][c]));
 #pragma unroll
-                for (int r = 0; r < 8; r++) {
-                    t = fmaxf(t, fabsf(x[r][c]));
-                    bad |= !isfinite(x[r][c]);
-                }
+                for (int r = 2; r < 8; r += 2) t = fmaxf(t, fmaxf(fabsf(x[r][c]), fabsf(x[r + 1][c])));
                 m[c] = t;
             }
+            // x * 0 is NaN exactly for a NaN or infinite x: one packed fma per
+            // pair finds any non-finite element of the block
+            float2 nf = f2(0.0f, 0.0f);
+#pragma unroll
+            for (int r = 0; r < 8; r++)
+#pragma unroll
+                for (int c = 0; c < 8; c += 2) nf = ffma2(f2(x[r][c], x[r][c + 1]), f2(0.0f, 0.0f), nf);
+            bad |= (nf.x != nf.x) || (nf.y != nf.y);
             float cm[8];
             colmax_finish<DK, DV>(m, sh.red, sh.tot, warp, rbl, j0, cm);
 #pragma unroll
@@ -203,11 +229,15 @@ __global__ void __launch_bounds__(Geo<DK, DV>::NT, 2) rc_kernel(const StepParams
         }
         // row by row: the row scale from the column-normalised magnitudes, then
         // round (BDR: a reversed element moves one code toward its update) and pack
+        constexpr float lo = kMagic - fq, hi = kMagic + fq;
 #pragma unroll
         for (int r = 0; r < 8; r++) {
             float t = 0.0f;
 #pragma unroll
-            for (int c = 0; c < 8; c++) t = fmaxf(t, __fmul_rn(fabsf(x[r][c]), ik[c]));
+            for (int c = 0; c < 8; c += 2) {
+                const float2 y2 = fmul2(f2(fabsf(x[r][c]), fabsf(x[r][c + 1])), f2(ik[c], ik[c + 1]));
+                t = fmaxf(t, fmaxf(y2.x, y2.y));
+            }
 #pragma unroll
             for (int off = 1; off < G::CBW; off <<= 1) t = fmaxf(t, __shfl_xor_sync(0xFFFFFFFFu, t, off));
             bool sat = false;
@@ -221,16 +251,22 @@ __global__ void __launch_bounds__(Geo<DK, DV>::NT, 2) rc_kernel(const StepParams
             if (BDR) decayed_row(r, ar);
             float t8[8];
 #pragma unroll
-            for (int c = 0; c < 8; c++) {
-                const float inv = __fmul_rn(ir, ik[c]);
-                float tc = fminf(fmaxf(__fmaf_rn(x[r][c], inv, kMagic), kMagic - fq), kMagic + fq);
+            for (int c = 0; c < 8; c += 2) {
+                const float2 inv2 = fmul2(f2(ir, ir), f2(ik[c], ik[c + 1]));
+                const float2 x2 = f2(x[r][c], x[r][c + 1]);
+                float2 t2 = ffma2(x2, inv2, f2(kMagic, kMagic));
+                t2.x = fminf(fmaxf(t2.x, lo), hi);
+                t2.y = fminf(fmaxf(t2.y, lo), hi);
                 if (BDR) {
-                    const float d = __fsub_rn(x[r][c], ar[c]);
-                    const float s = __fmaf_rn(ar[c], inv, -__fsub_rn(tc, kMagic));
-                    if (d > 0.0f && s > p.eps_b) tc = fminf(__fadd_rn(tc, 1.0f), kMagic + fq);
-                    else if (d < 0.0f && s < -p.eps_b) tc = fmaxf(__fsub_rn(tc, 1.0f), kMagic - fq);
+                    const float2 a2 = f2(ar[c], ar[c + 1]);
+                    const float2 d2 = ffma2(a2, f2(-1.0f, -1.0f), x2);                  // x - a
+                    const float2 cn = ffma2(t2, f2(-1.0f, -1.0f), f2(kMagic, kMagic));  // -code
+                    const float2 s2 = ffma2(a2, inv2, cn);
+                    t2.x = fminf(fmaxf(bdr1(t2.x, s2.x, d2.x, p.eps_b), lo), hi);
+                    t2.y = fminf(fmaxf(bdr1(t2.y, s2.y, d2.y, p.eps_b), lo), hi);
                 }
-                t8[c] = tc;
+                t8[c] = t2.x;
+                t8[c + 1] = t2.y;
             }
             pack_row<DK, DV, BITS>(ct, i0 + r, cb, t8);
         }
