@@ -69,6 +69,25 @@ const RcEntry* rc_table_64_128();
 const RcEntry* rc_table_128_64();
 const RcEntry* rc_table_128_128();
 
+// Launch a step kernel with programmatic stream serialization (the kernel
+// waits for the previous kernel of the stream before any global access, and
+// its prologue and scheduling overlap that kernel's tail).
+template <class K>
+inline void launch_pdl(K kernel, const StepParams& p, int grid, int threads, int dyn_smem,
+                       cudaStream_t st) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3((unsigned)threads);
+    cfg.dynamicSmemBytes = (size_t)dyn_smem;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    cudaLaunchKernelEx(&cfg, kernel, p);
+}
+
 // 0 = per-head widths, then 2, 4, 6, 8, 32 bits; -1 if invalid
 inline int bits_index(int bits) {
     switch (bits) {

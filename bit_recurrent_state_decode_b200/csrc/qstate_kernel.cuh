@@ -125,6 +125,17 @@ __device__ __forceinline__ uint32_t smem_addr(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// Programmatic dependent launch.  A step launched with programmatic stream
+// serialization may be scheduled while the previous kernel of its stream is
+// still running; griddepcontrol.wait returns once that kernel has completed
+// and its writes are visible (at once in a launch without the attribute), so
+// every global access of the step comes after it.  launch_dependents lets the
+// next such launch be scheduled onto SMs this grid no longer fills.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(smem_addr(bar)), "r"(count)
                  : "memory");
@@ -1292,6 +1303,8 @@ step_kernel(const StepParams p) {
         badf[0] = badf[1] = 0;
     }
     __syncthreads();
+    pdl_wait();
+    pdl_launch_dependents();
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; s++) {
             const long long t = blockIdx.x + (long long)s * gridDim.x;

@@ -93,6 +93,8 @@ __global__ void __launch_bounds__(RowsGeo<DK>::NT, 4) rows_kernel(const StepPara
         badf[0] = badf[1] = badf[2] = badf[3] = 0;
     }
     __syncthreads();
+    pdl_wait();
+    pdl_launch_dependents();
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; s++) {
             const long long t = blockIdx.x + (long long)s * gridDim.x;
