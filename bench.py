@@ -396,7 +396,7 @@ def run_ours(args, rank, world, local_rank):
     cold = footprint > 4 * props.L2_cache_size
     # DRAM traffic per launch from the committed ncu summary, scaled to this
     # launch by tiles (traffic grows in proportion once the launch is L2-cold)
-    traffic = read_traffic(wl0.name, T) if cold else None
+    traffic = read_traffic(wl0.name, T, kernel_name) if cold else None
     result = {
         "metric": "quantized state-updates/s",
         "value": world * T * K / (ms_total / 1e3),
@@ -437,10 +437,11 @@ def run_ours(args, rank, world, local_rank):
     return result
 
 
-def read_traffic(workload, tiles=None):
-    """DRAM bytes per launch from the committed ncu summary of this workload,
-    if its recorded kernel-source hash matches the current sources; scaled
-    from the summary's full-size launch to `tiles` tiles when given."""
+def read_traffic(workload, tiles=None, kernel="step_kernel"):
+    """DRAM bytes per launch from the committed ncu summary of this kernel on
+    this workload (profiles/<kernel>_<workload>.md), if its recorded
+    kernel-source hash matches the current sources; scaled from the
+    summary's full-size launch to `tiles` tiles when given."""
     import hashlib
     src = os.path.join(ROOT, "bit_recurrent_state_decode_b200", "csrc")
     h = hashlib.sha256()
@@ -449,7 +450,7 @@ def read_traffic(workload, tiles=None):
             with open(os.path.join(src, f), "rb") as fh:
                 h.update(fh.read())
     digest = h.hexdigest()[:16]
-    path = os.path.join(ROOT, "profiles", f"step_kernel_{workload}.md")
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
     if not os.path.exists(path):
         return None
     vals = {}

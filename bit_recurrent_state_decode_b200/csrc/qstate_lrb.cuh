@@ -275,8 +275,10 @@ __global__ void __launch_bounds__(Geo<DK, DV>::NT, 2) lrb_kernel(const StepParam
                 prefetch_l2<G::NT>(p.codes + nt * p.tile_bytes, p.tile_bytes);
                 prefetch_l2<G::NT>(static_cast<const uint8_t*>(p.scales) + nt * p.n_scales * ssz,
                                    (long long)p.n_scales * ssz);
-                prefetch_l2<G::NT>(L.u + nt * K * DK, (long long)K * DK * 2);
-                prefetch_l2<G::NT>(L.w + nt * K * DV, (long long)K * DV * 2);
+                // only the columns that tile holds (its counts: one cached line)
+                const int nn = L.n[2 * nt] + L.n[2 * nt + 1];
+                prefetch_l2<G::NT>(L.u + nt * K * DK, (long long)nn * DK * 2);
+                prefetch_l2<G::NT>(L.w + nt * K * DV, (long long)nn * DV * 2);
                 if (threadIdx.x == 0) {
                     asm volatile("prefetch.global.L2 [%0];" ::"l"(static_cast<const uint8_t*>(p.q) + nt * DK * isz));
                     asm volatile("prefetch.global.L2 [%0];" ::"l"(static_cast<const uint8_t*>(p.k) + nt * DK * isz));

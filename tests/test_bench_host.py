@@ -75,6 +75,6 @@ def test_committed_profiles_name_their_kernel_and_command():
     assert files
     for f in files:
         text = open(os.path.join(prof, f)).read()
-        assert f.startswith("step_kernel_")
+        assert f.split("_kernel_")[0] in ("step", "rows", "lrb", "pw", "rc"), f
         assert "source_sha256_16:" in text and "dram_bytes_per_launch_full_size:" in text
         assert "ncu " in text and "--clock-control none" in text and "python bench.py" in text
