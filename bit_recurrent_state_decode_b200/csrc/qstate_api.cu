@@ -68,6 +68,9 @@ struct qstate {
     long long drop_from = -1;
     // Low-Rank Bypass (qstate_set_lrb): bypass columns, coefficients, slot
     // counts and the decay since the last merge, per tile
+    // per key row the squared rounding error of the last step (allocated when
+    // the taxonomy is first switched on)
+    float* d_err = nullptr;
     bool lrb = false;
     int lrb_k = 0, lrb_m = 0;
     float lrb_eps = 0.0f;
@@ -154,6 +157,7 @@ qs::StepParams params_of(const qstate* s) {
     p.fast = s->import_pending ? 0 : 1;
     p.taxonomy = s->taxonomy ? 1 : 0;
     p.rotate = s->L.rotation;
+    p.err_rows = s->taxonomy ? s->d_err : nullptr;
     return p;
 }
 
@@ -172,6 +176,7 @@ void free_all(qstate* s) {
     cudaFree(s->st_v);
     cudaFree(s->st_g);
     cudaFree(s->st_out);
+    cudaFree(s->d_err);
     cudaFree(s->d_lu);
     cudaFree(s->d_lw);
     cudaFree(s->d_lg);
@@ -791,7 +796,26 @@ int qstate_status(qstate* s, qstate_counters* o, qstate_stream stream) {
 
 int qstate_set_taxonomy(qstate* s, int on) {
     if (!s || (on != 0 && on != 1)) return QSTATE_EINVAL;
+    if (on && !s->d_err && s->tiles > 0 && s->bits != 32) {
+        int rc = check_device(s);
+        if (rc != QSTATE_OK) return rc;
+        const size_t n = (size_t)s->tiles * s->L.d_k * sizeof(float);
+        if (cudaMalloc((void**)&s->d_err, n) != cudaSuccess) {
+            cudaGetLastError();
+            s->d_err = nullptr;
+            return QSTATE_ENOMEM;
+        }
+        if (cudaMemset(s->d_err, 0, n) != cudaSuccess) return QSTATE_ECUDA;
+    }
     s->taxonomy = on != 0;
+    return QSTATE_OK;
+}
+
+int qstate_error_rows(const qstate* s, float* out, qstate_stream stream) {
+    if (!s || !out || !s->d_err) return QSTATE_EINVAL;
+    const size_t n = (size_t)s->tiles * s->L.d_k * sizeof(float);
+    if (cudaMemcpyAsync(out, s->d_err, n, cudaMemcpyDefault, (cudaStream_t)stream) != cudaSuccess)
+        return QSTATE_ECUDA;
     return QSTATE_OK;
 }
 

@@ -99,6 +99,9 @@ struct StepParams {
     // 1: the state is kept rotated by the Hadamard matrix along d_v (the step
     // takes H v for v and emits H o_rot / d_v); 0: none
     int rotate;
+    // with the taxonomy on: [tiles][d_k], per key row the squared rounding
+    // error of the step, sum_j (S_hat_new - x)^2; null: not kept
+    float* err_rows;
 };
 
 constexpr int kNumCounters = 8;
@@ -738,11 +741,19 @@ __device__ __forceinline__ float rotate_out(float o, int j, float (*orot)[DV]) {
 template <int DK, int DV, int BITS, bool BDR, class URow>
 __device__ __forceinline__ void taxonomy_count(const StepParams& p, const uint8_t* st, int i0, int cb,
                                             const float (&eta)[8], URow urow,
-                                            const float (&wc)[8], const float (&inv)[8]) {
+                                            const float (&wc)[8], const float (&inv)[8],
+                                            long long tile, long long sbase, int ng, int gcol) {
     constexpr float fq = float((1 << (BITS - 1)) - 1);
+    using G = Geo<DK, DV>;
     unsigned nl = 0, nm = 0, nr = 0, nb = 0;
+    // the step's new scales, stored by other threads of the CTA
+    const bool energy = p.err_rows != nullptr;
+    if (energy) __syncthreads();
 #pragma unroll 1
     for (int r = 0; r < 8; r++) {
+        float dnew = 0.0f, e2 = 0.0f;
+        if (energy) dnew = scale_at(p.scales, p.group ? sbase + (i0 + r) * ng + gcol : sbase,
+                                    p.scale_f32 != 0);
         float c8[8];
         const uint8_t* srow = st + p.off_codes;
         if constexpr (BITS == 4) Decode<4>::run(srow + (i0 + r) * (DV / 2), cb, c8);
@@ -755,16 +766,30 @@ __device__ __forceinline__ void taxonomy_count(const StepParams& p, const uint8_
             const float a = __fmul_rn(c8[c], eta[r]);
             const float x = __fmaf_rn(ur, wc[c], a);
             const float d = __fsub_rn(x, a);
+            const float t = fminf(fmaxf(__fmaf_rn(x, inv[r], kMagic), kMagic - fq), kMagic + fq);
+            const float s = __fmaf_rn(a, inv[r], -__fsub_rn(t, kMagic));    // u - c
+            const bool bdr = BDR && ((d > 0.0f && s > p.eps_b) || (d < 0.0f && s < -p.eps_b));
             if (d != 0.0f) {
-                const float t = fminf(fmaxf(__fmaf_rn(x, inv[r], kMagic), kMagic - fq), kMagic + fq);
                 const float tu = fminf(fmaxf(__fmaf_rn(a, inv[r], kMagic), kMagic - fq), kMagic + fq);
-                const float s = __fmaf_rn(a, inv[r], -__fsub_rn(t, kMagic));    // u - c
                 const bool rev = (s > 0.0f && d > 0.0f) || (s < 0.0f && d < 0.0f);
                 nr += rev ? 1u : 0u;
                 nl += (!rev && t == tu) ? 1u : 0u;
                 nm += (!rev && t != tu) ? 1u : 0u;
-                if (BDR) nb += ((d > 0.0f && s > p.eps_b) || (d < 0.0f && s < -p.eps_b)) ? 1u : 0u;
+                nb += bdr ? 1u : 0u;
             }
+            if (energy) {
+                // the code stored: the RTN code, moved one step by BDR, clamped
+                const float tf = bdr ? fminf(fmaxf(__fadd_rn(t, d > 0.0f ? 1.0f : -1.0f), kMagic - fq),
+                                             kMagic + fq)
+                                     : t;
+                const float R = __fsub_rn(__fmul_rn(__fsub_rn(tf, kMagic), dnew), x);
+                e2 = __fmaf_rn(R, R, e2);
+            }
+        }
+        if (energy) {
+#pragma unroll
+            for (int off = 1; off < G::CBW; off <<= 1) e2 = __fadd_rn(e2, __shfl_xor_sync(0xFFFFFFFFu, e2, off));
+            if (cb == 0) p.err_rows[tile * DK + i0 + r] = e2;
         }
     }
     nl = __reduce_add_sync(0xFFFFFFFFu, nl);
@@ -1206,7 +1231,8 @@ __device__ __forceinline__ bool step_tile(const StepParams& p, long long tile, c
             float eta[8];
 #pragma unroll
             for (int r = 0; r < 8; r++) eta[r] = __fmul_rn(al[r], dprev[r]);
-            taxonomy_count<DK, DV, BITS, BDR>(p, st, i0, cb, eta, urow, wc, inv);
+            taxonomy_count<DK, DV, BITS, BDR>(p, st, i0, cb, eta, urow, wc, inv, tile, sbase, ng,
+                                              gcol);
         }
         // a tile-step is counted once if an output or a group maximum was not
         // finite (the flag is collected at the next tile's barrier)

@@ -27,7 +27,7 @@ EXPORTS = ("qstate_create", "qstate_destroy", "qstate_reset", "qstate_step", "qs
            "qstate_step_host_static", "qstate_dequant", "qstate_export", "qstate_import", "qstate_get_sizes",
            "qstate_bytes_per_step", "qstate_status", "qstate_set_taxonomy", "qstate_set_lrb",
            "qstate_lrb_export", "qstate_set_pw", "qstate_pw_export", "qstate_set_rowcol",
-           "qstate_kernel", "qstate_debug_set", "qstate_error_string")
+           "qstate_error_rows", "qstate_kernel", "qstate_debug_set", "qstate_error_string")
 
 
 class QStateError(RuntimeError):
@@ -89,6 +89,7 @@ def lib():
         L.qstate_set_pw.argtypes = [P, I]
         L.qstate_pw_export.argtypes = [P, P, P, P, P, S]
         L.qstate_set_rowcol.argtypes = [P]
+        L.qstate_error_rows.argtypes = [P, P, S]
         L.qstate_kernel.argtypes = [P]
         L.qstate_kernel.restype = ctypes.c_char_p
         L.qstate_error_string.argtypes = [I]
@@ -305,6 +306,13 @@ class QState:
     def kernel(self) -> str:
         """The kernel the next step launches (qstate_kernel)."""
         return lib().qstate_kernel(self._h).decode()
+
+    def error_rows(self, stream=None) -> torch.Tensor:
+        """Per tile and key row, the squared rounding error of the last step
+        taken with the taxonomy on (qstate_error_rows), [tiles, d_k]."""
+        out = torch.empty((self.tiles, self.d_k), dtype=torch.float32, device=f"cuda:{self.device}")
+        _check("qstate_error_rows", lib().qstate_error_rows(self._h, _ptr(out), _stream(stream)))
+        return out
 
     def set_rowcol(self):
         """Key-row x value-column scales (qstate_set_rowcol); before the

@@ -268,6 +268,19 @@ int qstate_status(qstate* s, qstate_counters* out, qstate_stream stream);
  * the state and outputs are unchanged.  QSTATE_EINVAL for other values. */
 int qstate_set_taxonomy(qstate* s, int on);
 
+/* With the taxonomy on, each step also keeps, per tile and key row, the
+ * squared rounding error it added, sum_j (S_hat_t - x_t)_ij^2 (S_hat_t the
+ * dequantized new state, x_t the updated state before rounding; binary32):
+ * the per-step R_t of the error accounting of "Preserving Updates in Low-Bit
+ * Recurrent State Quantization" (Figures 1 and 2, Table 5), from which a
+ * caller forms D_T = sum_t ||a_{t:T} R_t||^2 and the coherent gain.  Copies
+ * the last such step's values, [tiles][d_k] binary32, to `out` (device or
+ * host) on stream.  QSTATE_EINVAL if the taxonomy was never switched on
+ * (the buffer is allocated by the first qstate_set_taxonomy(s, 1), which may
+ * return QSTATE_ENOMEM).  Objects with a bypass, a window or row x column
+ * scales do not keep it. */
+int qstate_error_rows(const qstate* s, float* out, qstate_stream stream);
+
 /* Switch the object to steps with a Low-Rank Bypass (LRB) of "Preserving
  * Updates in Low-Bit Recurrent State Quantization" (Abstract, Figure 3,
  * Tables 6, 8, 9), before its first step.  Each tile keeps, next to its
