@@ -100,12 +100,22 @@ struct qstate {
     // imported state may hold the code -2^(bits-1), which no step produces)
     bool import_pending = false;
     qs::StepParams stage{};           // stage layout fields only
-    // staging buffers of qstate_step_host (allocated by its first call)
+    // staging buffers of qstate_step_host (allocated by its first call): the
+    // inputs in two sets used by alternate calls, copied on the object's own
+    // stream so that one call's copies overlap the previous call's step
     void* st_q = nullptr;
     void* st_k = nullptr;
     void* st_v = nullptr;
     void* st_g = nullptr;
     float* st_out = nullptr;
+    void* st2_q = nullptr;
+    void* st2_k = nullptr;
+    void* st2_v = nullptr;
+    void* st2_g = nullptr;
+    cudaStream_t h2d = nullptr;
+    cudaEvent_t copied[2] = {nullptr, nullptr};     // inputs of set b in device memory
+    cudaEvent_t consumed[2] = {nullptr, nullptr};   // the step reading set b has run
+    uint64_t host_calls = 0;
 };
 
 namespace {
@@ -176,6 +186,15 @@ void free_all(qstate* s) {
     cudaFree(s->st_v);
     cudaFree(s->st_g);
     cudaFree(s->st_out);
+    cudaFree(s->st2_q);
+    cudaFree(s->st2_k);
+    cudaFree(s->st2_v);
+    cudaFree(s->st2_g);
+    for (int b = 0; b < 2; b++) {
+        if (s->copied[b]) cudaEventDestroy(s->copied[b]);
+        if (s->consumed[b]) cudaEventDestroy(s->consumed[b]);
+    }
+    if (s->h2d) cudaStreamDestroy(s->h2d);
     cudaFree(s->d_err);
     cudaFree(s->d_lu);
     cudaFree(s->d_lw);
@@ -519,27 +538,57 @@ int qstate_step_host(qstate* s, const void* q, const void* k, const void* v, con
                   cudaMalloc(&s->st_k, z.q_bytes) == cudaSuccess &&
                   cudaMalloc(&s->st_v, z.v_bytes) == cudaSuccess &&
                   (!z.gate_bytes || cudaMalloc(&s->st_g, z.gate_bytes) == cudaSuccess) &&
-                  cudaMalloc((void**)&s->st_out, z.out_bytes) == cudaSuccess;
+                  cudaMalloc(&s->st2_q, z.q_bytes) == cudaSuccess &&
+                  cudaMalloc(&s->st2_k, z.q_bytes) == cudaSuccess &&
+                  cudaMalloc(&s->st2_v, z.v_bytes) == cudaSuccess &&
+                  (!z.gate_bytes || cudaMalloc(&s->st2_g, z.gate_bytes) == cudaSuccess) &&
+                  cudaMalloc((void**)&s->st_out, z.out_bytes) == cudaSuccess &&
+                  cudaStreamCreateWithFlags(&s->h2d, cudaStreamNonBlocking) == cudaSuccess;
+        for (int b = 0; ok && b < 2; b++)
+            ok = cudaEventCreateWithFlags(&s->copied[b], cudaEventDisableTiming) == cudaSuccess &&
+                 cudaEventCreateWithFlags(&s->consumed[b], cudaEventDisableTiming) == cudaSuccess;
         if (!ok) {
             cudaGetLastError();
             cudaFree(s->st_q); cudaFree(s->st_k); cudaFree(s->st_v);
             cudaFree(s->st_g); cudaFree(s->st_out);
+            cudaFree(s->st2_q); cudaFree(s->st2_k); cudaFree(s->st2_v); cudaFree(s->st2_g);
+            for (int b = 0; b < 2; b++) {
+                if (s->copied[b]) cudaEventDestroy(s->copied[b]);
+                if (s->consumed[b]) cudaEventDestroy(s->consumed[b]);
+                s->copied[b] = s->consumed[b] = nullptr;
+            }
+            if (s->h2d) cudaStreamDestroy(s->h2d);
+            s->h2d = nullptr;
             s->st_q = s->st_k = s->st_v = s->st_g = nullptr;
+            s->st2_q = s->st2_k = s->st2_v = s->st2_g = nullptr;
             s->st_out = nullptr;
             return QSTATE_ENOMEM;
         }
     }
     cudaStream_t st = (cudaStream_t)stream;
-    if (cudaMemcpyAsync(s->st_q, q, z.q_bytes, cudaMemcpyHostToDevice, st) != cudaSuccess ||
-        cudaMemcpyAsync(s->st_k, k, z.q_bytes, cudaMemcpyHostToDevice, st) != cudaSuccess ||
-        cudaMemcpyAsync(s->st_v, v, z.v_bytes, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+    const int b = (int)(s->host_calls & 1);
+    void* dq = b ? s->st2_q : s->st_q;
+    void* dk = b ? s->st2_k : s->st_k;
+    void* dv = b ? s->st2_v : s->st_v;
+    void* dg = b ? s->st2_g : s->st_g;
+    // the inputs of set b, on the object's copy stream, once the step that
+    // read set b two calls ago has run (and after the caller's earlier work
+    // on `stream` was issued: the copy stream waits for nothing else)
+    if (cudaStreamWaitEvent(s->h2d, s->consumed[b], 0) != cudaSuccess ||
+        cudaMemcpyAsync(dq, q, z.q_bytes, cudaMemcpyHostToDevice, s->h2d) != cudaSuccess ||
+        cudaMemcpyAsync(dk, k, z.q_bytes, cudaMemcpyHostToDevice, s->h2d) != cudaSuccess ||
+        cudaMemcpyAsync(dv, v, z.v_bytes, cudaMemcpyHostToDevice, s->h2d) != cudaSuccess ||
         (z.gate_bytes &&
-         cudaMemcpyAsync(s->st_g, gates, z.gate_bytes, cudaMemcpyHostToDevice, st) != cudaSuccess))
+         cudaMemcpyAsync(dg, gates, z.gate_bytes, cudaMemcpyHostToDevice, s->h2d) != cudaSuccess) ||
+        cudaEventRecord(s->copied[b], s->h2d) != cudaSuccess ||
+        cudaStreamWaitEvent(st, s->copied[b], 0) != cudaSuccess)
         return QSTATE_ECUDA;
-    rc = qstate_step(s, s->st_q, s->st_k, s->st_v, s->st_g, s->st_out, stream);
+    rc = qstate_step(s, dq, dk, dv, dg, s->st_out, stream);
     if (rc != QSTATE_OK) return rc;
-    if (cudaMemcpyAsync(out, s->st_out, z.out_bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    if (cudaEventRecord(s->consumed[b], st) != cudaSuccess ||
+        cudaMemcpyAsync(out, s->st_out, z.out_bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
         return QSTATE_ECUDA;
+    s->host_calls++;
     return QSTATE_OK;
 }
 

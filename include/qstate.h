@@ -190,12 +190,17 @@ int qstate_step(qstate* s, const void* q, const void* k, const void* v, const vo
                 float* out, qstate_stream stream);
 
 /* The same step from HOST buffers: copies q, k, v, gates host->device into
- * library-owned staging buffers, launches the step and copies out
- * device->host, all asynchronous on stream (synchronise the stream before
- * reading out).  Pinned host memory makes the copies asynchronous.  The
- * staging buffers are allocated by the first call and shared by every later
- * call on the object: issue all qstate_step_host calls of one object on one
- * stream (calls on different streams would overwrite each other's
+ * library-owned staging buffers, launches the step on stream and copies out
+ * device->host on stream, all asynchronous (synchronise the stream before
+ * reading out: its completion covers this call's copies and step).  The
+ * input copies run on a stream of the object's own, into one of two staging
+ * sets used by alternate calls, so that a call's input copies overlap the
+ * previous call's step; the step waits for them.  Pinned host memory makes
+ * the copies asynchronous; the caller keeps its input buffers unchanged
+ * until the stream has completed the call.  The staging buffers, the copy
+ * stream and its events are allocated by the first call and shared by every
+ * later call on the object: issue all qstate_step_host calls of one object
+ * on one stream (calls on different streams would overwrite each other's
  * operands). */
 int qstate_step_host(qstate* s, const void* q, const void* k, const void* v,
                      const void* gates, float* out, qstate_stream stream);
