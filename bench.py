@@ -364,20 +364,30 @@ def run_ours(args, rank, world, local_rank):
                                      else np.ascontiguousarray(a))
                 return t.pin_memory()
             pin.append((pinned(x.q), pinned(x.k), pinned(x.v), pinned(x.gates)))
-        hout = torch.empty((T, wl0.d_v), dtype=torch.float32).pin_memory()
+        # one pinned output per object and step parity (the output copies of
+        # consecutive calls are in flight together)
+        houts = [[torch.empty((T, wl0.d_v), dtype=torch.float32).pin_memory() for _ in range(2)]
+                 for _ in objs]
         h2d = sum(t.numel() * t.element_size() for t in pin[0] if t is not None)
-        d2h = hout.numel() * 4 * len(objs)
+        d2h = houts[0][0].numel() * 4 * len(objs)
         Ke = max(3, min(K, int(2.0 / max(est + (h2d + d2h) / 20e9, 1e-6))))
+        # the host-buffer calls of a stream of steps: each call's output copy
+        # overlaps the next call's step; the last one is waited for inside
+        # the timed region
         for i in range(2):
-            for o in objs:
-                o.step_host(*pin[i % len(pin)], hout, stream)
+            for o, ho in zip(objs, houts):
+                o.step_host_pipelined(*pin[i % len(pin)], ho[i & 1], stream)
+        for o in objs:
+            o.step_host_sync(stream)
         torch.cuda.synchronize()
         if dist:
             tdist.barrier()
         e0.record(stream)
         for i in range(Ke):
-            for o in objs:
-                o.step_host(*pin[i % len(pin)], hout, stream)
+            for o, ho in zip(objs, houts):
+                o.step_host_pipelined(*pin[i % len(pin)], ho[i & 1], stream)
+        for o in objs:
+            o.step_host_sync(stream)
         e1.record(stream)
         torch.cuda.synchronize()
         ems = max_over_ranks(e0.elapsed_time(e1), dev)

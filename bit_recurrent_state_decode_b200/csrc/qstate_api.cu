@@ -112,9 +112,12 @@ struct qstate {
     void* st2_k = nullptr;
     void* st2_v = nullptr;
     void* st2_g = nullptr;
+    float* st2_out = nullptr;
     cudaStream_t h2d = nullptr;
+    cudaStream_t d2h = nullptr;
     cudaEvent_t copied[2] = {nullptr, nullptr};     // inputs of set b in device memory
-    cudaEvent_t consumed[2] = {nullptr, nullptr};   // the step reading set b has run
+    cudaEvent_t consumed[2] = {nullptr, nullptr};   // the step of set b has run
+    cudaEvent_t delivered[2] = {nullptr, nullptr};  // the output of set b is in host memory
     uint64_t host_calls = 0;
 };
 
@@ -190,11 +193,14 @@ void free_all(qstate* s) {
     cudaFree(s->st2_k);
     cudaFree(s->st2_v);
     cudaFree(s->st2_g);
+    cudaFree(s->st2_out);
     for (int b = 0; b < 2; b++) {
         if (s->copied[b]) cudaEventDestroy(s->copied[b]);
         if (s->consumed[b]) cudaEventDestroy(s->consumed[b]);
+        if (s->delivered[b]) cudaEventDestroy(s->delivered[b]);
     }
     if (s->h2d) cudaStreamDestroy(s->h2d);
+    if (s->d2h) cudaStreamDestroy(s->d2h);
     cudaFree(s->d_err);
     cudaFree(s->d_lu);
     cudaFree(s->d_lw);
@@ -524,8 +530,20 @@ int qstate_get_sizes(const qstate* s, qstate_sizes* o) {
     return QSTATE_OK;
 }
 
-int qstate_step_host(qstate* s, const void* q, const void* k, const void* v, const void* gates,
-                     float* out, qstate_stream stream) {
+}  // extern "C"
+
+namespace {
+
+// The host-buffer step (qstate_step_host, qstate_step_host_pipelined): the
+// inputs and outputs in two staging sets used by alternate calls; the input
+// copies on the object's h2d stream, the output copy on its d2h stream, the
+// step on the caller's stream.  Each copy waits only for what it reads or
+// overwrites: the inputs of set b for the step two calls back (which read
+// them), the step for the output copy two calls back (which read set b's
+// output).  sync_out: the caller's stream also waits for this call's output
+// copy (else for the previous call's).
+int step_host_impl(qstate* s, const void* q, const void* k, const void* v, const void* gates,
+                   float* out, cudaStream_t st, bool sync_out) {
     if (!s || !q || !k || !v || !out) return QSTATE_EINVAL;
     if (s->n_gate && !gates) return QSTATE_EINVAL;
     if (s->tiles == 0) return QSTATE_OK;
@@ -543,37 +561,40 @@ int qstate_step_host(qstate* s, const void* q, const void* k, const void* v, con
                   cudaMalloc(&s->st2_v, z.v_bytes) == cudaSuccess &&
                   (!z.gate_bytes || cudaMalloc(&s->st2_g, z.gate_bytes) == cudaSuccess) &&
                   cudaMalloc((void**)&s->st_out, z.out_bytes) == cudaSuccess &&
-                  cudaStreamCreateWithFlags(&s->h2d, cudaStreamNonBlocking) == cudaSuccess;
+                  cudaMalloc((void**)&s->st2_out, z.out_bytes) == cudaSuccess &&
+                  cudaStreamCreateWithFlags(&s->h2d, cudaStreamNonBlocking) == cudaSuccess &&
+                  cudaStreamCreateWithFlags(&s->d2h, cudaStreamNonBlocking) == cudaSuccess;
         for (int b = 0; ok && b < 2; b++)
             ok = cudaEventCreateWithFlags(&s->copied[b], cudaEventDisableTiming) == cudaSuccess &&
-                 cudaEventCreateWithFlags(&s->consumed[b], cudaEventDisableTiming) == cudaSuccess;
+                 cudaEventCreateWithFlags(&s->consumed[b], cudaEventDisableTiming) == cudaSuccess &&
+                 cudaEventCreateWithFlags(&s->delivered[b], cudaEventDisableTiming) == cudaSuccess;
         if (!ok) {
             cudaGetLastError();
             cudaFree(s->st_q); cudaFree(s->st_k); cudaFree(s->st_v);
             cudaFree(s->st_g); cudaFree(s->st_out);
             cudaFree(s->st2_q); cudaFree(s->st2_k); cudaFree(s->st2_v); cudaFree(s->st2_g);
+            cudaFree(s->st2_out);
             for (int b = 0; b < 2; b++) {
                 if (s->copied[b]) cudaEventDestroy(s->copied[b]);
                 if (s->consumed[b]) cudaEventDestroy(s->consumed[b]);
-                s->copied[b] = s->consumed[b] = nullptr;
+                if (s->delivered[b]) cudaEventDestroy(s->delivered[b]);
+                s->copied[b] = s->consumed[b] = s->delivered[b] = nullptr;
             }
             if (s->h2d) cudaStreamDestroy(s->h2d);
-            s->h2d = nullptr;
+            if (s->d2h) cudaStreamDestroy(s->d2h);
+            s->h2d = s->d2h = nullptr;
             s->st_q = s->st_k = s->st_v = s->st_g = nullptr;
             s->st2_q = s->st2_k = s->st2_v = s->st2_g = nullptr;
-            s->st_out = nullptr;
+            s->st_out = s->st2_out = nullptr;
             return QSTATE_ENOMEM;
         }
     }
-    cudaStream_t st = (cudaStream_t)stream;
     const int b = (int)(s->host_calls & 1);
     void* dq = b ? s->st2_q : s->st_q;
     void* dk = b ? s->st2_k : s->st_k;
     void* dv = b ? s->st2_v : s->st_v;
     void* dg = b ? s->st2_g : s->st_g;
-    // the inputs of set b, on the object's copy stream, once the step that
-    // read set b two calls ago has run (and after the caller's earlier work
-    // on `stream` was issued: the copy stream waits for nothing else)
+    float* dout = b ? s->st2_out : s->st_out;
     if (cudaStreamWaitEvent(s->h2d, s->consumed[b], 0) != cudaSuccess ||
         cudaMemcpyAsync(dq, q, z.q_bytes, cudaMemcpyHostToDevice, s->h2d) != cudaSuccess ||
         cudaMemcpyAsync(dk, k, z.q_bytes, cudaMemcpyHostToDevice, s->h2d) != cudaSuccess ||
@@ -581,15 +602,41 @@ int qstate_step_host(qstate* s, const void* q, const void* k, const void* v, con
         (z.gate_bytes &&
          cudaMemcpyAsync(dg, gates, z.gate_bytes, cudaMemcpyHostToDevice, s->h2d) != cudaSuccess) ||
         cudaEventRecord(s->copied[b], s->h2d) != cudaSuccess ||
-        cudaStreamWaitEvent(st, s->copied[b], 0) != cudaSuccess)
+        cudaStreamWaitEvent(st, s->copied[b], 0) != cudaSuccess ||
+        cudaStreamWaitEvent(st, s->delivered[b], 0) != cudaSuccess)
         return QSTATE_ECUDA;
-    rc = qstate_step(s, dq, dk, dv, dg, s->st_out, stream);
+    rc = qstate_step(s, dq, dk, dv, dg, dout, (qstate_stream)st);
     if (rc != QSTATE_OK) return rc;
     if (cudaEventRecord(s->consumed[b], st) != cudaSuccess ||
-        cudaMemcpyAsync(out, s->st_out, z.out_bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        cudaStreamWaitEvent(s->d2h, s->consumed[b], 0) != cudaSuccess ||
+        cudaMemcpyAsync(out, dout, z.out_bytes, cudaMemcpyDeviceToHost, s->d2h) != cudaSuccess ||
+        cudaEventRecord(s->delivered[b], s->d2h) != cudaSuccess ||
+        cudaStreamWaitEvent(st, s->delivered[sync_out ? b : 1 - b], 0) != cudaSuccess)
         return QSTATE_ECUDA;
     s->host_calls++;
     return QSTATE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int qstate_step_host(qstate* s, const void* q, const void* k, const void* v, const void* gates,
+                     float* out, qstate_stream stream) {
+    return step_host_impl(s, q, k, v, gates, out, (cudaStream_t)stream, true);
+}
+
+int qstate_step_host_pipelined(qstate* s, const void* q, const void* k, const void* v,
+                               const void* gates, float* out, qstate_stream stream) {
+    return step_host_impl(s, q, k, v, gates, out, (cudaStream_t)stream, false);
+}
+
+int qstate_step_host_sync(qstate* s, qstate_stream stream) {
+    if (!s) return QSTATE_EINVAL;
+    if (!s->host_calls) return QSTATE_OK;
+    const int last = (int)((s->host_calls - 1) & 1);
+    return cudaStreamWaitEvent((cudaStream_t)stream, s->delivered[last], 0) == cudaSuccess
+               ? QSTATE_OK : QSTATE_ECUDA;
 }
 
 int qstate_dequant(const qstate* s, float* S_out, qstate_stream stream) {

@@ -24,7 +24,8 @@ F32, BF16, F16 = 0, 1, 2
 
 # every symbol include/qstate.h declares
 EXPORTS = ("qstate_create", "qstate_destroy", "qstate_reset", "qstate_step", "qstate_step_host",
-           "qstate_step_host_static", "qstate_dequant", "qstate_export", "qstate_import", "qstate_get_sizes",
+           "qstate_step_host_pipelined", "qstate_step_host_sync", "qstate_step_host_static",
+           "qstate_dequant", "qstate_export", "qstate_import", "qstate_get_sizes",
            "qstate_bytes_per_step", "qstate_status", "qstate_set_taxonomy", "qstate_set_lrb",
            "qstate_lrb_export", "qstate_set_pw", "qstate_pw_export", "qstate_set_rowcol",
            "qstate_error_rows", "qstate_kernel", "qstate_debug_set", "qstate_error_string")
@@ -75,6 +76,8 @@ def lib():
         L.qstate_step.argtypes = [P, P, P, P, P, P, S]
         L.qstate_step_host.argtypes = [P, P, P, P, P, P, S]
         L.qstate_step_host_static.argtypes = [P, P, P, P, P, P, S]
+        L.qstate_step_host_pipelined.argtypes = [P, P, P, P, P, P, S]
+        L.qstate_step_host_sync.argtypes = [P, S]
         L.qstate_dequant.argtypes = [P, P, S]
         L.qstate_export.argtypes = [P, P, P, P, S]
         L.qstate_import.argtypes = [P, P, P, P, S]
@@ -258,6 +261,19 @@ class QState:
         self._check_operands("step_host", (q, k, v, gates, out), host=True)
         _check("qstate_step_host", lib().qstate_step_host(self._h, _ptr(q), _ptr(k), _ptr(v),
                                                           _ptr(gates), _ptr(out), _stream(stream)))
+
+    def step_host_pipelined(self, q, k, v, gates, out, stream=None):
+        """step_host whose output copy overlaps the next call's step
+        (qstate_step_host_pipelined): the last call's output is complete
+        after step_host_sync and the stream."""
+        self._check_operands("step_host_pipelined", (q, k, v, gates, out), host=True)
+        _check("qstate_step_host_pipelined",
+               lib().qstate_step_host_pipelined(self._h, _ptr(q), _ptr(k), _ptr(v), _ptr(gates),
+                                                _ptr(out), _stream(stream)))
+
+    def step_host_sync(self, stream=None):
+        """The stream waits for the last host-buffer call's output copy."""
+        _check("qstate_step_host_sync", lib().qstate_step_host_sync(self._h, _stream(stream)))
 
     def step_host_static(self, q, k, v, gates, out, stream=None):
         """The host-buffer step that allocates no device memory: the operands

@@ -201,9 +201,26 @@ int qstate_step(qstate* s, const void* q, const void* k, const void* v, const vo
  * stream and its events are allocated by the first call and shared by every
  * later call on the object: issue all qstate_step_host calls of one object
  * on one stream (calls on different streams would overwrite each other's
- * operands). */
+ * operands).  The output copy runs on a second stream of the object's own,
+ * which `stream` waits for before the call returns control to later work. */
 int qstate_step_host(qstate* s, const void* q, const void* k, const void* v,
                      const void* gates, float* out, qstate_stream stream);
+
+/* qstate_step_host for a stream of calls (no counterpart on the pages): the
+ * same copies and step, but the output copy runs on a stream of the
+ * object's own, into the caller's `out` of this call, so that it overlaps
+ * the next call's step; completion of `stream` covers this call's input
+ * copies and step and the output copies of the calls before it.  The output
+ * of the last call is in host memory once `stream` has completed a
+ * following qstate_step_host_sync (or a following host-buffer call).  The
+ * same single-stream rule and staging buffers as qstate_step_host, with
+ * which it may be mixed. */
+int qstate_step_host_pipelined(qstate* s, const void* q, const void* k, const void* v,
+                               const void* gates, float* out, qstate_stream stream);
+
+/* Make `stream` wait for the output copy of the object's last host-buffer
+ * call (a no-op before the first). */
+int qstate_step_host_sync(qstate* s, qstate_stream stream);
 
 /* Size of the device array that qstate_step_host_static stages operands in. */
 #define QSTATE_STATIC_STAGING_BYTES (16u << 20)

@@ -227,6 +227,41 @@ def test_step_host_matches_step_and_dequant():
     b.close()
 
 
+def test_step_host_stream_of_calls():
+    """Host-buffer calls issued back to back with no synchronisation between
+    them (the copies of consecutive calls overlap the steps): plain calls are
+    complete once the stream is, pipelined ones once the stream has also
+    completed step_host_sync; every output equals the device-buffer step's."""
+    wl = C4.scaled(batch=2, heads=4, layers=2)
+    T = wl.batch * wl.heads * 2
+    steps = 7
+    xs = [concat_inputs([synth.gen_step(wl, s_, layer=l, tiles=np.arange(8)) for l in range(2)])
+          for s_ in range(steps)]
+    ref = gpu_object(wl, synth.PERSISTENT, 2, 2)
+    want = []
+    for x in xs:
+        out = torch.empty((T, wl.d_v), dtype=torch.float32, device="cuda")
+        ref.step(*gpu_inputs(wl, x), out)
+        want.append(out.cpu())
+    ref.close()
+    host_in = [tuple(t.cpu().pin_memory() for t in gpu_inputs(wl, x)) for x in xs]
+    stream = torch.cuda.current_stream()
+    for pipelined in (False, True):
+        obj = gpu_object(wl, synth.PERSISTENT, 2, 2)
+        outs = [torch.full((T, wl.d_v), float("nan")).pin_memory() for _ in range(steps)]
+        for i in range(steps):
+            if pipelined:
+                obj.step_host_pipelined(*host_in[i], outs[i])
+            else:
+                obj.step_host(*host_in[i], outs[i])
+        if pipelined:
+            obj.step_host_sync()
+        stream.synchronize()
+        for i in range(steps):
+            assert torch.equal(outs[i], want[i]), (pipelined, i)
+        obj.close()
+
+
 def test_export_import_roundtrip_and_reset():
     wl = C5.scaled(batch=2)
     a = gpu_object(wl, synth.YOKED, 2, 1)
