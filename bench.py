@@ -59,6 +59,8 @@ def parse():
                     help="override the number of layers stepped (small profiling cases)")
     ap.add_argument("--launch-samples", type=int, default=200,
                     help="launches timed one by one for the roofline figure")
+    ap.add_argument("--ring", type=int, default=16,
+                    help="decode steps of resident inputs the timed steps cycle through")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     return ap.parse_args()
@@ -271,7 +273,7 @@ def run_ours(args, rank, world, local_rank):
     bytes_per_step = sum(o.bytes_per_step() for o in objs)
 
     # ring of resident inputs (distinct layer seeds per rank)
-    ring_n = 16 if T <= 65536 else 8
+    ring_n = max(2, args.ring)
     bf = wl0.qkv_dtype == synth.BF16
     gbf = wl0.gate_dtype == synth.BF16
 

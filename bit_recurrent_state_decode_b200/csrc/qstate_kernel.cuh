@@ -65,9 +65,10 @@ struct StepParams {
     const void* gates;
     float* out;
     unsigned long long* counters;   // [0] non-finite tile-steps, [1] saturated scales,
-                                    // [2] pipeline wait timeouts, [3] warp-tiles that took
-                                    // the element-wise rounding path, [4..6] lost / moved /
-                                    // reversed elements, [7] BDR steps applied (taxonomy)
+                                    // [2] pipeline wait timeouts; with the taxonomy on,
+                                    // [3] warp-tiles that took the element-wise rounding
+                                    // path, [4..6] lost / moved / reversed elements, [7]
+                                    // BDR steps applied
     const long long* head_off;      // per-head byte offset in a (layer, batch) row, or null
     const unsigned char* head_bits; // per-head bit width, or null (uniform)
     long long row_bytes;            // code bytes of one (layer, batch) row (mixed bits)
@@ -1203,6 +1204,18 @@ __device__ __forceinline__ bool step_tile(const StepParams& p, long long tile, c
             for (int r = 1; r < 8; r++) mt = fmaxf(mt, m[r]);
             slow = !(__fmaf_rn(mt, inv[0], -(fq + 0.5f)) < 0.0f);
         }
+        // A BDR step leaves the code range only from a code at +-Qmax toward
+        // u with |u| > Qmax, and then |w| > Qmax as well (w lies beyond u).
+        // With every stored code within +-Qmax (not the step after an import),
+        // |u| <= Qmax |eta| inv (1 + 2^-23), eta = alpha * the previous scale.
+        // A persistent scale never shrinks (inv <= RN(1 / previous scale)),
+        // so with a scalar decay |alpha| <= 1 - 2^-20 every row has
+        // |eta| inv <= |alpha| (1 + 2^-24)^2 < 1 - 2^-22 and |u| < Qmax:
+        // then no row of the tile needs the clamp.
+        bool noclamp = false;
+        if constexpr (BDR && !YOKED)
+            noclamp = p.fast && p.scale_mode == M_PERSISTENT && !vec_alpha &&
+                      fabsf(al[0]) <= 1.0f - 0x1p-20f;
 #pragma unroll
         for (int r = 0; r < 8; r++) {
             if (group != 0) slow |= !(__fmaf_rn(m[r], inv[r], -(fq + 0.5f)) < 0.0f);
@@ -1210,19 +1223,12 @@ __device__ __forceinline__ bool step_tile(const StepParams& p, long long tile, c
                 const float eta = __fmul_rn(al[r], dprev[r]);
                 const float floor_ = fmaxf(__fmul_rn(eta, float(1 << (BITS - 1)) * 0x1p-21f), 0x1p-120f);
                 slow |= !(__fmaf_rn(fabsf(urow(r)), wmin, -floor_) > 0.0f);
-                // A BDR step leaves the code range only from a code at +-Qmax
-                // toward u with |u| > Qmax, and then |w| > Qmax as well (w lies
-                // beyond u).  With every stored code within +-Qmax (not the step
-                // after an import), |u| <= Qmax |eta| inv (1 + 2^-23), so rows
-                // with |eta| inv <= 1 - 2^-22 (a persistent scale with a decay
-                // below 1) never need the clamp.
-                const bool may_leave = __fmaf_rn(m[r], inv[r], -fq) > 0.0f &&
-                    (!p.fast || !(__fmaf_rn(fabsf(eta), inv[r], -(1.0f - 0x1p-22f)) <= 0.0f));
-                if (__any_sync(0xFFFFFFFFu, may_leave)) clampmask |= 1u << r;
+                if (__any_sync(0xFFFFFFFFu, __fmaf_rn(m[r], inv[r], -fq) > 0.0f)) clampmask |= 1u << r;
             }
         }
+        if (noclamp) clampmask = 0;
         if (__any_sync(0xFFFFFFFFu, slow)) {
-            if (lane == 0) atomicAdd(p.counters + 3, 1ull);
+            if (EXTRA && p.taxonomy && lane == 0) atomicAdd(p.counters + 3, 1ull);
             round_pack_exact<DK, DV, BITS, BDR>(a, urow, wc, inv, p.eps_b, ct, i0, cb);
         } else {
             round_pack_fast<DK, DV, BITS, BDR>(a, urow, wc, inv, p.eps_b, clampmask, ct, i0, cb);

@@ -137,7 +137,8 @@ typedef struct qstate_counters {
                                    copies (the step's results are then undefined) */
     uint64_t exact_path_warps; /* warp-tiles that rounded element by element (the
                                   general form, taken when the fast form's
-                                  conditions do not hold for every row of the warp) */
+                                  conditions do not hold for every row of the
+                                  warp); counted while qstate_set_taxonomy is on */
     /* Rounding taxonomy (only while qstate_set_taxonomy is on): elements with a
      * nonzero update d = x - a, classified on the grid of the new scale with
      * u = a * inv, w = x * inv and c = clamp(RTN(w)): reversed when c lies

@@ -87,6 +87,7 @@ def test_both_rounding_forms_against_the_oracle():
     heads = np.tile(np.arange(wl.heads), wl.batch)
     for tiny in (False, True):
         gpu = gpu_object(wl, synth.PERSISTENT, wl.batch, 1)
+        gpu.set_taxonomy(True)             # the path counter is kept with the taxonomy
         orc = oracle_state(wl, synth.PERSISTENT, heads)
         for step in range(16):
             x = synth.gen_step(wl, step, tiles=np.arange(T))
