@@ -376,7 +376,9 @@ class LrbState(State):
         self.g = np.zeros((T, K), np.float32)
         self.nres = np.zeros(T, np.int32)
         self.nnew = np.zeros(T, np.int32)
-        self.D = np.ones(T, np.float32)     # decay since the last merge
+        # decay since the last merge (GLA: one per key row)
+        self.gla = cfg.c.kind == GLA
+        self.D = np.ones((T, cfg.d_k) if self.gla else T, np.float32)
         self.merged = np.zeros(T, np.int32)
         self.peak_cols = 0                  # most columns held at once (before a merge)
         # the unmerged rest of the bypass at each tile's last merge
@@ -387,7 +389,8 @@ class LrbState(State):
         T = self.ntiles
         q, k, v = _f32(q).reshape(T, -1), _f32(k).reshape(T, -1), _f32(v).reshape(T, -1)
         if alpha is not None:
-            alpha = _f32(alpha).reshape(T, -1)[:, :1].copy()
+            alpha = _f32(alpha).reshape(T, -1)
+            alpha = alpha.copy() if self.gla else alpha[:, :1].copy()
         if beta is not None:
             beta = _f32(beta).reshape(T)
         out = np.zeros((T, cfg.d_v), np.float32)
@@ -409,14 +412,21 @@ class LrbState(State):
         """Bypass columns held per tile after the last step."""
         return self.nres + self.nnew
 
+    def _dfac(self, t: int):
+        """Tile t's decay since the last merge, as a column to scale rows."""
+        return self.D[t].astype(np.float64)[:, None] if self.gla else float(self.D[t])
+
     def state(self, t: int) -> np.ndarray:
-        """The tile's state D * S_hat + P (fp64)."""
-        return float(self.D[t]) * self.dequant()[t].astype(np.float64) + self.bypass(t)
+        """The tile's state D * S_hat + P (fp64; GLA: D per key row)."""
+        return self._dfac(t) * self.dequant()[t].astype(np.float64) + self.bypass(t)
 
     def bypass(self, t: int) -> np.ndarray:
-        """The bypass matrix P = sum_l g_l u_l w_l^T of tile t (fp64)."""
+        """The bypass matrix P = sum_l g_l u_l w_l^T of tile t (fp64; GLA: the
+        key sides read as D * u)."""
         n = int(self.nres[t] + self.nnew[t])
         u = self.u[t, :n].view(np.float16).astype(np.float64)
+        if self.gla:
+            u = u * self.D[t].astype(np.float64)[None, :]
         w = self.w[t, :n].view(np.float16).astype(np.float64)
         return np.einsum("l,li,lj->ij", self.g[t, :n].astype(np.float64), u, w)
 

@@ -525,6 +525,13 @@ void or_dequant(const or_cfg* c, int bits, const int8_t* codes, const float* sca
  *     r_j <- fma(g_l * csum_i(u_li k_i), w_lj, r_j).
  *  L5 The output is o_t = (a + P_t)^T q_t in the same form: the canonical
  *     sum over the decayed quantized part, then the columns in slot order.
+ *  L7 GLA (decay Diag(alpha_t)): D is one binary32 factor per key row
+ *     (D_i <- alpha_t,i * D_i; the 32 bits per row are the extra 1/16 bit of
+ *     GLA in Table 6 at d_v = 512); no coefficient decays (g stays 1); a
+ *     column's key side is stored divided by the row factors of its step,
+ *     binary16(k_i / D_i), and read as D_i * u_i, which carries every later
+ *     step's decay of row i; the merge threshold uses D_i of the element's
+ *     row.
  *  L6 When the m-th fresh column arrives the bypass is merged: the dense
  *     P_ij = sum_l fma(g_l * u_li, w_lj, .) (slots in order, from +0) is
  *     formed; an element is merged when |P_ij| >= eps_L * (D * scale_ij), eps_L
@@ -623,7 +630,7 @@ double or_lrb_bits(int bits, int group, int scale_bits, int d_k, int d_v, double
 static int valid_lrb(const or_cfg* c, const or_lrb_cfg* L)
 {
     if (!valid_cfg(c) || !L) return 0;
-    if (c->kind == OR_GLA || c->scale_mode == OR_YOKED || c->rotate) return 0;
+    if (c->scale_mode == OR_YOKED || c->rotate) return 0;
     if (L->k < 0 || L->m < 1 || L->k + L->m > OR_LRB_MAX_COLS) return 0;
     if (!(L->eps_l >= 0.0f)) return 0;
     return 1;
@@ -646,23 +653,34 @@ static void lrb_tile_step(const or_cfg* c, const or_lrb_cfg* L, int bits, int8_t
     float* x = (float*)malloc(sizeof(float) * n_el);
     float* P = (float*)malloc(sizeof(float) * n_el);
     float uf[OR_LRB_MAX_COLS][512], wf[OR_LRB_MAX_COLS][512];
+    const int gla = c->kind == OR_GLA;
     const float al = c->kind == OR_RETNET ? c->gamma : alpha[0];
 
-    /* L3: the decay accumulates in D; the decayed quantized part as the plain
-     * step's decay with D for alpha; the columns' own decays */
-    *D = al * *D;
+    /* L3: the decay accumulates in D (GLA: one factor per key row, L7); the
+     * decayed quantized part as the plain step's decay with D for alpha; the
+     * columns' own decays (scalar decays: their coefficients) */
+    if (gla) {
+        for (int i = 0; i < dk; i++) D[i] = alpha[i] * D[i];
+    } else {
+        *D = al * *D;
+    }
     for (int i = 0; i < dk; i++)
         for (int j = 0; j < dv; j++) {
             size_t e = (size_t)i * dv + j;
             float delta = c->group ? scales[i * ng + j / gs] : scales[0];
-            a[e] = (float)codes[e] * (*D * delta);
+            a[e] = (float)codes[e] * ((gla ? D[i] : *D) * delta);
         }
     int n = *nres + *nnew;
-    for (int l = 0; l < n; l++) g[l] = al * g[l];
+    if (!gla)
+        for (int l = 0; l < n; l++) g[l] = al * g[l];
 
-    /* L4: the update as a new column */
+    /* L4: the update as a new column (GLA, L7: the key side held divided by
+     * D, each column's effective key side D * u formed when it is read) */
     for (int l = 0; l < n; l++) {
-        for (int i = 0; i < dk; i++) uf[l][i] = or_f16_to_f32(u[(size_t)l * dk + i]);
+        for (int i = 0; i < dk; i++) {
+            uf[l][i] = or_f16_to_f32(u[(size_t)l * dk + i]);
+            if (gla) uf[l][i] = D[i] * uf[l][i];
+        }
         for (int j = 0; j < dv; j++) wf[l][j] = or_f16_to_f32(w[(size_t)l * dv + j]);
     }
     float wnew[512], unew[512];
@@ -677,9 +695,12 @@ static void lrb_tile_step(const or_cfg* c, const or_lrb_cfg* L, int bits, int8_t
         for (int i = 0; i < dk; i++) unew[i] = f16r(beta * k[i]);
     } else {
         for (int j = 0; j < dv; j++) wnew[j] = f16r(v[j]);
-        for (int i = 0; i < dk; i++) unew[i] = f16r(k[i]);
+        for (int i = 0; i < dk; i++) unew[i] = f16r(gla ? k[i] / D[i] : k[i]);
     }
-    for (int i = 0; i < dk; i++) { u[(size_t)n * dk + i] = or_f32_to_f16(unew[i]); uf[n][i] = unew[i]; }
+    for (int i = 0; i < dk; i++) {
+        u[(size_t)n * dk + i] = or_f32_to_f16(unew[i]);
+        uf[n][i] = gla ? D[i] * unew[i] : unew[i];
+    }
     for (int j = 0; j < dv; j++) { w[(size_t)n * dv + j] = or_f32_to_f16(wnew[j]); wf[n][j] = wnew[j]; }
     g[n] = 1.0f;
     n++;
@@ -708,7 +729,7 @@ static void lrb_tile_step(const or_cfg* c, const or_lrb_cfg* L, int bits, int8_t
             for (int j = 0; j < dv; j++) {
                 size_t e = (size_t)i * dv + j;
                 float dprev = c->group ? scales[i * ng + j / gs] : scales[0];
-                if (fabsf(P[e]) >= L->eps_l * (*D * dprev)) {
+                if (fabsf(P[e]) >= L->eps_l * ((gla ? D[i] : *D) * dprev)) {
                     x[e] = a[e] + P[e];
                     P[e] = 0.0f;                     /* merged: leaves the residual */
                     n_merged++;
@@ -771,7 +792,10 @@ static void lrb_tile_step(const or_cfg* c, const or_lrb_cfg* L, int bits, int8_t
         }
         *nres = kk;
         *nnew = 0;
-        *D = 1.0f;
+        if (gla)
+            for (int i = 0; i < dk; i++) D[i] = 1.0f;
+        else
+            *D = 1.0f;
     }
     if (merged_out) *merged_out = n_merged;
     free(a);
@@ -791,8 +815,9 @@ int or_lrb_step(const or_cfg* c, const or_lrb_cfg* L, int64_t ntiles, const int*
         if (tile_bits[t] < 2 || tile_bits[t] > 8 || tile_bits[t] % 2) return -1;
     for (int64_t t = 0; t < ntiles; t++)
         lrb_tile_step(c, L, tile_bits[t], codes + t * dk * dv, scales + t * nsc,
-                      u + t * K * dk, w + t * K * dv, g + t * K, nres + t, nnew + t, D + t,
-                      q + t * dk, k + t * dk, v + t * dv, alpha ? alpha + t : NULL,
+                      u + t * K * dk, w + t * K * dv, g + t * K, nres + t, nnew + t,
+                      D + (c->kind == OR_GLA ? t * dk : t), q + t * dk, k + t * dk, v + t * dv,
+                      alpha ? alpha + (c->kind == OR_GLA ? t * dk : t) : NULL,
                       beta ? beta[t] : 0.0f, out + t * dv, cnt, merged ? merged + t : NULL,
                       resid ? resid + t * (int64_t)dk * dv : NULL);
     return 0;

@@ -128,11 +128,11 @@ typedef struct {
     float eps_l;      /* merge threshold, in grid steps of the element's scale */
 } or_lrb_cfg;
 
-/* One LRB step over ntiles tiles (quantized widths 2..8 only; RetNet,
- * Mamba2, GDN; dynamic or persistent scales).  Bypass per tile: u
+/* One LRB step over ntiles tiles (quantized widths 2..8 only; all four
+ * kinds; dynamic or persistent scales).  Bypass per tile: u
  * [k+m][d_k] and w [k+m][d_v] binary16 bit patterns, g [k+m] binary32,
  * nres / nnew the residual and fresh slot counts, D [ntiles] the decay since
- * the last merge (1 at the start).  merged (may be NULL):
+ * the last merge (GLA: [ntiles][d_k], one per key row; 1 at the start).  merged (may be NULL):
  * per tile, the number of elements merged by this step.  resid (may be
  * NULL): [ntiles][d_k][d_v], at a merge the unmerged rest of the bypass
  * (before its rank-k approximation), untouched otherwise.  -1 if invalid. */
