@@ -225,6 +225,9 @@ int zero_window(qstate* s, cudaStream_t st) {
     return QSTATE_OK;
 }
 
+// decay factors a tile's bypass holds: one per key row for GLA, else one
+int64_t lrb_dlen(const qstate* s) { return s->L.kind == QSTATE_GLA ? s->L.d_k : 1; }
+
 // bypass empty, D = 1 for every tile
 int zero_bypass(qstate* s, cudaStream_t st) {
     if (!s->lrb || s->tiles == 0) return QSTATE_OK;
@@ -236,7 +239,7 @@ int zero_bypass(qstate* s, cudaStream_t st) {
         return QSTATE_ECUDA;
     // D = 1: copied from a host array (a copy from pageable memory has left
     // the array when the call returns)
-    std::vector<float> ones((size_t)s->tiles, 1.0f);
+    std::vector<float> ones((size_t)(s->tiles * lrb_dlen(s)), 1.0f);
     if (cudaMemcpyAsync(s->d_lD, ones.data(), ones.size() * 4, cudaMemcpyHostToDevice, st) != cudaSuccess)
         return QSTATE_ECUDA;
     return QSTATE_OK;
@@ -704,7 +707,8 @@ int64_t qstate_bytes_per_step(const qstate* s) {
         const int64_t k = s->lrb_k, m = s->lrb_m;
         const int64_t col = (dk + dv) * 2 + 4;
         int64_t b = m * (s->code_bytes + s->scale_bytes) + s->code_bytes + s->scale_bytes;
-        b += s->tiles * ((k * m + m * (m - 1) / 2) * col + m * col + k * col + m * 16);
+        b += s->tiles * ((k * m + m * (m - 1) / 2) * col + m * col + k * col +
+                         m * (8 + 8 * lrb_dlen(s)));
         return b / m + ops;
     }
     int64_t b = 2 * s->code_bytes + 2 * s->scale_bytes + 2 * s->ref_bytes;
@@ -801,13 +805,14 @@ int qstate_set_lrb(qstate* s, int k, int m, float eps_l) {
     if (!s || s->lrb || s->pw || s->rowcol) return QSTATE_EINVAL;
     if (k < 0 || k > 1 || m < 1 || k + m > qs::kLrbMaxCols) return QSTATE_EINVAL;
     if (!(eps_l >= 0.0f) || !std::isfinite(eps_l)) return QSTATE_EINVAL;
-    if (s->L.kind == QSTATE_GLA || s->scale_mode == QSTATE_YOKED || s->L.rotation ||
+    if (s->scale_mode == QSTATE_YOKED || s->L.rotation ||
         !s->head_bits.empty() || !(s->bits == 4 || s->bits == 8) || s->L.d_k != s->L.d_v)
         return QSTATE_EUNSUPPORTED;
     int rc = check_device(s);
     if (rc != QSTATE_OK) return rc;
     const int d = s->L.d_k;
-    const int idx = ((((d == 128) * 2 + (s->bits == 8)) * 2 + (s->L.kind == QSTATE_GDN)) * 2 +
+    const int kind = s->L.kind == QSTATE_GDN ? 1 : s->L.kind == QSTATE_GLA ? 2 : 0;
+    const int idx = ((((d == 128) * 2 + (s->bits == 8)) * 3 + kind) * 2 +
                      (s->round_mode == QSTATE_BDR)) * 2 + (s->L.qkv_dtype == QSTATE_BF16);
     const qs::LrbEntry* e = &qs::lrb_table()[idx];
     const int smem = k == 1 ? 64 * e->threads * 4 : 0;
@@ -817,7 +822,7 @@ int qstate_set_lrb(qstate* s, int k, int m, float eps_l) {
     auto alloc = [&](void** p, size_t n) -> bool { return !n || cudaMalloc(p, n) == cudaSuccess; };
     if (!alloc((void**)&s->d_lu, T * K * s->L.d_k * 2) || !alloc((void**)&s->d_lw, T * K * s->L.d_v * 2) ||
         !alloc((void**)&s->d_lg, T * K * 4) || !alloc((void**)&s->d_ln, T * 2 * 4) ||
-        !alloc((void**)&s->d_lD, T * 4)) {
+        !alloc((void**)&s->d_lD, T * lrb_dlen(s) * 4)) {
         cudaGetLastError();
         cudaFree(s->d_lu); cudaFree(s->d_lw); cudaFree(s->d_lg); cudaFree(s->d_ln); cudaFree(s->d_lD);
         s->d_lu = s->d_lw = nullptr;
@@ -860,7 +865,7 @@ int qstate_lrb_export(const qstate* s, uint16_t* u, uint16_t* w, float* g, int32
         cudaMemcpyAsync(w, s->d_lw, T * K * s->L.d_v * 2, cudaMemcpyDefault, st) != cudaSuccess ||
         cudaMemcpyAsync(g, s->d_lg, T * K * 4, cudaMemcpyDefault, st) != cudaSuccess ||
         cudaMemcpyAsync(n, s->d_ln, T * 2 * 4, cudaMemcpyDefault, st) != cudaSuccess ||
-        cudaMemcpyAsync(D, s->d_lD, T * 4, cudaMemcpyDefault, st) != cudaSuccess)
+        cudaMemcpyAsync(D, s->d_lD, T * lrb_dlen(s) * 4, cudaMemcpyDefault, st) != cudaSuccess)
         return QSTATE_ECUDA;
     return QSTATE_OK;
 }

@@ -36,7 +36,7 @@ struct LrbParams {
     uint16_t* w;      // [tiles][k + m][d_v] binary16
     float* g;         // [tiles][k + m]
     int* n;           // [tiles][2]: residual slots in use, fresh slots in use
-    float* D;         // [tiles]: decay since the last merge
+    float* D;         // [tiles] (GLA: [tiles][d_k]): decay since the last merge
     int k, m;
     float eps_l;
 };
@@ -85,6 +85,7 @@ struct __align__(16) LrbShared {
     float gco[kLrbMaxCols];          // decayed coefficients, the new column's = 1
     float ck[kLrbMaxCols], cq[kLrbMaxCols];   // g_l (u_l . k), g_l (u_l . q)
     float unew[DK], wnew[DV];        // the new column (binary16 values)
+    float drow[DK];                  // GLA: the per-row decay since the last merge, this step's
     // the tile's scales before the step, in their stored format
     __align__(16) uint8_t sprev[DK * (DV / 8) * 4];
     // the columns held at the start of the step (binary16 patterns)
@@ -235,10 +236,14 @@ __device__ __forceinline__ void requantize(const StepParams& p, XS& xs, const ui
 // Two CTAs per SM: the decayed quantized part a is re-derived from the codes
 // (an L1 hit after the first read) wherever the step needs it, so only the
 // merge's 8 x 8 block stays in registers.
-template <int DK, int DV, int BITS, bool GDN, bool BDR, bool BF>
+// VEC: GLA's per-row decay: D holds one factor per key row, the coefficients
+// do not decay, and a column's key side is held divided by the row factors of
+// its step and read as D_i * u_i.
+template <int DK, int DV, int BITS, bool GDN, bool VEC, bool BDR, bool BF>
 __global__ void __launch_bounds__(Geo<DK, DV>::NT, 2) lrb_kernel(const StepParams p, const LrbParams L) {
     using G = Geo<DK, DV>;
     static_assert(DK == DV, "square tiles");
+    static_assert(!(GDN && VEC), "the delta rule has a scalar decay");
     static_assert(BITS == 4 || BITS == 8, "4- or 8-bit codes");
     constexpr int QMAX = (1 << (BITS - 1)) - 1;
     constexpr float fq = float(QMAX);
@@ -262,9 +267,15 @@ __global__ void __launch_bounds__(Geo<DK, DV>::NT, 2) lrb_kernel(const StepParam
         const uint16_t* Wc = L.w + tile * K * DV;
         uint8_t* ct = p.codes + tile * p.tile_bytes;
         const long long sbase = tile * (long long)p.n_scales;
-        const float alpha = p.kind == K_RETNET ? p.gamma : ldg1(p.gates, tile * p.n_gate, p.gate_bf16 != 0);
+        const float alpha = VEC ? 1.0f
+                          : p.kind == K_RETNET ? p.gamma : ldg1(p.gates, tile * p.n_gate, p.gate_bf16 != 0);
         const float beta = GDN ? ldg1(p.gates, tile * p.n_gate + 1, p.gate_bf16 != 0) : 0.0f;
-        const float Dn = __fmul_rn(alpha, L.D[tile]);
+        const float Dn = VEC ? 0.0f : __fmul_rn(alpha, L.D[tile]);
+        if constexpr (VEC) {
+            for (int i = threadIdx.x; i < DK; i += G::NT)
+                sh.drow[i] = __fmul_rn(ldg1(p.gates, tile * p.n_gate + i, p.gate_bf16 != 0),
+                                       L.D[tile * DK + i]);
+        }
 
         // the next tile's bytes on their way to L2 while this one is stepped
         {
@@ -308,16 +319,22 @@ __global__ void __launch_bounds__(Geo<DK, DV>::NT, 2) lrb_kernel(const StepParam
             if (sf32) return reinterpret_cast<const float*>(sh.sprev)[idx];
             return __half2float(reinterpret_cast<const __half*>(sh.sprev)[idx]);
         };
-        for (int l = threadIdx.x; l < n; l += G::NT) sh.gco[l] = __fmul_rn(alpha, L.g[tile * K + l]);
+        for (int l = threadIdx.x; l < n; l += G::NT)
+            sh.gco[l] = VEC ? L.g[tile * K + l] : __fmul_rn(alpha, L.g[tile * K + l]);
         __syncthreads();
+        // a column's key side as the step reads it (GLA: D_i * u_i)
+        auto ueff = [&](int l, int i) -> float {
+            const float u = h2f(sh.ucol[l * DK + i]);
+            return VEC ? __fmul_rn(sh.drow[i], u) : u;
+        };
         // g_l (u_l . k) and g_l (u_l . q) for the columns held
         const uint8_t* kin = static_cast<const uint8_t*>(p.k) + tile * DK * (BF ? 2 : 4);
         const uint8_t* qin = static_cast<const uint8_t*>(p.q) + tile * DK * (BF ? 2 : 4);
         auto kval = [&](int i) { return ldg1(kin, i, BF); };
         auto qval = [&](int i) { return ldg1(qin, i, BF); };
         for (int l = warp; l < n; l += G::NWARPS) {
-            auto uval = [&](int i) { return h2f(sh.ucol[l * DK + i]); };
-            const float dk_ = warp_canon_dot<DK>(uval, kval, lane);
+            auto uval = [&](int i) { return ueff(l, i); };
+            const float dk_ = GDN ? warp_canon_dot<DK>(uval, kval, lane) : 0.0f;
             const float dq_ = warp_canon_dot<DK>(uval, qval, lane);
             if (lane == 0) {
                 sh.ck[l] = __fmul_rn(sh.gco[l], dk_);
@@ -332,7 +349,7 @@ __global__ void __launch_bounds__(Geo<DK, DV>::NT, 2) lrb_kernel(const StepParam
             kk[r] = kval(i0 + r);
             qq[r] = qval(i0 + r);
             const float dp = prev_scale(group ? (i0 + r) * ng + gcol : 0);
-            eta[r] = __fmul_rn(Dn, dp);
+            eta[r] = __fmul_rn(VEC ? sh.drow[i0 + r] : Dn, dp);
         }
         {
             const uint8_t* vin = static_cast<const uint8_t*>(p.v) + tile * DV * (BF ? 2 : 4);
@@ -395,11 +412,13 @@ __global__ void __launch_bounds__(Geo<DK, DV>::NT, 2) lrb_kernel(const StepParam
         }
         if (cb == 0) {
 #pragma unroll
-            for (int r = 0; r < 8; r++) sh.unew[i0 + r] = f16r(GDN ? __fmul_rn(beta, kk[r]) : kk[r]);
+            for (int r = 0; r < 8; r++)
+                sh.unew[i0 + r] = f16r(GDN ? __fmul_rn(beta, kk[r])
+                                           : VEC ? __fdiv_rn(kk[r], sh.drow[i0 + r]) : kk[r]);
         }
         __syncthreads();
         if (warp == 0) {
-            auto uval = [&](int i) { return sh.unew[i]; };
+            auto uval = [&](int i) { return VEC ? __fmul_rn(sh.drow[i], sh.unew[i]) : sh.unew[i]; };
             const float dq_ = warp_canon_dot<DK>(uval, qval, lane);
             if (lane == 0) {
                 sh.cq[n] = __fmul_rn(1.0f, dq_);
@@ -450,8 +469,11 @@ __global__ void __launch_bounds__(Geo<DK, DV>::NT, 2) lrb_kernel(const StepParam
         for (int l = threadIdx.x; l <= n; l += G::NT) L.g[tile * K + l] = sh.gco[l];
 
         if (nnew + 1 < L.m) {                              // no merge: codes untouched
+            if constexpr (VEC) {
+                for (int i = threadIdx.x; i < DK; i += G::NT) L.D[tile * DK + i] = sh.drow[i];
+            }
             if (threadIdx.x == 0) {
-                L.D[tile] = Dn;
+                if (!VEC) L.D[tile] = Dn;
                 L.n[2 * tile + 1] = nnew + 1;
             }
             __syncthreads();
@@ -479,6 +501,10 @@ __global__ void __launch_bounds__(Geo<DK, DV>::NT, 2) lrb_kernel(const StepParam
                         u8[i] = sh.unew[i0 + i];
                         w8[i] = sh.wnew[j0 + i];
                     }
+                }
+                if constexpr (VEC) {
+#pragma unroll
+                    for (int i = 0; i < 8; i++) u8[i] = __fmul_rn(sh.drow[i0 + i], u8[i]);
                 }
 #pragma unroll
                 for (int r = 0; r < 8; r++) {
@@ -586,8 +612,11 @@ __global__ void __launch_bounds__(Geo<DK, DV>::NT, 2) lrb_kernel(const StepParam
                 L.w[(tile * K) * DV + j] = f2h(sig > 0.0f ? rs * sh.vec[j] : 0.0f);
             if (threadIdx.x == 0) L.g[tile * K] = 1.0f;
         }
+        if constexpr (VEC) {
+            for (int i = threadIdx.x; i < DK; i += G::NT) L.D[tile * DK + i] = 1.0f;
+        }
         if (threadIdx.x == 0) {
-            L.D[tile] = 1.0f;
+            if (!VEC) L.D[tile] = 1.0f;
             L.n[2 * tile] = L.k;
             L.n[2 * tile + 1] = 0;
         }

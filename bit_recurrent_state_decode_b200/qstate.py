@@ -369,7 +369,7 @@ class QState:
     def lrb_export(self, stream=None) -> dict:
         """The bypass as new CUDA tensors: u [tiles, k+m, d_k] and
         w [tiles, k+m, d_v] (float16), g [tiles, k+m], n [tiles, 2]
-        (residual and fresh columns held), D [tiles]."""
+        (residual and fresh columns held), D [tiles] (GLA: [tiles, d_k])."""
         if self.lrb is None:
             raise QStateError("qstate_lrb_export", 1)
         K = self.lrb[0] + self.lrb[1]
@@ -379,7 +379,7 @@ class QState:
         w = torch.empty((T, K, self.d_v), dtype=torch.float16, device=dev)
         g = torch.empty((T, K), dtype=torch.float32, device=dev)
         n = torch.empty((T, 2), dtype=torch.int32, device=dev)
-        D = torch.empty((T,), dtype=torch.float32, device=dev)
+        D = torch.empty((T, self.d_k) if self.kind == GLA else (T,), dtype=torch.float32, device=dev)
         _check("qstate_lrb_export", lib().qstate_lrb_export(self._h, _ptr(u), _ptr(w), _ptr(g), _ptr(n),
                                                             _ptr(D), _stream(stream)))
         return {"u": u, "w": w, "g": g, "n": n, "D": D}

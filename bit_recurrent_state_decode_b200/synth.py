@@ -217,6 +217,14 @@ VARIANTS = {
         (DYNAMIC,), BDR, BF16, BF16, F16, layers=24, rowcol=True,
         description="Gated DeltaNet x24 layers, INT4 with fp16 key-row x value-column scales "
                     "fitted every step, BDR, bf16"),
+    # the GLA decode with the same bypass (k = 1, m = 15, eps_L = 0.50): a
+    # decay factor per key row instead of one per tile
+    "gla_b128_h16_d128_int4g32_lrb": Workload(
+        "gla_b128_h16_d128_int4g32_lrb", 9, GLA, 128, 16, 128, 128, 4096, 4, 32,
+        (PERSISTENT,), RTN, BF16, F32, F16, q_sigma=float(np.float32(1 / np.sqrt(128))),
+        k_sigma=float(np.float32(1 / np.sqrt(128))), lrb=(1, 15, 0.5),
+        description="GLA diagonal decay, INT4 g32 fp16 persistent scale, RTN, bf16, with a "
+                    "Low-Rank Bypass (k=1, m=15, eps_L=0.5; one decay factor per key row)"),
 }
 
 

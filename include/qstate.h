@@ -317,9 +317,12 @@ int qstate_error_rows(const qstate* s, float* out, qstate_stream stream);
  * object's scale and rounding modes (BDR with the merged update as d), D
  * reset to 1 and the rest kept as its leading singular pair (k = 1, found by
  * power iteration) or dropped (k = 0).  The state a tile stands for is
- * D * dequant(codes) + sum_l g_l u_l w_l^T.
- * k in {0, 1}, m >= 1, k + m <= 32, eps_l >= 0.  Supported for RetNet,
- * Mamba2 and Gated DeltaNet objects with one code width of 4 or 8 bits,
+ * D * dequant(codes) + sum_l g_l u_l w_l^T.  GLA (decay Diag(alpha)) keeps
+ * one D per key row instead: the coefficients do not decay, a column's key
+ * side is stored as fp16(k / D) of its step and read as D_i u_i, and the
+ * tile stands for Diag(D) (dequant(codes) + sum_l g_l u_l w_l^T).
+ * k in {0, 1}, m >= 1, k + m <= 32, eps_l >= 0.  Supported for all four
+ * kinds with one code width of 4 or 8 bits,
  * d_k = d_v in {64, 128}, dynamic or persistent scales, no rotation
  * (QSTATE_EUNSUPPORTED otherwise); allocates the bypass (QSTATE_ENOMEM).
  * QSTATE_EINVAL if a bypass, a window or row x column scales are already set
@@ -377,7 +380,8 @@ const char* qstate_kernel(const qstate* s);
 
 /* Copy an LRB object's bypass to caller buffers (device or host):
  * u [tiles][k+m][d_k] and w [tiles][k+m][d_v] binary16 bit patterns,
- * g [tiles][k+m], n [tiles][2] (residual and fresh columns held), D [tiles]. */
+ * g [tiles][k+m], n [tiles][2] (residual and fresh columns held), D [tiles]
+ * (GLA: [tiles][d_k]). */
 int qstate_lrb_export(const qstate* s, uint16_t* u, uint16_t* w, float* g, int32_t* n, float* D,
                       qstate_stream stream);
 

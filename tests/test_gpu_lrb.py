@@ -1,6 +1,8 @@
 """GPU parity of the decode step with a Low-Rank Bypass (LRB) of "Preserving
 Updates in Low-Bit Recurrent State Quantization" (Abstract, Figure 3,
-Tables 6, 8, 9) against the oracle's LRB step.
+Tables 6, 8, 9) against the oracle's LRB step, for the scalar decays, the
+delta rule and GLA's per-row decay (one factor D_i per key row, key sides
+held divided by it).
 
 - k = 0 (no residual): every result is defined element by element (canonical
   sums, columns in slot order, one fma each), so outputs, codes, scales, the
@@ -51,11 +53,18 @@ CASES = {
                                         group=32, scale_modes=(synth.DYNAMIC,),
                                         round_mode=synth.RTN), 0, 1, 0.25),
     "gdn_d128_int4_bdr_k0_m15": (C4.scaled(batch=1, heads=4, layers=1, eps_b=0.3), 0, 15, 0.5),
+    # GLA (one decay factor per key row): d 128 INT4 g32 persistent, bf16
+    # inputs; d 64 INT8 per-token dynamic scales with BDR, fp32 inputs
+    "gla_d128_int4g32_k0_m4": (C3.scaled(batch=2, heads=4), 0, 4, 0.5),
+    "gla_d64_int8tok_bdr_k0_m3": (C3.scaled(batch=2, heads=4, d_k=64, d_v=64, bits=8, group=0,
+                                            scale_modes=(synth.DYNAMIC,), round_mode=synth.BDR,
+                                            eps_b=0.3, qkv_dtype=synth.F32), 0, 3, 0.5),
 }
 CASES_K1 = {
     "retnet_d64_int4_k1_m3": (C1.scaled(batch=3, heads=4), 1, 3, 0.5),
     "gdn_d128_int4_bdr_k1_m4": (C4.scaled(batch=2, heads=4, layers=1, eps_b=0.3), 1, 4, 0.5),
     "mamba2_d128_int8tok_k1_m5": (C2.scaled(batch=2, heads=4, d_v=128), 1, 5, 0.5),
+    "gla_d128_int4g32_k1_m3": (C3.scaled(batch=2, heads=4), 1, 3, 0.5),
 }
 
 
@@ -108,14 +117,18 @@ def _assert_exact(gpu, orc, o_gpu, o_orc, step):
 
 
 def _gpu_states(gpu, b):
-    """D * S_hat + P of every GPU tile (fp64)."""
+    """D * S_hat + P of every GPU tile (fp64; GLA: D per key row, the key
+    sides read as D * u)."""
     deq = gpu.dequant().double().cpu().numpy()
     for t in range(gpu.tiles):
         n = int(b["n"][t].sum())
         u = b["u"][t, :n].astype(np.float64)
         w = b["w"][t, :n].astype(np.float64)
-        deq[t] = float(b["D"][t]) * deq[t] + np.einsum("l,li,lj->ij", b["g"][t, :n].astype(np.float64),
-                                                       u, w)
+        D = b["D"][t].astype(np.float64)
+        if D.ndim:
+            u = u * D[None, :]
+            D = D[:, None]
+        deq[t] = D * deq[t] + np.einsum("l,li,lj->ij", b["g"][t, :n].astype(np.float64), u, w)
     return deq
 
 
@@ -207,7 +220,6 @@ def test_lrb_k1(name):
 def test_lrb_rejects():
     """Layouts the bypass kernel does not take, and invalid k, m, eps_L."""
     bad_layouts = [
-        C3.scaled(batch=1, heads=2),                                           # GLA
         C4.scaled(batch=1, heads=2, layers=1, scale_modes=(synth.YOKED,)),    # yoked
         C2.scaled(batch=1, heads=2),                                           # d_k != d_v
         C4.scaled(batch=1, heads=2, layers=1, bits=6),                         # 6-bit codes

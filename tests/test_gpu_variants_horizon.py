@@ -94,3 +94,23 @@ def test_lrb_no_residual_horizon():
             assert np.array_equal(b["u"][t, :n].view(np.uint16), o.u[t, :n]), (step, t)
             assert np.array_equal(b["w"][t, :n].view(np.uint16), o.w[t, :n]), (step, t)
     _run("gdn_l24_b256_h32_d128_int4g32_lrb", make, check, steps=8 * m + 7)
+
+
+def test_lrb_gla_no_residual_horizon():
+    """GLA's bypass (a decay factor per key row) through eight merge cycles of
+    the 16-head GLA workload's streams (d 128, INT4 g32, persistent scales)."""
+    m = 15
+
+    def make(wl, mode):
+        g = gpu_object(wl, mode, 1, 1)
+        g.set_lrb(0, m, 0.5)
+        return g, oracle.LrbState(_cfg(wl, mode), np.full(g.tiles, wl.bits), k=0, m=m, eps_l=0.5)
+
+    def check(g, o, step):
+        b = {n: t.cpu().numpy() for n, t in g.lrb_export().items()}
+        assert np.array_equal(b["n"][:, 1], o.nnew)
+        assert np.array_equal(b["D"].view(np.uint32), o.D.view(np.uint32)), step
+        for t in range(g.tiles):
+            n = int(o.nnew[t])
+            assert np.array_equal(b["u"][t, :n].view(np.uint16), o.u[t, :n]), (step, t)
+    _run("gla_b128_h16_d128_int4g32_persistent", make, check, steps=8 * m + 7)
