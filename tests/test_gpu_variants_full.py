@@ -6,10 +6,12 @@ the sampled tiles' outputs, codes, scales and side state are compared.
 
 - INT4+Had and key-row x value-column scales: bit-exact after 3 steps.
 - PW-S8: bit-exact after 10 steps (the window full, two pairs merged).
-- LRB+BDR (k = 1, m = 15): bit-exact through the first merge and up to the
-  second; at the second merge outputs, codes, scales and counts are still
-  bit-exact and the kept rank-1 residual is within the tolerance of the
-  small-case test of its optimum (the oracle's truncated SVD).
+- LRB+BDR (k = 1, m = 15), and the same bypass on the GLA decode (a decay
+  factor per key row; 24 layer replicas of B128 H16, 49 152 tiles, as the
+  benchmark steps that L2-sized layer): bit-exact through the first merge and
+  up to the second; at the second merge outputs, codes, scales and counts
+  are still bit-exact and the kept rank-1 residual is within the tolerance
+  of the small-case test of its optimum (the oracle's truncated SVD).
 """
 import numpy as np
 import pytest
@@ -93,8 +95,10 @@ def test_full_size_sampled_pw():
     gpu.close()
 
 
-def test_full_size_sampled_lrb():
-    wl = synth.workload("gdn_l24_b256_h32_d128_int4g32_lrb")
+@pytest.mark.parametrize("name,layers", [("gdn_l24_b256_h32_d128_int4g32_lrb", 24),
+                                         ("gla_b128_h16_d128_int4g32_lrb", 24)])
+def test_full_size_sampled_lrb(name, layers):
+    wl = synth.workload(name).scaled(layers=layers)
     k, m, eps_l = wl.lrb
     sample, T = _sample(wl)
     mode = wl.scale_modes[0]
@@ -109,7 +113,7 @@ def test_full_size_sampled_lrb():
         assert np.array_equal(o_gpu.view(np.uint32), o_orc.view(np.uint32)), step
     b = {n: t[idx].cpu().numpy() for n, t in gpu.lrb_export().items()}
     assert np.array_equal(b["n"][:, 0], orc.nres) and np.array_equal(b["n"][:, 1], orc.nnew)
-    assert np.all(b["D"] == 1.0)
+    assert np.all(b["D"] == 1.0) and np.all(orc.D == 1.0)
     view = GpuView(gpu)
     for i, t in enumerate(sample):
         assert np.array_equal(view.tile_codes(t), orc.codes[i]), t
