@@ -288,6 +288,8 @@ class QState:
     def dequant(self, out=None, stream=None) -> torch.Tensor:
         if out is None:
             out = torch.empty((self.tiles, self.d_k, self.d_v), dtype=torch.float32, device="cuda")
+        if self.tiles == 0:             # nothing to write (an empty tensor has no address)
+            return out
         _check("qstate_dequant", lib().qstate_dequant(self._h, _ptr(out), _stream(stream)))
         return out
 
@@ -300,11 +302,15 @@ class QState:
                              dtype=sdt, device="cuda")
         ref = (torch.empty(z["ref_bytes"] // 4, dtype=torch.float32, device="cuda")
                if z["ref_bytes"] else None)
+        if self.tiles == 0:
+            return codes, scales, ref
         _check("qstate_export", lib().qstate_export(self._h, _ptr(codes), _ptr(scales), _ptr(ref),
                                                     _stream(stream)))
         return codes, scales, ref
 
     def import_(self, codes, scales, ref=None, stream=None):
+        if self.tiles == 0:
+            return
         _check("qstate_import", lib().qstate_import(self._h, _ptr(codes), _ptr(scales), _ptr(ref),
                                                     _stream(stream)))
 
@@ -327,6 +333,8 @@ class QState:
         """Per tile and key row, the squared rounding error of the last step
         taken with the taxonomy on (qstate_error_rows), [tiles, d_k]."""
         out = torch.empty((self.tiles, self.d_k), dtype=torch.float32, device=f"cuda:{self.device}")
+        if self.tiles == 0:
+            return out
         _check("qstate_error_rows", lib().qstate_error_rows(self._h, _ptr(out), _stream(stream)))
         return out
 
@@ -356,6 +364,8 @@ class QState:
         B = torch.empty((T, W, self.d_v), dtype=torch.uint8, device=dev)
         head = torch.empty((T,), dtype=torch.int32, device=dev)
         count = torch.empty((T,), dtype=torch.int32, device=dev)
+        if T == 0:
+            return {"A": A, "B": B, "head": head, "count": count}
         _check("qstate_pw_export", lib().qstate_pw_export(self._h, _ptr(A), _ptr(B), _ptr(head),
                                                           _ptr(count), _stream(stream)))
         return {"A": A, "B": B, "head": head, "count": count}
@@ -380,6 +390,8 @@ class QState:
         g = torch.empty((T, K), dtype=torch.float32, device=dev)
         n = torch.empty((T, 2), dtype=torch.int32, device=dev)
         D = torch.empty((T, self.d_k) if self.kind == GLA else (T,), dtype=torch.float32, device=dev)
+        if T == 0:
+            return {"u": u, "w": w, "g": g, "n": n, "D": D}
         _check("qstate_lrb_export", lib().qstate_lrb_export(self._h, _ptr(u), _ptr(w), _ptr(g), _ptr(n),
                                                             _ptr(D), _stream(stream)))
         return {"u": u, "w": w, "g": g, "n": n, "D": D}

@@ -131,6 +131,36 @@ def test_empty_batch_is_noop():
     obj.close()
 
 
+@pytest.mark.parametrize("variant", ["lrb", "lrb_gla", "pw", "rowcol"])
+def test_empty_batch_with_a_variant(variant):
+    """An object of no tiles takes every layout variant; its steps, dequant
+    and exports are no-ops that return empty tensors."""
+    kind = Q.GLA if variant == "lrb_gla" else Q.GDN
+    obj = Q.QState(0, 4, 128, 128, kind, bits=4, group=32, qkv_dtype=Q.BF16,
+                   gate_dtype=Q.F32 if kind == Q.GLA else Q.BF16)
+    if variant.startswith("lrb"):
+        obj.set_lrb(1, 15, 0.5)
+        side = obj.lrb_export()
+    elif variant == "pw":
+        obj.set_pw(8)
+        side = obj.pw_export()
+    else:
+        obj.set_rowcol()
+        side = None
+    x = torch.zeros(16, dtype=torch.bfloat16, device="cuda")
+    g = torch.zeros(16, dtype=torch.float32 if kind == Q.GLA else torch.bfloat16, device="cuda")
+    o = torch.zeros(16, dtype=torch.float32, device="cuda")
+    obj.step(x, x, x, g, o)
+    assert obj.bytes_per_step() == 0 and not o.any()
+    assert obj.dequant().shape == (0, 128, 128)
+    codes, scales, _ = obj.export()
+    assert codes.numel() == 0 and scales.numel() == 0
+    if side is not None:
+        assert all(t.shape[0] == 0 for t in side.values())
+    torch.cuda.synchronize()
+    obj.close()
+
+
 def test_zero_update_gives_zero_state():
     obj = Q.QState(2, 3, 64, 64, Q.RETNET, bits=4, group=64)
     q, k, v, g, out = obj.alloc_inputs()
