@@ -56,6 +56,9 @@ CASES = {
     # GLA (one decay factor per key row): d 128 INT4 g32 persistent, bf16
     # inputs; d 64 INT8 per-token dynamic scales with BDR, fp32 inputs
     "gla_d128_int4g32_k0_m4": (C3.scaled(batch=2, heads=4), 0, 4, 0.5),
+    # the most columns a tile holds (k + m = 32): d 128, GDN with BDR and GLA
+    "gdn_d128_int4_bdr_k0_m32": (C4.scaled(batch=1, heads=2, layers=1, eps_b=0.3), 0, 32, 0.5),
+    "gla_d128_int4g32_k0_m32": (C3.scaled(batch=1, heads=2), 0, 32, 0.5),
     "gla_d64_int8tok_bdr_k0_m3": (C3.scaled(batch=2, heads=4, d_k=64, d_v=64, bits=8, group=0,
                                             scale_modes=(synth.DYNAMIC,), round_mode=synth.BDR,
                                             eps_b=0.3, qkv_dtype=synth.F32), 0, 3, 0.5),
@@ -65,6 +68,7 @@ CASES_K1 = {
     "gdn_d128_int4_bdr_k1_m4": (C4.scaled(batch=2, heads=4, layers=1, eps_b=0.3), 1, 4, 0.5),
     "mamba2_d128_int8tok_k1_m5": (C2.scaled(batch=2, heads=4, d_v=128), 1, 5, 0.5),
     "gla_d128_int4g32_k1_m3": (C3.scaled(batch=2, heads=4), 1, 3, 0.5),
+    "gdn_d128_int4_bdr_k1_m31": (C4.scaled(batch=1, heads=2, layers=1, eps_b=0.3), 1, 31, 0.5),
 }
 
 
