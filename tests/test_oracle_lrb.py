@@ -12,6 +12,10 @@ Low-Bit Recurrent State Quantization" (Abstract, Figure 3, Tables 6, 8, 9).
   quantized step (same codes and scales), with inputs exact in binary16.
 - The merge threshold: merged elements are those of the bypass at least
   eps_L grid steps large, and fewer as eps_L grows.
+- GLA (a decay factor per key row): the row-factor bits of Table 6's GLA
+  row; all gates 1 is RetNet with gamma = 1 bit for bit; a merge every step
+  with exact binary16 inputs is the plain GLA step; before the first merge
+  the bypass is the unquantized GLA recurrence within binary16 rounding.
 """
 import numpy as np
 import pytest
@@ -283,3 +287,51 @@ def test_gla_lrb_tracks_the_unquantized_state_better(orc):
     e_plain = np.linalg.norm(plain.dequant() - S)
     e_lrb = np.linalg.norm(np.stack([lrb.state(t) for t in range(T)]) - S)
     assert e_lrb < 0.8 * e_plain, (e_lrb, e_plain)
+
+
+def test_gla_bypass_before_its_first_merge_is_the_recurrence(orc):
+    """Before its first merge a GLA tile's codes are zero, so the state its
+    bypass stands for is Diag(D_t) sum_l fp16(k_l / D_l) fp16(v_l)^T: the
+    column added at step l, read at step t, is (D_t / D_l) k_l v_l^T with
+    D_t / D_l the product of the gates of steps l+1 .. t.  That is the
+    unquantized GLA recurrence S_t = Diag(alpha_t) S_{t-1} + k_t v_t^T (GLA in
+    Table 1) up to the binary16 rounding of each column (2^-11 relative per
+    side, 2^-25 absolute below the binary16 normal range) and the binary32
+    products that form D.  Checked element by element in fp64 at every step,
+    and the outputs against S_t^T q_t; the decay the pin checks is far larger
+    than its tolerance, so a row factor dropped, applied twice or applied
+    along d_v fails it."""
+    wl = C3.scaled(batch=1, heads=4, d_k=64, d_v=64, group=32,
+                   qkv_dtype=synth.F32, gate_dtype=synth.F32)
+    T, m, dk, dv = 4, 31, 64, 64
+    cfg = oracle.Config(dk, dv, synth.GLA, 32, scale_mode=synth.PERSISTENT)
+    lrb = oracle.LrbState(cfg, [4] * T, k=0, m=m, eps_l=0.5)
+    S = np.zeros((T, dk, dv))
+    S_nodecay = np.zeros((T, dk, dv))
+    A = np.zeros((T, dk, dv))            # the recurrence of |k_l v_l^T|
+    K = np.zeros((T, dk))
+    V = np.zeros((T, dv))
+    for s in range(m - 1):
+        q, k, v, g = _gla_stream(wl, s, T)
+        o = lrb.step(q, k, v, g).astype(np.float64)
+        a = g.astype(np.float64)[:, :, None]
+        kv = k.astype(np.float64)[:, :, None] * v.astype(np.float64)[:, None, :]
+        S = a * S + kv
+        S_nodecay = S_nodecay + kv
+        A = a * A + np.abs(kv)
+        K += np.abs(k)
+        V += np.abs(v)
+        assert not lrb.codes.any() and int(lrb.nnew[0]) == s + 1
+        P = np.stack([lrb.state(t) for t in range(T)])
+        tol = 1.05 * 2.0**-10 * A + 2.0**-24 * (K[:, :, None] + V[:, None, :])
+        assert np.all(np.abs(P - S) <= tol), (s, np.abs(P - S).max())
+        qa = np.abs(q.astype(np.float64))
+        o_ref = np.einsum("tij,ti->tj", S, q.astype(np.float64))
+        tol_o = 2.0**-9 * np.einsum("tij,ti->tj", A, qa) + \
+            2.0**-23 * (V * qa.sum(1)[:, None] + (K * qa).sum(1)[:, None])
+        assert np.all(np.abs(o - o_ref) <= tol_o), (s, np.abs(o - o_ref).max())
+    # the readings the pin tells apart: no decay at all, and a key side held
+    # undivided (every column decayed by the whole D_t)
+    assert np.abs(S_nodecay - S).max() > 100 * tol.max()
+    Dt = lrb.D.astype(np.float64)[:, :, None]
+    assert np.abs(Dt * S_nodecay - S).max() > 100 * tol.max()
