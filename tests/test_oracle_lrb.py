@@ -16,6 +16,9 @@ Low-Bit Recurrent State Quantization" (Abstract, Figure 3, Tables 6, 8, 9).
   row; all gates 1 is RetNet with gamma = 1 bit for bit; a merge every step
   with exact binary16 inputs is the plain GLA step; before the first merge
   the bypass is the unquantized GLA recurrence within binary16 rounding.
+- Before the first merge the bypass is the unquantized recurrence (Mamba2
+  element by element, Gated DeltaNet in Frobenius norm) within the binary16
+  rounding of its columns.
 """
 import numpy as np
 import pytest
@@ -335,3 +338,81 @@ def test_gla_bypass_before_its_first_merge_is_the_recurrence(orc):
     assert np.abs(S_nodecay - S).max() > 100 * tol.max()
     Dt = lrb.D.astype(np.float64)[:, :, None]
     assert np.abs(Dt * S_nodecay - S).max() > 100 * tol.max()
+
+
+@pytest.mark.parametrize("kind", ["mamba2", "gdn"])
+def test_bypass_before_its_first_merge_is_the_recurrence(kind, orc):
+    """Before the first merge the codes are zero and the bypass alone holds
+    the state, so it must follow the unquantized recurrence of Table 1 up to
+    the binary16 rounding of its columns.
+
+    Mamba2 (scalar decay): column l read at step t is g_l fp16(k_l) fp16(v_l)^T
+    with g_l the binary32 product of the gates since step l; checked element
+    by element against S_t = alpha_t S_{t-1} + k_t v_t^T with the same bound
+    as the GLA pin.  Gated DeltaNet: the column is (fp16(beta k), fp16(e)) with
+    e = v - r and r over the bypass itself; with unit keys, alpha <= 1 and
+    beta <= 1 the transition alpha (I - beta k k^T) has norm at most 1, so the
+    rounding of each column adds to the Frobenius distance from
+    S_t = alpha_t S_{t-1} + beta_t k_t (v_t - alpha_t S_{t-1}^T k_t)^T and
+    never grows: ||P_t - S_t||_F <= 1.1 * 2^-10 * sum_l ||beta_l k_l|| ||e_l||
+    plus the binary32 sums.  Outputs are checked against S_t^T q_t."""
+    if kind == "mamba2":
+        wl = C2.scaled(batch=1, heads=4)
+    else:
+        wl = C4.scaled(batch=1, heads=4, layers=1)
+    T, m, dk, dv = 4, 31, wl.d_k, wl.d_v
+    cfg = oracle.Config(dk, dv, wl.kind, wl.group, scale_mode=synth.DYNAMIC,
+                        scale_f32=wl.scale_dtype == synth.F32)
+    lrb = oracle.LrbState(cfg, [wl.bits] * T, k=0, m=m, eps_l=0.5)
+    S = np.zeros((T, dk, dv))
+    S_nodecay = np.zeros((T, dk, dv))
+    A = np.zeros((T, dk, dv))
+    K = np.zeros((T, dk))
+    V = np.zeros((T, dv))
+    budget = np.zeros(T)
+    for s in range(m - 1):
+        x = synth.gen_step(wl, s, tiles=np.arange(T))
+        q, k, v, g = x.as_f32(wl)
+        q64, k64, v64 = (z.astype(np.float64) for z in (q, k, v))
+        if kind == "mamba2":
+            o = lrb.step(q, k, v, g).astype(np.float64)
+            a = g.astype(np.float64)[:, :1, None]
+            kv = k64[:, :, None] * v64[:, None, :]
+            S = a * S + kv
+            A = a * A + np.abs(kv)
+            K += np.abs(k64)
+            V += np.abs(v64)
+        else:
+            alpha, beta = g[:, :1], g[:, 1]
+            o = lrb.step(q, k, v, alpha, beta).astype(np.float64)
+            a = alpha.astype(np.float64)[:, :, None]
+            b = beta.astype(np.float64)
+            e = v64 - np.einsum("tij,ti->tj", a * S, k64)
+            upd = (b[:, None] * k64)[:, :, None] * e[:, None, :]
+            S = a * S + upd
+            budget += np.linalg.norm(b[:, None] * k64, axis=1) * np.linalg.norm(e, axis=1)
+        S_nodecay = S_nodecay + (upd if kind == "gdn" else kv)
+        assert not lrb.codes.any() and int(lrb.nnew[0]) == s + 1
+        P = np.stack([lrb.state(t) for t in range(T)])
+        o_ref = np.einsum("tij,ti->tj", S, q64)
+        qa = np.abs(q64)
+        if kind == "mamba2":
+            tol = 1.05 * 2.0**-10 * A + 2.0**-24 * (K[:, :, None] + V[:, None, :])
+            assert np.all(np.abs(P - S) <= tol), (s, np.abs(P - S).max())
+            tol_o = 2.0**-9 * np.einsum("tij,ti->tj", A, qa) + \
+                2.0**-23 * (V * qa.sum(1)[:, None] + (K * qa).sum(1)[:, None])
+            assert np.all(np.abs(o - o_ref) <= tol_o), (s, np.abs(o - o_ref).max())
+        else:
+            fro = np.linalg.norm((P - S).reshape(T, -1), axis=1)
+            tol = 1.1 * 2.0**-10 * budget + 2.0**-20 * (s + 1)
+            assert np.all(fro <= tol), (s, fro, tol)
+            # |o - S^T q| <= ||P - S||_F ||q|| plus the binary32 sums
+            err_o = np.linalg.norm(o - o_ref, axis=1)
+            assert np.all(err_o <= 1.05 * tol * np.linalg.norm(q64, axis=1) + 2.0**-20), s
+    # the decay the pin resolves is far above its tolerance (for GDN the
+    # tolerance is the worst case of the triangle inequality, about 35 times
+    # the distance the roundings actually leave)
+    if kind == "mamba2":
+        assert np.abs(S_nodecay - S).max() > 100 * tol.max()
+    else:
+        assert np.linalg.norm((S_nodecay - S).reshape(T, -1), axis=1).min() > 50 * tol.max()
