@@ -449,19 +449,32 @@ def run_ours(args, rank, world, local_rank):
     return result
 
 
-def read_traffic(workload, tiles=None, kernel="step_kernel"):
-    """DRAM bytes per launch from the committed ncu summary of this kernel on
-    this workload (profiles/<kernel>_<workload>.md), if its recorded
-    kernel-source hash matches the current sources; scaled from the
-    summary's full-size launch to `tiles` tiles when given."""
+def source_digest(src):
+    """First 16 hex digits of a sha256 over the kernel sources in `src` as
+    code: in file-name order, each file's name and its text with comments
+    removed and whitespace runs collapsed (string and character literals
+    kept).  The committed ncu counters are tied to the code they were taken
+    on, so an edit of a comment leaves them valid and any other edit does not."""
     import hashlib
-    src = os.path.join(ROOT, "bit_recurrent_state_decode_b200", "csrc")
+    import re
+    token = re.compile(r'//[^\n]*|/\*.*?\*/|"(?:\\.|[^"\\\n])*"|\'(?:\\.|[^\'\\\n])*\'', re.S)
     h = hashlib.sha256()
     for f in sorted(os.listdir(src)):
         if f.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(src, f), "rb") as fh:
-                h.update(fh.read())
-    digest = h.hexdigest()[:16]
+            with open(os.path.join(src, f), encoding="utf-8", errors="surrogateescape") as fh:
+                text = fh.read()
+            code = token.sub(lambda m: " " if m.group(0)[0] == "/" else m.group(0), text)
+            h.update(f.encode() + b"\0" + " ".join(code.split()).encode("utf-8", "surrogateescape")
+                     + b"\0")
+    return h.hexdigest()[:16]
+
+
+def read_traffic(workload, tiles=None, kernel="step_kernel"):
+    """DRAM bytes per launch from the committed ncu summary of this kernel on
+    this workload (profiles/<kernel>_<workload>.md), if its recorded
+    kernel-source digest (source_digest) matches the current sources; scaled
+    from the summary's full-size launch to `tiles` tiles when given."""
+    digest = source_digest(os.path.join(ROOT, "bit_recurrent_state_decode_b200", "csrc"))
     path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
     if not os.path.exists(path):
         return None

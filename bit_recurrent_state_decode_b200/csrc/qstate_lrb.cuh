@@ -1,7 +1,7 @@
 // qstate_lrb.cuh -- the decode step with a Low-Rank Bypass (LRB) of
 // "Preserving Updates in Low-Bit Recurrent State Quantization" (Abstract,
 // Figure 3, Tables 6, 8, 9), for uniform 4- or 8-bit states of RetNet,
-// Mamba2 and Gated DeltaNet tiles with d_k = d_v.
+// Mamba2, GLA and Gated DeltaNet tiles with d_k = d_v.
 //
 // A tile's state is D * S_hat + P: the quantized part S_hat (codes, scales)
 // times the decay D accumulated since the last merge, plus the bypass
@@ -14,7 +14,10 @@
 // grid steps of the decayed grid large are merged: x = a + P there, x = a
 // elsewhere, requantized with the object's scale and rounding rules (BDR with
 // d = x - a), D reset to 1, and the unmerged rest kept as its leading
-// singular pair (k = 1, by power iteration) or dropped (k = 0).
+// singular pair (k = 1, by power iteration) or dropped (k = 0).  GLA's decay
+// Diag(alpha) keeps one D per key row instead: the coefficients do not
+// decay, a column's key side is stored divided by the D of its step and read
+// as D_i u_i, and the tile stands for Diag(D) (S_hat + P).
 //
 // Arithmetic and order follow the specification of the bypass (canonical
 // sums; each column in slot order as one fma per element); every result is

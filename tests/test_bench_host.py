@@ -32,11 +32,7 @@ def _fake_root(tmp_path, profile_hash, value="123456"):
     (csrc / "a.cuh").write_bytes(b"kernel source A")
     (csrc / "b.cu").write_bytes(b"kernel source B")
     (csrc / "notes.txt").write_bytes(b"not hashed")
-    h = hashlib.sha256()
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh", ".h")):
-            h.update((csrc / f).read_bytes())
-    digest = h.hexdigest()[:16]
+    digest = bench.source_digest(str(csrc))
     prof = tmp_path / "profiles"
     prof.mkdir()
     (prof / "step_kernel_w.md").write_text(
@@ -78,3 +74,27 @@ def test_committed_profiles_name_their_kernel_and_command():
         assert f.split("_kernel_")[0] in ("step", "rows", "lrb", "pw", "rc"), f
         assert "source_sha256_16:" in text and "dram_bytes_per_launch_full_size:" in text
         assert "ncu " in text and "--clock-control none" in text and "python bench.py" in text
+
+
+def test_source_digest_is_of_the_code(tmp_path):
+    """Comments and whitespace do not change the digest that ties a profile
+    to the kernel sources; code, a file name, or a // inside a string
+    literal does."""
+    d = tmp_path / "csrc"
+    d.mkdir()
+    f = d / "k.cuh"
+
+    def digest(text, name="k.cuh"):
+        for p in d.iterdir():
+            p.unlink()
+        (d / name).write_text(text)
+        return bench.source_digest(str(d))
+
+    base = digest('int x = 1;  // the count\nconst char* s = "a//b"; /* it\'s */ char c = \'/\';\n')
+    assert digest('int x = 1;\n\n   const char* s = "a//b";\nchar c = \'/\'; // other words\n') == base
+    assert digest('int x = 2; const char* s = "a//b"; char c = \'/\';') != base
+    assert digest('int x = 1; const char* s = "a/ /b"; char c = \'/\';') != base
+    assert digest('int x = 1; const char* s = "a//b"; char c = \'/\';', name="j.cuh") != base
+    assert digest('int x = 1; const char* s = "a//b"; char c = \'/\';') == base
+    (d / "notes.txt").write_text("not a source")
+    assert bench.source_digest(str(d)) == base
