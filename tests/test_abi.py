@@ -104,6 +104,16 @@ def test_null_object_calls(q):
     assert lib.qstate_debug_set(None, -1, 1) == q.EINVAL
     assert lib.qstate_set_taxonomy(None, 1) == q.EINVAL
     assert lib.qstate_destroy(None) == q.EINVAL
+    # the layout variants, their side state and the host pipeline
+    assert lib.qstate_set_lrb(None, 1, 15, 0.5) == q.EINVAL
+    assert lib.qstate_lrb_export(None, None, None, None, None, None, None) == q.EINVAL
+    assert lib.qstate_set_pw(None, 8) == q.EINVAL
+    assert lib.qstate_pw_export(None, None, None, None, None, None) == q.EINVAL
+    assert lib.qstate_set_rowcol(None) == q.EINVAL
+    assert lib.qstate_error_rows(None, None, None) == q.EINVAL
+    assert lib.qstate_step_host_pipelined(None, None, None, None, None, None, None) == q.EINVAL
+    assert lib.qstate_step_host_sync(None, None) == q.EINVAL
+    assert lib.qstate_kernel(None) == b""
 
 
 def test_product_never_imports_oracle():
