@@ -361,9 +361,10 @@ def lrb_bits(bits: int, group: int, d_k: int, d_v: int, cols_used: float,
 
 
 class LrbState(State):
-    """A quantized state with a Low-Rank Bypass (readings L1-L6 of the C
+    """A quantized state with a Low-Rank Bypass (readings L1-L7 of the C
     code): codes and scales as State, plus per tile u [k+m][d_k] and
-    w [k+m][d_v] (binary16 patterns), g [k+m] and the slot counts."""
+    w [k+m][d_v] (binary16 patterns), g [k+m], the slot counts and the decay
+    D since the last merge (GLA: one factor per key row, [d_k])."""
 
     def __init__(self, cfg: Config, tile_bits, k: int, m: int, eps_l: float,
                  keep_resid: bool = False):

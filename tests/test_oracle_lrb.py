@@ -19,6 +19,8 @@ Low-Bit Recurrent State Quantization" (Abstract, Figure 3, Tables 6, 8, 9).
 - Before the first merge the bypass is the unquantized recurrence (Mamba2
   element by element, Gated DeltaNet in Frobenius norm) within the binary16
   rounding of its columns.
+- At a GLA merge the elements that leave are those at least eps_L grid
+  steps of their own row's decayed grid (D_i * Delta) large.
 """
 import numpy as np
 import pytest
@@ -416,3 +418,55 @@ def test_bypass_before_its_first_merge_is_the_recurrence(kind, orc):
         assert np.abs(S_nodecay - S).max() > 100 * tol.max()
     else:
         assert np.linalg.norm((S_nodecay - S).reshape(T, -1), axis=1).min() > 50 * tol.max()
+
+
+def test_gla_merge_threshold_uses_each_rows_factor(orc):
+    """At a merge the elements that leave a GLA bypass are those with
+    |P_ij| >= eps_L * (D_i * Delta_ij), D_i the row's decay factor of that
+    step (reading L7).  The test forms P itself from the bypass the oracle
+    held before the merge step (columns read as D_i u_i, the new column
+    fp16(k / D) and fp16(v)) and checks which elements the oracle kept as its
+    residual, away from a thin band around the threshold where the fp32 and
+    fp64 sums may round to opposite sides.  Gates spread over [1/2, 1] make
+    the row factors differ by far more than that band, so a threshold
+    without D_i, or with one factor for the whole tile, selects other
+    elements."""
+    wl = C3.scaled(batch=1, heads=4, d_k=64, d_v=64, group=32,
+                   qkv_dtype=synth.F32, gate_dtype=synth.F32)
+    T, m, eps = 4, 6, 0.5
+    cfg = oracle.Config(64, 64, synth.GLA, 32, scale_mode=synth.PERSISTENT)
+    st = oracle.LrbState(cfg, [4] * T, k=1, m=m, eps_l=eps, keep_resid=True)
+    rng = np.random.default_rng(7)
+    spread = lambda s, shape: rng.uniform(0.5, 1.0, shape).astype(np.float32)
+    for s in range(2 * m - 1):
+        st.step(*_gla_stream(wl, s, T, spread))
+    assert np.all(st.nnew == m - 1)
+    u0, w0, g0 = st.u.copy(), st.w.copy(), st.g.copy()
+    D0, scales0, n0 = st.D.copy(), st.scales.copy(), (st.nres + st.nnew).copy()
+    q, k, v, g = _gla_stream(wl, 2 * m - 1, T, spread)
+    st.step(q, k, v, g)
+    assert np.all(st.nnew == 0)                      # this step merged
+    agree = differs = differs_tile = 0
+    for t in range(T):
+        Dn = g[t] * D0[t]                            # binary32, as the step forms it
+        n = int(n0[t])
+        U = u0[t, :n].view(np.float16).astype(np.float32) * Dn[None, :]
+        u_new = (k[t] / Dn).astype(np.float16).astype(np.float32) * Dn
+        Wc = w0[t, :n].view(np.float16).astype(np.float64)
+        w_new = v[t].astype(np.float16).astype(np.float64)
+        P = np.einsum("l,li,lj->ij", g0[t, :n].astype(np.float64), U.astype(np.float64), Wc) + \
+            np.outer(u_new.astype(np.float64), w_new)
+        delta = np.repeat(scales0[t].reshape(64, 2), 32, axis=1).astype(np.float64)
+        thr = eps * (Dn.astype(np.float64)[:, None] * delta)
+        far = (np.abs(np.abs(P) - thr) > 1e-4 * thr) & (P != 0)
+        merged = st.resid[t] == 0
+        want = np.abs(P) >= thr
+        assert np.array_equal(merged[far], want[far]), t
+        band = int(((~far) & (P != 0)).sum())
+        assert abs(int(st.merged[t]) - int(want.sum())) <= band, t
+        agree += int(far.sum())
+        alt = np.abs(P) >= eps * delta                             # no D_i
+        alt_tile = np.abs(P) >= eps * (float(Dn.mean()) * delta)  # one factor per tile
+        differs += int((alt[far] != want[far]).sum())
+        differs_tile += int((alt_tile[far] != want[far]).sum())
+    assert agree > 0.95 * T * 64 * 64 and differs > 100 and differs_tile > 10
