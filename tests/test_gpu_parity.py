@@ -78,21 +78,39 @@ def test_gdn_teacher_forced():
 
 
 # ------------------------------------------------------------ full sizes, sampled tiles
+def _bench_layers(wl):
+    """The layers the benchmark steps in one launch: the workload's own, or,
+    for a one-layer state that fits in L2, as many independent replicas of
+    the layer as take state and inputs past 4x L2 (bench.pick_replicas on
+    the same per-layer byte count)."""
+    import bench
+    probe = gpu_object(wl, wl.scale_modes[0], wl.batch, 1)
+    z = probe.sizes
+    resident = z["code_bytes"] + z["scale_bytes"] + z["ref_bytes"]
+    per_layer = resident + probe.bytes_per_step() - 2 * resident
+    probe.close()
+    l2 = torch.cuda.get_device_properties(0).L2_cache_size
+    return wl.layers * bench.pick_replicas(wl, l2, per_layer)
+
+
 @pytest.mark.parametrize("name,steps", [("mamba2", 3), ("gla", 3), ("gdn", 2), ("mixed", 3)])
 def test_full_size_sampled_tiles(name, steps):
     """The full-size object in the launch configuration the benchmark times
-    (one launch over every tile of every layer); the oracle steps 48 sampled
-    tiles from the same zero state with the same inputs."""
+    (one launch over every tile of every layer, the layer replicas of the
+    L2-sized configurations included); the oracle steps 48 sampled tiles
+    from the same zero state with the same inputs."""
     wl = {"mamba2": C2, "gla": C3, "gdn": C4, "mixed": C5}[name]
+    layers = _bench_layers(wl)
+    assert layers > 1
     rng = np.random.default_rng(7)
-    T = wl.tiles_per_layer * wl.layers
+    T = wl.tiles_per_layer * layers
     sample = np.unique(np.concatenate([[0, T - 1], rng.integers(0, T, 46)]))
     heads = sample % wl.heads
     for mode in wl.scale_modes:
-        gpu = gpu_object(wl, mode, wl.batch, wl.layers)
+        gpu = gpu_object(wl, mode, wl.batch, layers)
         orc = oracle_state(wl, mode, heads)
         for step in range(steps):
-            x = concat_inputs([synth.gen_step(wl, step, layer=l) for l in range(wl.layers)])
+            x = concat_inputs([synth.gen_step(wl, step, layer=l) for l in range(layers)])
             qd, kd, vd, gd = gpu_inputs(wl, x)
             out = torch.empty((T, wl.d_v), dtype=torch.float32, device="cuda")
             gpu.step(qd, kd, vd, gd, out)
