@@ -37,6 +37,28 @@ def gpu_object(wl: synth.Workload, mode: int, batch: int, layers: int) -> Q.QSta
                     scale_dtype=wl.scale_dtype, head_bits=hb, rotation=wl.rotation)
 
 
+def bench_layers(wl: synth.Workload) -> int:
+    """The layers the benchmark steps in one launch: the workload's own, or,
+    for a one-layer state that fits in L2, as many independent replicas of
+    the layer as take state and inputs past 4x L2 (bench.pick_replicas on
+    the per-layer byte count bench.py forms, layout variant included)."""
+    import bench
+    import torch
+    probe = gpu_object(wl, wl.scale_modes[0], wl.batch, 1)
+    if wl.lrb:
+        probe.set_lrb(*wl.lrb)
+    if wl.pw:
+        probe.set_pw(wl.pw)
+    if wl.rowcol:
+        probe.set_rowcol()
+    z = probe.sizes
+    resident = z["code_bytes"] + z["scale_bytes"] + z["ref_bytes"]
+    per_layer = resident + probe.bytes_per_step() - 2 * resident
+    probe.close()
+    l2 = torch.cuda.get_device_properties(0).L2_cache_size
+    return wl.layers * bench.pick_replicas(wl, l2, per_layer)
+
+
 def oracle_state(wl: synth.Workload, mode: int, tile_heads: np.ndarray, bits=None):
     cfg = oracle.Config(wl.d_k, wl.d_v, wl.kind, wl.group, scale_mode=mode,
                         round_mode=wl.round_mode, scale_f32=wl.scale_dtype == synth.F32,

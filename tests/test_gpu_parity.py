@@ -15,7 +15,7 @@ import oracle
 from bit_recurrent_state_decode_b200 import qstate as Q
 from bit_recurrent_state_decode_b200 import synth
 
-from parity_util import (GpuView, compare, concat_inputs, gpu_inputs, gpu_object,
+from parity_util import (GpuView, bench_layers, compare, concat_inputs, gpu_inputs, gpu_object,
                          import_oracle_state, oracle_inputs, oracle_state, rel_err, run_pair)
 
 pytestmark = pytest.mark.gpu
@@ -78,21 +78,6 @@ def test_gdn_teacher_forced():
 
 
 # ------------------------------------------------------------ full sizes, sampled tiles
-def _bench_layers(wl):
-    """The layers the benchmark steps in one launch: the workload's own, or,
-    for a one-layer state that fits in L2, as many independent replicas of
-    the layer as take state and inputs past 4x L2 (bench.pick_replicas on
-    the same per-layer byte count)."""
-    import bench
-    probe = gpu_object(wl, wl.scale_modes[0], wl.batch, 1)
-    z = probe.sizes
-    resident = z["code_bytes"] + z["scale_bytes"] + z["ref_bytes"]
-    per_layer = resident + probe.bytes_per_step() - 2 * resident
-    probe.close()
-    l2 = torch.cuda.get_device_properties(0).L2_cache_size
-    return wl.layers * bench.pick_replicas(wl, l2, per_layer)
-
-
 @pytest.mark.parametrize("name,steps", [("mamba2", 3), ("gla", 3), ("gdn", 2), ("mixed", 3)])
 def test_full_size_sampled_tiles(name, steps):
     """The full-size object in the launch configuration the benchmark times
@@ -100,7 +85,7 @@ def test_full_size_sampled_tiles(name, steps):
     L2-sized configurations included); the oracle steps 48 sampled tiles
     from the same zero state with the same inputs."""
     wl = {"mamba2": C2, "gla": C3, "gdn": C4, "mixed": C5}[name]
-    layers = _bench_layers(wl)
+    layers = bench_layers(wl)
     assert layers > 1
     rng = np.random.default_rng(7)
     T = wl.tiles_per_layer * layers

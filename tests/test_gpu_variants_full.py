@@ -7,8 +7,8 @@ the sampled tiles' outputs, codes, scales and side state are compared.
 - INT4+Had and key-row x value-column scales: bit-exact after 3 steps.
 - PW-S8: bit-exact after 10 steps (the window full, two pairs merged).
 - LRB+BDR (k = 1, m = 15), and the same bypass on the GLA decode (a decay
-  factor per key row; 24 layer replicas of B128 H16, 49 152 tiles, as the
-  benchmark steps that L2-sized layer): bit-exact through the first merge and
+  factor per key row; as many replicas of the L2-sized B128 H16 layer as
+  the benchmark steps, 32 x 2 048 tiles on B200): bit-exact through the first merge and
   up to the second; at the second merge outputs, codes, scales and counts
   are still bit-exact and the kept rank-1 residual is within the tolerance
   of the small-case test of its optimum (the oracle's truncated SVD).
@@ -20,8 +20,8 @@ import torch
 import oracle
 from bit_recurrent_state_decode_b200 import synth
 
-from parity_util import (GpuView, compare, concat_inputs, gpu_inputs, gpu_object, oracle_inputs,
-                         oracle_state)
+from parity_util import (GpuView, bench_layers, compare, concat_inputs, gpu_inputs, gpu_object,
+                         oracle_inputs, oracle_state)
 
 pytestmark = pytest.mark.gpu
 THREADS = 16
@@ -95,10 +95,11 @@ def test_full_size_sampled_pw():
     gpu.close()
 
 
-@pytest.mark.parametrize("name,layers", [("gdn_l24_b256_h32_d128_int4g32_lrb", 24),
-                                         ("gla_b128_h16_d128_int4g32_lrb", 24)])
-def test_full_size_sampled_lrb(name, layers):
-    wl = synth.workload(name).scaled(layers=layers)
+@pytest.mark.parametrize("name", ["gdn_l24_b256_h32_d128_int4g32_lrb",
+                                  "gla_b128_h16_d128_int4g32_lrb"])
+def test_full_size_sampled_lrb(name):
+    wl = synth.workload(name)
+    wl = wl.scaled(layers=bench_layers(wl))
     k, m, eps_l = wl.lrb
     sample, T = _sample(wl)
     mode = wl.scale_modes[0]
