@@ -67,3 +67,27 @@ def test_c_client_builds_links_and_runs(tmp_path, lang):
                    check=True, capture_output=True, text=True)
     r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
     assert r.returncode == 0 and "c client ok" in r.stdout, (r.returncode, r.stdout, r.stderr)
+
+
+def test_readme_c_example_compiles(tmp_path):
+    """The C example in README.md, placed in a function whose parameters are
+    the buffers it names, compiles against the header as C99 with every
+    warning an error (its field names and calls are the header's)."""
+    cc = shutil.which("gcc")
+    if cc is None:
+        pytest.skip("no host compiler")
+    text = open(os.path.join(ROOT, "README.md")).read()
+    start = text.index("```c\n") + len("```c\n")
+    body = text[start:text.index("```", start)]
+    lines = [l for l in body.splitlines() if not l.startswith("#include")]
+    src = tmp_path / "readme_example.c"
+    src.write_text(
+        "#include <stdio.h>\n#include \"qstate.h\"\n"
+        "void example(const void* q, const void* k, const void* v, const void* gates, float* out,\n"
+        "             float* S_hat, qstate_stream stream) {\n"
+        + "\n".join("    " + l for l in lines) + "\n    (void)rc;\n}\n"
+        "int main(void) { return 0; }\n")
+    r = subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-I",
+                        os.path.join(ROOT, "include"), "-c", str(src), "-o",
+                        str(tmp_path / "readme_example.o")], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
