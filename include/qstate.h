@@ -186,7 +186,9 @@ int qstate_reset(qstate* s, qstate_stream stream);
  * Quantization"), o_t = S_t^T q_t, then the scale, rounding and repacking of
  * the state in the order given at the top of this file.
  * q, k, v, gates, out: caller-owned DEVICE buffers in the layouts above
- * (gates may be NULL for RetNet).  Returns after the launch. */
+ * (gates may be NULL for RetNet), each starting on a 16-byte boundary;
+ * QSTATE_EINVAL for a NULL or misaligned one, also for an object of no
+ * tiles, whose step then does nothing.  Returns after the launch. */
 int qstate_step(qstate* s, const void* q, const void* k, const void* v, const void* gates,
                 float* out, qstate_stream stream);
 
