@@ -43,7 +43,6 @@ def bench_layers(wl: synth.Workload) -> int:
     the layer as take state and inputs past 4x L2 (bench.pick_replicas on
     the per-layer byte count bench.py forms, layout variant included)."""
     import bench
-    import torch
     probe = gpu_object(wl, wl.scale_modes[0], wl.batch, 1)
     if wl.lrb:
         probe.set_lrb(*wl.lrb)
