@@ -324,9 +324,9 @@ int qstate_error_rows(const qstate* s, float* out, qstate_stream stream);
  * side is stored as fp16(k / D) of its step and read as D_i u_i, and the
  * tile stands for Diag(D) (dequant(codes) + sum_l g_l u_l w_l^T).
  * k in {0, 1}, m >= 1, k + m <= 32, eps_l >= 0.  Supported for all four
- * kinds with one code width of 4 or 8 bits,
- * d_k = d_v in {64, 128}, dynamic or persistent scales, no rotation
- * (QSTATE_EUNSUPPORTED otherwise); allocates the bypass (QSTATE_ENOMEM).
+ * kinds with one code width of 4 or 8 bits, d_k = d_v in {64, 128},
+ * dynamic or persistent scales, no rotation (QSTATE_EUNSUPPORTED
+ * otherwise); allocates the bypass (QSTATE_ENOMEM).
  * QSTATE_EINVAL if a bypass, a window or row x column scales are already set
  * or for invalid k, m, eps_l. */
 int qstate_set_lrb(qstate* s, int k, int m, float eps_l);
